@@ -1,0 +1,165 @@
+/*
+ * pagedkv.h — C ABI of the B200 (sm_100a) paged KV-cache library.
+ *
+ * Two operations on a paged KV cache, as described in "vLLM 推理引擎源码级拆解：
+ * PagedAttention 显存虚拟化、Continuous Batching 调度与量化落地全指南"
+ * (chenxutan.com/d/5333):
+ *   - paged_kv_append: each new token's K/V row is written into the slot the
+ *     caller assigned it in a shared pool of fixed-size blocks (§2.1-§2.2: the
+ *     token fills the last block's next slot, or the first slot of a block just
+ *     taken from the free pool);
+ *   - paged_attention_decode: one query token per sequence attends over that
+ *     sequence's cached tokens, walking its block table from logical to
+ *     physical block (§2.3), with grouped-query heads (GQA/MQA, §2.3), blocks
+ *     shared between sequences (§2.1), an optional split of long sequences into
+ *     partitions merged by log-sum-exp, and an FP8-E4M3 cache with per-tensor
+ *     scales ("vLLM 0.5 深度拆解", chenxutan.com/d/4924, §4.2).
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, C-contiguous,
+ *     and 16-byte aligned. The library allocates nothing and keeps no state
+ *     between calls.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls only
+ *     enqueue work and return; they never synchronise and never read device
+ *     memory on the host.
+ *   - Arguments are checked on the host before anything is enqueued; a negative
+ *     pkv_status is returned and nothing runs. PKV_ERR_CUDA reports a launch
+ *     failure; faults inside a kernel surface at the caller's next
+ *     synchronisation, as with any CUDA call.
+ *   - Pool layout: k_cache and v_cache are [num_blocks, block_size,
+ *     num_kv_heads, head_dim] in cache_dtype. Token t of sequence i lives in
+ *     physical block block_table[i][t / block_size] at offset t % block_size;
+ *     its flat slot is physical_block * block_size + offset.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element types. PKV_FP8_E4M3 is the OCP E4M3 format: bias 7, 3 mantissa bits,
+ * subnormals, largest finite 448, no infinities, S.1111.111 = NaN. */
+typedef enum {
+  PKV_F32 = 0,
+  PKV_F16 = 1,
+  PKV_BF16 = 2,
+  PKV_FP8_E4M3 = 3
+} pkv_dtype;
+
+typedef enum {
+  PKV_OK = 0,
+  PKV_ERR_NULL = -1,        /* a required pointer is NULL */
+  PKV_ERR_SHAPE = -2,       /* a size is out of range or inconsistent */
+  PKV_ERR_DTYPE = -3,       /* an unknown dtype or an unsupported dtype pair */
+  PKV_ERR_UNSUPPORTED = -4, /* head_dim or block_size outside the supported set */
+  PKV_ERR_WORKSPACE = -5,   /* workspace missing or smaller than required */
+  PKV_ERR_CUDA = -6,        /* a CUDA runtime call or kernel launch failed */
+  PKV_ERR_ALIGN = -7        /* a pointer is not 16-byte aligned */
+} pkv_status;
+
+/* Flags for paged_attention_decode. */
+#define PKV_DECODE_FORCE_SIMT 1u  /* use the CUDA-core kernel even where the
+                                     tensor-core kernel applies */
+
+/*
+ * paged_kv_append — write new tokens' K/V into their slots ("reshape and cache").
+ *
+ *   key, value    [num_tokens, num_kv_heads, head_dim], src_dtype (F32/F16/BF16)
+ *   k_cache,
+ *   v_cache       [num_blocks, block_size, num_kv_heads, head_dim], cache_dtype;
+ *                 cache_dtype is src_dtype (bytes are copied) or PKV_FP8_E4M3
+ *   slot_mapping  [num_tokens] int64, device: flat slot of each token. A slot
+ *                 < 0 (padding) or >= num_blocks * block_size writes nothing.
+ *   k_scale,
+ *   v_scale       device fp32 scalars, read only for an FP8 cache: the stored
+ *                 code is E4M3(x / scale), x widened to fp32, the division in
+ *                 IEEE fp32, rounded to nearest-even, saturated to +-448.
+ *
+ * Slots within one call must be distinct, and must belong to blocks no other
+ * sequence shares (copy-on-write of shared blocks is the caller's job). Every
+ * other byte of the pool is left untouched.
+ * Requirements: num_tokens >= 0, num_kv_heads > 0, head_dim a positive
+ * multiple of 8, block_size > 0, num_blocks > 0.
+ */
+int paged_kv_append(const void* key, const void* value, void* k_cache, void* v_cache,
+                    const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                    int head_dim, int block_size, int64_t num_blocks, int src_dtype,
+                    int cache_dtype, const float* k_scale, const float* v_scale,
+                    void* stream);
+
+/*
+ * Bytes of workspace paged_attention_decode needs for these sizes: zero when
+ * partition_size is 0 (no split); otherwise room for one fp32 partial output
+ * row, one log-sum-exp value and one int32 link per (sequence, query head,
+ * partition), partitions = ceil(max_seq_len / partition_size).
+ * Returns 0 for invalid sizes.
+ */
+size_t paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
+                                      int head_dim, int max_seq_len, int partition_size);
+
+/*
+ * paged_attention_decode — one-token attention per sequence over a paged cache.
+ *
+ * For sequence i and query head j (KV head h = j / (num_heads / num_kv_heads)):
+ *   K[t] = k_cache[block_table[i][t / block_size], t % block_size, h, :]
+ *          (times *k_scale for an FP8 cache), t = 0 .. seq_lens[i]-1; V alike
+ *   s_t  = scale * <query[i, j, :], K[t]>
+ *   out[i, j, :] = sum_t softmax(s)_t V[t]
+ *
+ *   out          [num_seqs, num_heads, head_dim], q_dtype; written for every
+ *                (i, j); a sequence of length 0 gets zeros
+ *   query        [num_seqs, num_heads, head_dim], q_dtype (F32/F16/BF16)
+ *   k_cache,
+ *   v_cache      pool as above, cache_dtype = q_dtype or PKV_FP8_E4M3
+ *   block_table  [num_seqs, max_blocks_per_seq] int32, device. Entries past a
+ *                sequence's last block are never read. An entry outside
+ *                [0, num_blocks) reads as a block of zeros.
+ *   seq_lens     [num_seqs] int32, device: tokens per sequence, including the
+ *                token appended this step. Values are clamped to
+ *                [0, min(max_seq_len, max_blocks_per_seq * block_size)].
+ *   max_seq_len  host upper bound on seq_lens (sizes the split and workspace)
+ *   scale        softmax scale (usually 1/sqrt(head_dim))
+ *   k_scale,
+ *   v_scale      device fp32 scalars, read only for an FP8 cache
+ *   partition_size  0: a sequence is never split. > 0 (a multiple of
+ *                block_size): a sequence may be split at multiples of this many
+ *                tokens; each piece yields a partial (output, log-sum-exp) in the
+ *                workspace, and a second kernel merges the pieces by
+ *                log-sum-exp. The split points are chosen on the device to
+ *                balance work across the GPU.
+ *   max_ctas     0: one resident wave of CTAs; > 0: at most this many CTAs (a
+ *                tuning and testing knob)
+ *   flags        PKV_DECODE_* bits
+ *   workspace    device scratch of at least paged_attention_workspace_size()
+ *                bytes (may be NULL when that is 0); the caller owns it, need not
+ *                initialise it, and must not use it concurrently for another call
+ *
+ * Requirements: num_seqs >= 0, num_heads > 0, num_kv_heads > 0,
+ * num_heads % num_kv_heads == 0, head_dim in {64, 128}, block_size in
+ * {8, 16, 32}, max_blocks_per_seq > 0, num_blocks > 0, max_seq_len >= 0.
+ */
+int paged_attention_decode(void* out, const void* query, const void* k_cache,
+                           const void* v_cache, const int32_t* block_table,
+                           const int32_t* seq_lens, int num_seqs, int num_heads,
+                           int num_kv_heads, int head_dim, int block_size,
+                           int max_blocks_per_seq, int64_t num_blocks, int max_seq_len,
+                           float scale, int q_dtype, int cache_dtype, const float* k_scale,
+                           const float* v_scale, int partition_size, int max_ctas,
+                           unsigned flags, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/* Static, NUL-terminated description of a pkv_status value. */
+const char* pkv_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int pkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

@@ -1,1 +1,136 @@
-"""B200-native paged KV append and PagedAttention decode."""
+"""B200-native paged KV append and PagedAttention decode.
+
+A thin ctypes binding over ``libpagedkv.so`` (C ABI in include/pagedkv.h). It
+only marshals arguments: every step of the path runs in the library's CUDA
+kernels. PyTorch tensors supply device memory and the current CUDA stream.
+There is no fallback: if the library is missing, every call raises.
+
+Build the library with ``python -m paged_kv_cache_367_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["paged_kv_append", "paged_attention_decode", "paged_attention_workspace_size",
+           "pkv_status_string", "pkv_version", "load_library", "PagedKVError",
+           "PKV_F32", "PKV_F16", "PKV_BF16", "PKV_FP8_E4M3", "PKV_DECODE_FORCE_SIMT",
+           "LIB_PATH", "EXPORTED_SYMBOLS"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedkv.so")
+
+PKV_F32, PKV_F16, PKV_BF16, PKV_FP8_E4M3 = 0, 1, 2, 3
+PKV_DECODE_FORCE_SIMT = 1
+
+EXPORTED_SYMBOLS = ("paged_kv_append", "paged_attention_workspace_size",
+                    "paged_attention_decode", "pkv_status_string", "pkv_version")
+
+_DTYPE_CODES = {torch.float32: PKV_F32, torch.float16: PKV_F16, torch.bfloat16: PKV_BF16,
+                torch.uint8: PKV_FP8_E4M3, torch.float8_e4m3fn: PKV_FP8_E4M3}
+
+_lib = None
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: status {status} ({pkv_status_string(status)})")
+        self.status = status
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libpagedkv.so once; raise if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
+                          "`python -m paged_kv_cache_367_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, I64, F, U, SZ = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
+                           ctypes.c_uint, ctypes.c_size_t)
+    lib.paged_kv_append.argtypes = [P, P, P, P, P, I, I, I, I, I64, I, I, P, P, P]
+    lib.paged_kv_append.restype = I
+    lib.paged_attention_workspace_size.argtypes = [I, I, I, I, I, I]
+    lib.paged_attention_workspace_size.restype = SZ
+    lib.paged_attention_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I64, I, F, I, I,
+                                           P, P, I, I, U, P, SZ, P]
+    lib.paged_attention_decode.restype = I
+    lib.pkv_status_string.argtypes = [I]
+    lib.pkv_status_string.restype = ctypes.c_char_p
+    lib.pkv_version.argtypes = []
+    lib.pkv_version.restype = I
+    _lib = lib
+    return lib
+
+
+def pkv_status_string(status: int) -> str:
+    return load_library().pkv_status_string(int(status)).decode()
+
+
+def pkv_version() -> int:
+    return load_library().pkv_version()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    try:
+        return _DTYPE_CODES[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype}") from None
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def paged_kv_append(key, value, k_cache, v_cache, slot_mapping, *, k_scale=None, v_scale=None,
+                    stream=None) -> None:
+    """Write key/value [T, Hkv, D] into the pool [num_blocks, bs, Hkv, D] at
+    slot_mapping [T] (int64); see paged_kv_append in include/pagedkv.h."""
+    lib = load_library()
+    T, Hkv, D = key.shape
+    nb, bs = k_cache.shape[0], k_cache.shape[1]
+    st = lib.paged_kv_append(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
+                             _ptr(slot_mapping), T, Hkv, D, bs, nb, _dtype_code(key),
+                             _dtype_code(k_cache), _ptr(k_scale), _ptr(v_scale), _stream(stream))
+    if st != 0:
+        raise PagedKVError("paged_kv_append", st)
+
+
+def paged_attention_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_seq_len,
+                                   partition_size) -> int:
+    return load_library().paged_attention_workspace_size(num_seqs, num_heads, num_kv_heads,
+                                                         head_dim, max_seq_len, partition_size)
+
+
+def paged_attention_decode(out, query, k_cache, v_cache, block_table, seq_lens, *, max_seq_len,
+                           scale, partition_size=0, workspace=None, k_scale=None, v_scale=None,
+                           max_ctas=0, flags=0, stream=None) -> None:
+    """out[i, j] = softmax attention of query[i, j] over sequence i's paged K/V;
+    see paged_attention_decode in include/pagedkv.h."""
+    lib = load_library()
+    S, Hq, D = query.shape
+    nb, bs, Hkv, _ = k_cache.shape
+    mbps = block_table.shape[1]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.paged_attention_decode(_ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache),
+                                    _ptr(block_table), _ptr(seq_lens), S, Hq, Hkv, D, bs, mbps,
+                                    nb, int(max_seq_len), float(scale), _dtype_code(query),
+                                    _dtype_code(k_cache), _ptr(k_scale), _ptr(v_scale),
+                                    int(partition_size), int(max_ctas), int(flags),
+                                    _ptr(workspace), ws_bytes, _stream(stream))
+    if st != 0:
+        raise PagedKVError("paged_attention_decode", st)

@@ -1,0 +1,128 @@
+"""The C ABI library loads without a GPU, exports every function include/pagedkv.h
+declares, and rejects bad arguments on the host (nothing is enqueued, so these
+run on a machine without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "pagedkv.h")
+
+OK, ENULL, ESHAPE, EDTYPE, EUNSUP, EWS, ECUDA, EALIGN = 0, -1, -2, -3, -4, -5, -6, -7
+F32, F16, BF16, FP8 = 0, 1, 2, 3
+A = 1 << 20          # a fake, 256-byte aligned "device" address; never dereferenced
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_cache_367_b200 import build
+    build.build()
+    import paged_kv_cache_367_b200 as pkv
+    return pkv.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_0-9]+)\s*\(",
+                                 text, flags=re.M)))
+
+
+def test_every_declared_function_is_exported(lib):
+    names = declared_functions()
+    assert {"paged_kv_append", "paged_attention_decode", "paged_attention_workspace_size",
+            "pkv_status_string", "pkv_version"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_binding_names_match_the_header(lib):
+    import paged_kv_cache_367_b200 as pkv
+    assert set(pkv.EXPORTED_SYMBOLS) == set(declared_functions())
+    for n in pkv.EXPORTED_SYMBOLS:
+        assert callable(getattr(pkv, n))
+
+
+def test_status_strings(lib):
+    for s in (OK, ENULL, ESHAPE, EDTYPE, EUNSUP, EWS, ECUDA, EALIGN):
+        assert lib.pkv_status_string(s)
+    assert lib.pkv_status_string(12345) == b"unknown status"
+    assert lib.pkv_version() >= 100
+
+
+def decode(lib, **kw):
+    a = dict(out=A, query=A, k_cache=A, v_cache=A, block_table=A, seq_lens=A, num_seqs=4,
+             num_heads=8, num_kv_heads=2, head_dim=128, block_size=16, max_blocks_per_seq=8,
+             num_blocks=100, max_seq_len=128, scale=0.1, q_dtype=BF16, cache_dtype=BF16,
+             k_scale=A, v_scale=A, partition_size=0, max_ctas=0, flags=0, workspace=None,
+             workspace_bytes=0, stream=None)
+    a.update(kw)
+    return lib.paged_attention_decode(*a.values())
+
+
+def append(lib, **kw):
+    a = dict(key=A, value=A, k_cache=A, v_cache=A, slot_mapping=A, num_tokens=4, num_kv_heads=2,
+             head_dim=128, block_size=16, num_blocks=10, src_dtype=BF16, cache_dtype=BF16,
+             k_scale=A, v_scale=A, stream=None)
+    a.update(kw)
+    return lib.paged_kv_append(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(out=None), ENULL), (dict(query=None), ENULL), (dict(block_table=None), ENULL),
+    (dict(seq_lens=None), ENULL), (dict(cache_dtype=FP8, k_scale=None), ENULL),
+    (dict(num_heads=6, num_kv_heads=4), ESHAPE), (dict(num_kv_heads=0), ESHAPE),
+    (dict(num_seqs=-1), ESHAPE), (dict(max_seq_len=-1), ESHAPE), (dict(num_blocks=0), ESHAPE),
+    (dict(max_blocks_per_seq=0), ESHAPE), (dict(partition_size=-16), ESHAPE),
+    (dict(partition_size=24), ESHAPE), (dict(max_ctas=-1), ESHAPE),
+    (dict(scale=float("nan")), ESHAPE), (dict(scale=float("inf")), ESHAPE),
+    (dict(head_dim=96), EUNSUP), (dict(head_dim=256), EUNSUP), (dict(block_size=4), EUNSUP),
+    (dict(block_size=64), EUNSUP), (dict(q_dtype=FP8, cache_dtype=FP8), EDTYPE),
+    (dict(q_dtype=7), EDTYPE), (dict(q_dtype=BF16, cache_dtype=F16), EDTYPE),
+    (dict(out=A + 8), EALIGN), (dict(k_cache=A + 4), EALIGN), (dict(seq_lens=A + 2), EALIGN),
+    (dict(partition_size=512), EWS),
+    (dict(partition_size=512, workspace=A, workspace_bytes=100), EWS),
+    (dict(num_seqs=0, out=None), OK),
+])
+def test_decode_rejects_bad_arguments_on_the_host(lib, kw, code):
+    assert decode(lib, **kw) == code
+
+
+def test_workspace_size(lib):
+    ws = lib.paged_attention_workspace_size
+    assert ws(4, 8, 2, 128, 128, 0) == 0
+    parts = -(-1000 // 512)
+    need = ws(4, 8, 2, 128, 1000, 512)
+    assert need >= 4 * 8 * parts * (128 + 1) * 4 + 4 * 2 * parts * 4
+    assert need % 256 == 0
+    assert ws(-1, 8, 2, 128, 1000, 512) == 0
+    assert decode(lib, partition_size=512, max_seq_len=1000, workspace=A + 256,
+                  workspace_bytes=need - 1) == EWS
+    assert decode(lib, partition_size=512, max_seq_len=1000, workspace=A + 16,
+                  workspace_bytes=need) == EALIGN
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(key=None), ENULL), (dict(slot_mapping=None), ENULL),
+    (dict(cache_dtype=FP8, v_scale=None), ENULL), (dict(num_tokens=-1), ESHAPE),
+    (dict(head_dim=100), ESHAPE), (dict(num_kv_heads=0), ESHAPE), (dict(block_size=0), ESHAPE),
+    (dict(num_blocks=0), ESHAPE), (dict(src_dtype=FP8, cache_dtype=FP8), EDTYPE),
+    (dict(src_dtype=F32, cache_dtype=BF16), EDTYPE), (dict(key=A + 8), EALIGN),
+    (dict(slot_mapping=A + 4), EALIGN), (dict(num_tokens=0, key=None), OK),
+])
+def test_append_rejects_bad_arguments_on_the_host(lib, kw, code):
+    assert append(lib, **kw) == code
+
+
+def test_binding_raises_when_the_library_is_missing(tmp_path):
+    import paged_kv_cache_367_b200 as pkv
+    saved = pkv._lib
+    pkv._lib = None
+    try:
+        with pytest.raises(ImportError):
+            pkv.load_library(str(tmp_path / "absent.so"))
+    finally:
+        pkv._lib = saved
