@@ -1,0 +1,414 @@
+#!/usr/bin/env python
+"""Benchmark of the paged decode hot path on B200.
+
+One step = one decode iteration of one attention layer over a batch of
+sequences: paged_kv_append of each sequence's new token, then
+paged_attention_decode (plus its log-sum-exp merge launch when sequences are
+split). Inputs are seeded synthetic tensors already resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gqa70b]
+    python bench.py --impl reference ...    # the fp64 CPU oracle on host cores
+
+Under torchrun every rank runs its own replica of the workload (weak scaling;
+decode has no data-path collective); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import paged_kv_cache_367_b200 as pkv  # noqa: E402
+from paged_kv_cache_367_b200 import roofline  # noqa: E402
+from paged_kv_cache_367_b200 import workloads as W  # noqa: E402
+
+METRIC = "paged decode attention HBM GB/s (% of B200 peak) and decode tokens/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 2**20
+
+WORKLOAD_TEXT = {
+    "gqa70b": "70B-class GQA decode: 128 seqs, 64 q / 8 KV heads, head_dim 128, bf16 N(0,1), "
+              "block 16, lognormal lengths (median 1024, sigma 0.8) clipped to [16, 8192], "
+              "shuffled pool, one appended token per sequence",
+    "llama2_13b_mha": "Llama-2-13B-shaped decode: 64 seqs, 40 q = 40 KV heads, head_dim 128, fp16, "
+                      "block 16, lengths U[128, 2048], shuffled pool, append of 1 token per seq",
+    "long_splitk": "long-context split-K decode: 8 seqs, 32 q / 8 KV heads, head_dim 128, bf16, "
+                   "block 32, lengths U[32768, 131072], partitions of 512 merged by LSE",
+    "fp8_prefix": "FP8 E4M3 KV with per-tensor scales and a shared 1024-token prefix: 64 seqs, "
+                  "32 q / 8 KV heads, head_dim 128, bf16 Q, private suffix U[16, 512], block 16",
+    "tiny": "tiny fp32 decode: 4 seqs, 8 heads, head_dim 64, block 16, lengths U[1, 100]",
+}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="gqa70b", choices=sorted(W.CONFIGS))
+    ap.add_argument("--partition-size", type=int, default=None)
+    ap.add_argument("--max-ctas", type=int, default=0)
+    ap.add_argument("--flags", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_367_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, name), "rb").read())
+    h.update(open(os.path.join(ROOT, "include", "pagedkv.h"), "rb").read())
+    return h.hexdigest()[:12]
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback 6.65 TB/s"
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was taken
+    on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", f"ncu_decode_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_sha = re.search(r"^source_sha:\s*(\w+)", text, re.M)
+    m_b = re.search(r"^traffic_bytes_per_launch:\s*([0-9.eE+]+)", text, re.M)
+    if not (m_sha and m_b) or m_sha.group(1) != source_sha():
+        return None
+    return float(m_b.group(1))
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x10: "sync_boost"}
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            p = torch.cuda.get_device_properties(index)
+            try:
+                bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set() and self._nv is not None:
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": float(np.median(self.samples)) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "reasons": sorted(self.reasons)}
+
+
+def workload_config(wl, partition_size):
+    c = wl.cfg
+    kv_bytes = 2 * int(wl.seq_lens.sum()) * c.num_kv_heads * c.head_dim * W.ELEM_BYTES[c.cache_dtype]
+    return {"workload": WORKLOAD_TEXT.get(c.name, c.name), "name": c.name,
+            "num_seqs": c.num_seqs, "num_heads": c.num_heads, "num_kv_heads": c.num_kv_heads,
+            "head_dim": c.head_dim, "block_size": c.block_size, "q_dtype": c.q_dtype,
+            "cache_dtype": c.cache_dtype, "total_tokens": int(wl.seq_lens.sum()),
+            "max_seq_len": wl.max_seq_len, "partition_size": partition_size,
+            "l2": (f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of K/V read per step vs "
+                   f"126 MB L2" if kv_bytes > L2_BYTES else
+                   "K/V fit in L2: timing reuses L2-resident data (no flush)"),
+            "parallelism": "replicas: one independent workload per GPU, no collective"}
+
+
+def step_bytes(wl):
+    c = wl.cfg
+    eq, ekv = W.ELEM_BYTES[c.q_dtype], W.ELEM_BYTES[c.cache_dtype]
+    dec = roofline.decode_bytes(wl.seq_lens, c.num_heads, c.num_kv_heads, c.head_dim,
+                                c.block_size, eq, ekv, shared_prefix_tokens=c.prefix_len)
+    app = roofline.append_bytes(c.num_seqs, c.num_kv_heads, c.head_dim, eq, ekv)
+    return dec, app
+
+
+# ------------------------------------------------------------------ our arm ----
+
+def run_ours(args, rank, world, dev):
+    cfg = W.CONFIGS[args.workload]
+    cfg = cfg.replace(seed=cfg.seed + 7919 * rank)
+    P = cfg.partition_size if args.partition_size is None else args.partition_size
+    wl = W.make_workload(cfg, device=dev)
+    c = wl.cfg
+    bt = torch.from_numpy(wl.block_table).to(dev)
+    lens = torch.from_numpy(wl.seq_lens).to(dev)
+    slots = torch.from_numpy(wl.slot_mapping).to(dev)
+    ks = vs = None
+    if c.cache_dtype == "e4m3":
+        ks = torch.tensor([wl.k_scale], dtype=torch.float32, device=dev)
+        vs = torch.tensor([wl.v_scale], dtype=torch.float32, device=dev)
+    msl = wl.max_seq_len
+    ws_bytes = pkv.paged_attention_workspace_size(c.num_seqs, c.num_heads, c.num_kv_heads,
+                                                  c.head_dim, msl, P)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev) if ws_bytes else None
+    out = torch.empty_like(wl.query)
+    stream = torch.cuda.current_stream()
+    launches_per_step = 2 + (1 if P > 0 else 0)
+
+    def append(key, value, slot_t):
+        pkv.paged_kv_append(key, value, wl.k_cache, wl.v_cache, slot_t, k_scale=ks, v_scale=vs)
+
+    def decode(q, bt_t, lens_t, out_t):
+        pkv.paged_attention_decode(out_t, q, wl.k_cache, wl.v_cache, bt_t, lens_t, max_seq_len=msl,
+                                   scale=c.scale, partition_size=P, workspace=ws, k_scale=ks,
+                                   v_scale=vs, max_ctas=args.max_ctas, flags=args.flags)
+
+    for _ in range(max(args.warmup, 3)):
+        append(wl.new_key, wl.new_value, slots)
+        decode(wl.query, bt, lens, out)
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t0.record(stream)
+        for k in range(K):
+            append(wl.new_key, wl.new_value, slots)
+            ev[k][0].record(stream)
+            decode(wl.query, bt, lens, out)
+            ev[k][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    step_ms = t0.elapsed_time(t1) / K
+    decode_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    if world > 1:
+        torch.distributed.barrier()
+
+    # End to end: per-step inputs start in pinned host memory, the output ends there.
+    KE = args.e2e_steps or min(K, 200)
+    h_q = wl.query.cpu().pin_memory()
+    h_k, h_v = wl.new_key.cpu().pin_memory(), wl.new_value.cpu().pin_memory()
+    h_slots = torch.from_numpy(wl.slot_mapping).pin_memory()
+    h_bt = torch.from_numpy(wl.block_table).pin_memory()
+    h_lens = torch.from_numpy(wl.seq_lens).pin_memory()
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    d_q, d_k, d_v = torch.empty_like(wl.query), torch.empty_like(wl.new_key), torch.empty_like(wl.new_value)
+    d_slots, d_bt, d_lens = torch.empty_like(slots), torch.empty_like(bt), torch.empty_like(lens)
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_bt, h_lens))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        for d, h in ((d_q, h_q), (d_k, h_k), (d_v, h_v), (d_slots, h_slots), (d_bt, h_bt),
+                     (d_lens, h_lens)):
+            d.copy_(h, non_blocking=True)
+        append(d_k, d_v, d_slots)
+        decode(d_q, d_bt, d_lens, out)
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(KE):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / KE
+    assert torch.isfinite(h_out.float()).all(), "non-finite decode output"
+
+    if world > 1:
+        t = torch.tensor([step_ms, decode_ms, e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        step_ms, decode_ms, e2e_ms = t.tolist()
+
+    dec_b, app_b = step_bytes(wl)
+    peak, peak_src = measured_hbm_peak()
+    value = world * (dec_b + app_b) / (step_ms * 1e-3) / 1e9
+    achieved = dec_b / (decode_ms * 1e-3) / 1e9
+    res = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": c.q_dtype if c.cache_dtype == c.q_dtype else f"{c.q_dtype}+{c.cache_dtype}",
+        "data": "synthetic (seeded N(0,1) tensors, shuffled block pool)",
+        "config": workload_config(wl, P),
+        "tokens_per_s": round(world * c.num_seqs / (step_ms * 1e-3), 1),
+        "pct_of_8TBs_nominal": round(100 * value / world / NOMINAL_HBM_GBS, 2),
+        "decode_ms": round(decode_ms, 5),
+        "bytes_per_step": {"decode": dec_b, "append": app_b},
+        "roofline": {"bound": "hbm", "kernel": "paged_attention_decode (decode + merge launches)",
+                     "achieved": round(achieved, 2), "peak": peak, "peak_source": peak_src,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": profiled_traffic(c.name)},
+        "e2e": {"value": round(world * dec_b / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 5), "steps": KE, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": K * launches_per_step,
+        "clocks": clk.summary(),
+        "source_sha": source_sha(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+    return res
+
+
+# -------------------------------------------------------- oracle on the host ----
+
+def _oracle_rate(wl, kc, vc, items, threads=0):
+    import oracle
+    c = wl.cfg
+    t = time.perf_counter()
+    _, used = oracle.decode(W.host(wl.query), kc, vc, wl.block_table, wl.seq_lens,
+                            num_heads=c.num_heads, num_kv_heads=c.num_kv_heads, head_dim=c.head_dim,
+                            block_size=c.block_size, scale=c.scale, q_dtype=c.q_dtype,
+                            cache_dtype=c.cache_dtype, k_scale=wl.k_scale, v_scale=wl.v_scale,
+                            items=items, threads=threads)
+    return time.perf_counter() - t, used
+
+
+def _item_bytes(wl, items):
+    c = wl.cfg
+    eq, ekv = W.ELEM_BYTES[c.q_dtype], W.ELEM_BYTES[c.cache_dtype]
+    per_seq = [roofline.decode_bytes([L], c.num_heads, c.num_kv_heads, c.head_dim, c.block_size,
+                                     eq, ekv) for L in wl.seq_lens]
+    return sum(per_seq[i] for i, _ in items) / c.num_heads
+
+
+def cpu_baseline(wl, seconds):
+    """The fp64 oracle, as it stands, on a bounded sample of the same workload."""
+    c = wl.cfg
+    kc, vc = W.host(wl.k_cache), W.host(wl.v_cache)
+    all_items = [(i, j) for i in range(c.num_seqs) for j in range(c.num_heads)]
+    probe = all_items[:c.num_heads]
+    dt, _ = _oracle_rate(wl, kc, vc, probe)
+    per_seq = max(dt, 1e-4)
+    n_seq = int(max(1, min(c.num_seqs, seconds / per_seq)))
+    items = all_items[:n_seq * c.num_heads]
+    dt, used = _oracle_rate(wl, kc, vc, items)
+    b = _item_bytes(wl, items)
+    return {"value": round(b / dt / 1e9, 4), "unit": "GB/s", "cores": used, "kind": "oracle",
+            "seconds": round(dt, 2),
+            "sample": f"first {n_seq} of {c.num_seqs} sequences, all {c.num_heads} query heads "
+                      f"({sum(int(wl.seq_lens[i]) for i in range(n_seq))} tokens), fp64 C "
+                      f"oracle with OpenMP over (sequence, head)"}
+
+
+def run_reference(args):
+    cfg = W.CONFIGS[args.workload]
+    wl = W.make_workload(cfg, device="cpu")
+    c = wl.cfg
+    kc, vc = W.host(wl.k_cache), W.host(wl.v_cache)
+    # Fill each sequence's newest slot as the append of a step would.
+    import oracle
+    oracle.append(W.host(wl.new_key), W.host(wl.new_value), kc, vc, wl.slot_mapping,
+                  num_kv_heads=c.num_kv_heads, head_dim=c.head_dim, block_size=c.block_size,
+                  num_blocks=wl.num_blocks, src_dtype=c.q_dtype, cache_dtype=c.cache_dtype,
+                  k_scale=wl.k_scale, v_scale=wl.v_scale)
+    all_items = [(i, j) for i in range(c.num_seqs) for j in range(c.num_heads)]
+    dt, _ = _oracle_rate(wl, kc, vc, all_items[:c.num_heads])
+    rate = c.num_heads / max(dt, 1e-6)                        # items per second, all threads
+    budget = 90.0 / max(1, args.steps + args.warmup)          # seconds per step
+    n = int(max(1, min(len(all_items), budget * rate)))
+    pos = 0
+    total_b, total_t, used = 0.0, 0.0, 1
+    for k in range(args.warmup + args.steps):
+        items = [all_items[(pos + m) % len(all_items)] for m in range(n)]
+        pos += n
+        dt, used = _oracle_rate(wl, kc, vc, items)
+        if k >= args.warmup:
+            total_t += dt
+            total_b += _item_bytes(wl, items)
+    value = total_b / total_t / 1e9
+    ms = total_t / args.steps * 1e3
+    sample = (f"{n} (sequence, query head) items per step, cycling through the workload; "
+              f"fp64 C oracle, OpenMP over items")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) tensors)",
+            "config": workload_config(wl, c.partition_size),
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": used,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    try:
+        res = run_ours(args, rank, world, dev)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,13 +1,567 @@
-// Tensor-core PagedAttention decode (16-bit caches). Not yet built: every
-// configuration goes to the CUDA-core kernel.
+// PagedAttention decode on tensor cores, K/V tiles staged by TMA (sm_100a).
+//
+// What it computes is the per-sequence walk of "vLLM 推理引擎源码级拆解"
+// (chenxutan.com/d/5333) §2.3: logical block = tok / block_size, physical
+// block = block_table[logical block], score = dot(q, k) * scale, online
+// softmax, accumulate V, write back; with GQA (§2.3), the g query heads of one
+// KV head are served by a single read of its K/V.
+//
+// How, on B200:
+//  * One CTA per SM (persistent) takes a balanced, contiguous share of the
+//    (sequence, KV head) work (schedule.cuh).
+//  * A producer warp walks the same segments and streams 64-token chunks of K
+//    and V into a ring of shared-memory stages. Each physical block is one TMA
+//    tensor copy: the pool [num_blocks, bs, Hkv, D] is described as a 5-D tensor
+//    (d_lo 64, token, d_hi, head, block) so a (block, head) tile lands as
+//    128-byte rows with the 128B swizzle; a block id outside the pool is out of
+//    the tensor's bounds and lands as zeros. The query rows of a segment come
+//    with its first chunk by a bulk copy. Stages are handed over with mbarriers.
+//  * Four consumer warps each take 16 tokens of a chunk. The dense part is
+//    small (g <= 16 query heads, head_dim 64/128) but it is a real contraction,
+//    so it runs on the tensor pipe with mma.sync m16n8k16 in the transposed form
+//    S^T = K Q^T (tokens on M, query heads on N = 8), keeping the CUDA cores free
+//    and avoiding per-element conversions and cross-lane dot-product reductions.
+//    P is rounded to the cache dtype, transposed in registers (movmatrix) into
+//    the B operand of O^T += V^T P^T, with V^T fed by ldmatrix.trans.
+//  * At the end of a segment the four warps' softmax states are merged through
+//    shared memory; a whole unit is written out directly, a piece of a split
+//    unit leaves a partial (output row, base-2 log-sum-exp) for the merge kernel.
+//  * Every mbarrier wait is bounded (about a second); on expiry the CTA sets an
+//    error word, skips the rest of its work and still waits, bounded, for its
+//    own copies in flight before it exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "schedule.cuh"
 
 namespace pkv {
 
-bool tc_supported(int, int, int, int) { return false; }
+__device__ int g_tc_timeout = 0;
 
-cudaError_t launch_decode_tc(const DecodeParams&, int, int, int, int, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace tc {
+
+constexpr int kChunk = 64;          // tokens per stage
+constexpr int kConsumerWarps = 4;   // 16 tokens each
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr long long kWaitCycles = 1ll << 31;  // ~1 s at 2 GHz
+
+template <int D, int NT, int NS>
+struct Cfg {
+  static constexpr int kKV = kChunk * D * 2;       // bytes of K (or V) per stage
+  static constexpr int kQ = 8 * NT * D * 2;        // query rows of one KV head group
+  static constexpr int kStage = (2 * kKV + kQ + 1023) / 1024 * 1024;
+  static constexpr int kHeads = 8 * NT;
+  static constexpr int kRedO = kConsumerWarps * kHeads * D * 4;
+  static constexpr int kRedML = 2 * kConsumerWarps * kHeads * 4;
+  static constexpr int kBar = 2 * NS * 8;
+  static constexpr int kSmem = 1024 + NS * kStage + kRedO + kRedML + kBar +
+                               (int)sizeof(SchedShared) + 16;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase of `bar` with the given parity. Returns false if
+// the CTA is aborting or the wait expired (which starts the abort).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (*abort) return false;
+  const long long t0 = clock64();
+  for (int it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 31) == 0) {
+      if (*abort) return false;
+      if (clock64() - t0 > kWaitCycles) {
+        *abort = 1;
+        atomicExch(&g_tc_timeout, 1);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            int c3, int c4, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
+      "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+
+template <typename T> struct Mma;
+template <> struct Mma<__nv_bfloat16> {
+  static __device__ __forceinline__ void run(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                             uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+  static __device__ __forceinline__ uint32_t pack(float lo, float hi, float& rlo, float& rhi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    rlo = __low2float(v);
+    rhi = __high2float(v);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+};
+template <> struct Mma<__half> {
+  static __device__ __forceinline__ void run(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                             uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+  static __device__ __forceinline__ uint32_t pack(float lo, float hi, float& rlo, float& rhi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    rlo = __low2float(v);
+    rhi = __high2float(v);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+};
+
+__device__ __forceinline__ void named_sync_consumers() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+}
+
+template <typename T, int D, int NT, int NS>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_tc_kernel(const DecodeParams prm, const __grid_constant__ CUtensorMap tmap_k,
+                     const __grid_constant__ CUtensorMap tmap_v) {
+  using C = Cfg<D, NT, NS>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  float* red_o = reinterpret_cast<float*>(smem + NS * C::kStage);
+  float* red_m = red_o + kConsumerWarps * C::kHeads * D;
+  float* red_l = red_m + kConsumerWarps * C::kHeads;
+  uint64_t* full = reinterpret_cast<uint64_t*>(red_l + kConsumerWarps * C::kHeads);
+  uint64_t* empty = full + NS;
+  SchedShared* sched = reinterpret_cast<SchedShared*>(empty + NS);
+  volatile int* abort = reinterpret_cast<volatile int*>(sched + 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, kConsumerWarps);
+    }
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  SegmentWalker walker;
+  init_walker<T>(prm, *sched, walker);  // ends with __syncthreads
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int Hq = prm.num_heads, Hkv = prm.num_kv_heads, g = Hq / Hkv, bs = prm.block_size;
+  const int tile = bs * D * 2;  // bytes of one (block, head) tile
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ producer ----
+    int stage = 0;
+    uint32_t phase = 0, armed = 0, last_parity = 0;
+    bool ok = true;
+    const T* qbase = static_cast<const T*>(prm.query);
+    Segment seg;
+    while (walker.next(seg)) {
+      const int32_t* bt = prm.block_table + (int64_t)seg.seq * prm.max_blocks_per_seq;
+      const int lb0 = seg.t0 / bs;
+      const int nlb = (seg.t1 + bs - 1) / bs - lb0;
+      int cur = lane < nlb ? __ldg(bt + lb0 + lane) : 0;
+      int nxt = lane + 32 < nlb ? __ldg(bt + lb0 + 32 + lane) : 0;
+      int batch = 0;
+      for (int c0 = seg.t0; c0 < seg.t1; c0 += kChunk) {
+        const int rel = (c0 - seg.t0) / bs;
+        if (rel >= batch + 32) {
+          cur = nxt;
+          batch += 32;
+          nxt = lane + batch + 32 < nlb ? __ldg(bt + lb0 + batch + 32 + lane) : 0;
+        }
+        const int ntok = min(kChunk, seg.t1 - c0);
+        const int nblk = (ntok + bs - 1) / bs;
+        const bool first = c0 == seg.t0;
+        if (lane == 0 && ok) ok = mbar_wait(empty + stage, phase ^ 1u, abort);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        uint8_t* st = ring + stage * C::kStage;
+        if (ok && lane == 0) {
+          const uint32_t qbytes = first ? (uint32_t)(g * D * 2) : 0u;
+          mbar_expect_tx(full + stage, (uint32_t)(2 * nblk * tile) + qbytes);
+          if (first)
+            bulk_load(st + 2 * C::kKV, qbase + ((int64_t)seg.seq * Hq + seg.head * g) * D, qbytes,
+                      full + stage);
+        }
+        for (int b = 0; b < nblk; ++b) {
+          const int phys = __shfl_sync(0xffffffffu, cur, rel - batch + b);
+          if (ok && lane == 0) {
+            tma_load_5d(st + b * tile, &tmap_k, 0, 0, 0, seg.head, phys, full + stage);
+            tma_load_5d(st + C::kKV + b * tile, &tmap_v, 0, 0, 0, seg.head, phys, full + stage);
+          }
+        }
+        if (ok) {
+          armed |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+        }
+        if (++stage == NS) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    // Wait, bounded, for this CTA's copies in flight before leaving.
+    if (lane == 0) {
+      for (int s = 0; s < NS; ++s) {
+        if (!(armed >> s & 1u)) continue;
+        const long long t0 = clock64();
+        while (!mbar_try(full + s, (last_parity >> s) & 1u)) {
+          if (clock64() - t0 > kWaitCycles) {
+            atomicExch(&g_tc_timeout, 1);
+            break;
+          }
+        }
+      }
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers ----
+  const int w = warp;
+  const int g0 = lane >> 2, cq = lane & 3, x7 = lane & 7;
+  const int kt = 16 * w + ((lane >> 3) & 1) * 8 + x7;  // token row this lane addresses for K
+  const int vt = 16 * w + ((lane >> 4) & 1) * 8 + x7;  // ... and for V
+  const int kj = (lane >> 4) & 1, vj = (lane >> 3) & 1;
+  const uint32_t krow = (uint32_t)((kt / bs) * tile + (kt % bs) * 128);
+  const uint32_t vrow = (uint32_t)((vt / bs) * tile + (vt % bs) * 128);
+  const uint32_t dh_stride = (uint32_t)(bs * 128);
+  const uint32_t ring_u32 = smem_u32(ring);
+  const float sscale = prm.score_scale;
+  constexpr int MT = D / 16;
+
+  int stage = 0;
+  uint32_t phase = 0;
+  Segment seg;
+  while (walker.next(seg)) {
+    float m[2 * NT], l[2 * NT];
+    float o[MT][NT][4];
+    uint32_t bq[MT][NT][2];
+#pragma unroll
+    for (int x = 0; x < 2 * NT; ++x) {
+      m[x] = -INFINITY;
+      l[x] = 0.f;
+    }
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
+
+    for (int c0 = seg.t0; c0 < seg.t1; c0 += kChunk) {
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(full + stage, phase, abort));
+      const uint32_t st = ring_u32 + stage * C::kStage;
+      if (ok && c0 == seg.t0) {
+        // Q^T fragments: b0b1 = Q[head g0][16ks + 2cq, +1], b2b3 = the same + 8 dims.
+        const uint8_t* qs = ring + stage * C::kStage + 2 * C::kKV;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int head = nt * 8 + g0;
+#pragma unroll
+          for (int ks = 0; ks < MT; ++ks) {
+            uint32_t b0 = 0, b1 = 0;
+            if (head < g) {
+              const uint32_t* row = reinterpret_cast<const uint32_t*>(qs + head * D * 2);
+              b0 = row[(16 * ks + 2 * cq) / 2];
+              b1 = row[(16 * ks + 8 + 2 * cq) / 2];
+            }
+            bq[ks][nt][0] = b0;
+            bq[ks][nt][1] = b1;
+          }
+        }
+      }
+      const int nv = min(16, max(0, seg.t1 - (c0 + 16 * w)));
+      if (ok && nv > 0) {
+        // S^T = K Q^T for this warp's 16 tokens.
+        float s[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < MT; ++ks) {
+          uint32_t a[4];
+          const int dh = ks >> 2, j = ((ks & 3) << 1) + kj;
+          ldsm_x4(a, st + krow + dh * dh_stride + ((j ^ x7) << 4));
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) Mma<T>::run(s[nt], a, bq[ks][nt][0], bq[ks][nt][1]);
+        }
+        const bool v0 = g0 < nv, v1 = g0 + 8 < nv;
+        uint32_t bp[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float alpha[2], p[2][2];
+#pragma unroll
+          for (int hi = 0; hi < 2; ++hi) {
+            const float s0 = v0 ? s[nt][hi] * sscale : -INFINITY;
+            const float s1 = v1 ? s[nt][2 + hi] * sscale : -INFINITY;
+            float mx = fmaxf(s0, s1);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const int x = nt * 2 + hi;
+            const float mn = fmaxf(m[x], mx);
+            const float mu = mn == -INFINITY ? 0.f : mn;
+            alpha[hi] = fast_exp2(m[x] - mu);
+            m[x] = mn;
+            p[hi][0] = fast_exp2(s0 - mu);
+            p[hi][1] = fast_exp2(s1 - mu);
+          }
+          float r00, r01, r10, r11;
+          const uint32_t P0 = Mma<T>::pack(p[0][0], p[1][0], r00, r01);  // token g0, heads 2cq, 2cq+1
+          const uint32_t P1 = Mma<T>::pack(p[0][1], p[1][1], r10, r11);  // token g0 + 8
+          l[nt * 2 + 0] = l[nt * 2 + 0] * alpha[0] + (r00 + r10);
+          l[nt * 2 + 1] = l[nt * 2 + 1] * alpha[1] + (r01 + r11);
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            o[mt][nt][0] *= alpha[0];
+            o[mt][nt][1] *= alpha[1];
+            o[mt][nt][2] *= alpha[0];
+            o[mt][nt][3] *= alpha[1];
+          }
+          bp[nt][0] = movmatrix_t(P0);
+          bp[nt][1] = movmatrix_t(P1);
+        }
+        // Tokens past the end of the segment hold stale or poisoned rows: zero
+        // their V operands (their P is already 0, and 0 * NaN would be NaN).
+        uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+        if (nv < 16) {
+          mlo = (2 * cq < nv ? 0x0000ffffu : 0u) | (2 * cq + 1 < nv ? 0xffff0000u : 0u);
+          mhi = (2 * cq + 8 < nv ? 0x0000ffffu : 0u) | (2 * cq + 9 < nv ? 0xffff0000u : 0u);
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          uint32_t a[4];
+          const int dh = mt >> 2, j = ((mt & 3) << 1) + vj;
+          ldsm_x4_t(a, st + C::kKV + vrow + dh * dh_stride + ((j ^ x7) << 4));
+          a[0] &= mlo;
+          a[1] &= mlo;
+          a[2] &= mhi;
+          a[3] &= mhi;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) Mma<T>::run(o[mt][nt], a, bp[nt][0], bp[nt][1]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty + stage);
+      if (++stage == NS) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+
+    // ---- segment epilogue: merge the four warps' states ----
+#pragma unroll
+    for (int x = 0; x < 2 * NT; ++x) {
+      l[x] += __shfl_xor_sync(0xffffffffu, l[x], 4);
+      l[x] += __shfl_xor_sync(0xffffffffu, l[x], 8);
+      l[x] += __shfl_xor_sync(0xffffffffu, l[x], 16);
+    }
+    if (g0 == 0) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int hi = 0; hi < 2; ++hi) {
+          const int head = nt * 8 + 2 * cq + hi;
+          red_m[w * C::kHeads + head] = m[nt * 2 + hi];
+          red_l[w * C::kHeads + head] = l[nt * 2 + hi];
+        }
+    }
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int h0 = nt * 8 + 2 * cq, d0 = mt * 16 + g0;
+        float* base = red_o + (w * C::kHeads) * D;
+        base[h0 * D + d0] = o[mt][nt][0];
+        base[(h0 + 1) * D + d0] = o[mt][nt][1];
+        base[h0 * D + d0 + 8] = o[mt][nt][2];
+        base[(h0 + 1) * D + d0 + 8] = o[mt][nt][3];
+      }
+    named_sync_consumers();
+    const bool whole = seg.t0 == 0 && seg.t1 == seg.len;
+    const int i = seg.seq, h = seg.head;
+    for (int e = threadIdx.x; e < g * D; e += kConsumerWarps * 32) {
+      const int j = e / D, d = e - j * D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int x = 0; x < kConsumerWarps; ++x) M = fmaxf(M, red_m[x * C::kHeads + j]);
+      float L = 0.f, O = 0.f;
+#pragma unroll
+      for (int x = 0; x < kConsumerWarps; ++x) {
+        const float wgt = fast_exp2(red_m[x * C::kHeads + j] - M);
+        L = fmaf(wgt, red_l[x * C::kHeads + j], L);
+        O = fmaf(wgt, red_o[(x * C::kHeads + j) * D + d], O);
+      }
+      const int qh = h * g + j;
+      if (whole) {
+        static_cast<T*>(prm.out)[((int64_t)i * Hq + qh) * D + d] = from_f32<T>(O / L);
+      } else {
+        const int64_t rowp = ((int64_t)i * Hq + qh) * prm.max_parts + seg.t0 / prm.part;
+        prm.ws_o[rowp * D + d] = O / L;
+        if (d == 0) prm.ws_lse[rowp] = M + fast_log2(L);
+      }
+    }
+    if (threadIdx.x == 0 && prm.part > 0) {
+      const int64_t u = (int64_t)i * Hkv + h;
+      prm.ws_link[u * prm.max_parts + seg.t0 / prm.part] = (seg.t1 + prm.part - 1) / prm.part;
+    }
+    named_sync_consumers();
+  }
+}
+
+}  // namespace tc
+
+// ---------------------------------------------------------------- host side ----
+
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 5-D view of a [num_blocks, bs, Hkv, D] 16-bit pool: (d_lo 64, token bs, d_hi D/64,
+// head Hkv, block num_blocks); one box is a whole (block, head) tile.
+static bool encode_pool_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int D,
+                            int bs, int Hkv, int64_t nb) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t e = 2;
+  cuuint64_t dims[5] = {64, (cuuint64_t)bs, (cuuint64_t)(D / 64), (cuuint64_t)Hkv, (cuuint64_t)nb};
+  cuuint64_t strides[4] = {(cuuint64_t)Hkv * D * e, 64 * e, (cuuint64_t)D * e,
+                           (cuuint64_t)bs * Hkv * D * e};
+  cuuint32_t box[5] = {64, (cuuint32_t)bs, (cuuint32_t)(D / 64), 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(map, dt, 5, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool tc_supported(int q_dtype, int cache_dtype, int head_dim, int group) {
+  return (q_dtype == PKV_BF16 || q_dtype == PKV_F16) && cache_dtype == q_dtype &&
+         (head_dim == 64 || head_dim == 128) && group >= 1 && group <= 16;
+}
+
+template <typename T, int D, int NT, int NS>
+static cudaError_t launch_tc_t(const DecodeParams& prm, const CUtensorMap& mk,
+                               const CUtensorMap& mv, int max_ctas, int num_sms,
+                               cudaStream_t stream) {
+  using C = tc::Cfg<D, NT, NS>;
+  auto kernel = tc::decode_tc_kernel<T, D, NT, NS>;
+  static int occ = 0;
+  if (occ == 0) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmem);
+    if (e != cudaSuccess) return e;
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, tc::kThreads, C::kSmem);
+    if (e != cudaSuccess) return e;
+    occ = n > 0 ? n : 1;
+  }
+  int grid = occ * num_sms;
+  if (max_ctas > 0 && max_ctas < grid) grid = max_ctas;
+  kernel<<<grid, tc::kThreads, C::kSmem, stream>>>(prm, mk, mv);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+static cudaError_t launch_tc_d(const DecodeParams& prm, const CUtensorMap& mk,
+                               const CUtensorMap& mv, int max_ctas, int num_sms,
+                               cudaStream_t stream) {
+  const int g = prm.num_heads / prm.num_kv_heads;
+  if (g <= 8) return launch_tc_t<T, D, 1, (D == 128 ? 5 : 8)>(prm, mk, mv, max_ctas, num_sms, stream);
+  return launch_tc_t<T, D, 2, (D == 128 ? 5 : 8)>(prm, mk, mv, max_ctas, num_sms, stream);
+}
+
+cudaError_t launch_decode_tc(const DecodeParams& prm, int q_dtype, int cache_dtype, int max_ctas,
+                             int num_sms, cudaStream_t stream) {
+  (void)cache_dtype;
+  const CUtensorMapDataType dt =
+      q_dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUtensorMap mk, mv;
+  if (!encode_pool_map(&mk, prm.k_cache, dt, prm.head_dim, prm.block_size, prm.num_kv_heads,
+                       prm.num_blocks) ||
+      !encode_pool_map(&mv, prm.v_cache, dt, prm.head_dim, prm.block_size, prm.num_kv_heads,
+                       prm.num_blocks))
+    return cudaErrorInvalidValue;
+  if (q_dtype == PKV_BF16) {
+    return prm.head_dim == 128
+               ? launch_tc_d<__nv_bfloat16, 128>(prm, mk, mv, max_ctas, num_sms, stream)
+               : launch_tc_d<__nv_bfloat16, 64>(prm, mk, mv, max_ctas, num_sms, stream);
+  }
+  return prm.head_dim == 128 ? launch_tc_d<__half, 128>(prm, mk, mv, max_ctas, num_sms, stream)
+                             : launch_tc_d<__half, 64>(prm, mk, mv, max_ctas, num_sms, stream);
 }
 
 }  // namespace pkv

@@ -23,7 +23,7 @@ def read_golden(name: str) -> dict:
             if not line or line.startswith("#"):
                 continue
             key, *vals = line.split()
-            nums = [int(v) for v in vals]
+            nums = [float(v) if "." in v else int(v) for v in vals]
             out[key] = nums if len(nums) > 1 else nums[0]
     return out
 
