@@ -152,6 +152,15 @@ int paged_attention_decode(void* out, const void* query, const void* k_cache,
                            unsigned flags, void* workspace, size_t workspace_bytes,
                            void* stream);
 
+/*
+ * Health word of the device kernels. Every wait inside a kernel is bounded
+ * (about one second); a wait that expires makes its CTA skip the rest of its
+ * work and sets this word, so a wrong result is reported instead of a hung GPU.
+ * Returns 0 (no expiry since the last clear), 1 (a wait expired), or
+ * PKV_ERR_CUDA. Synchronises the current device; clear != 0 resets the word.
+ */
+int pkv_device_status(int clear);
+
 /* Static, NUL-terminated description of a pkv_status value. */
 const char* pkv_status_string(int status);
 

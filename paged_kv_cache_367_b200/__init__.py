@@ -15,7 +15,7 @@ import os
 import torch
 
 __all__ = ["paged_kv_append", "paged_attention_decode", "paged_attention_workspace_size",
-           "pkv_status_string", "pkv_version", "load_library", "PagedKVError",
+           "pkv_device_status", "pkv_status_string", "pkv_version", "load_library", "PagedKVError",
            "PKV_F32", "PKV_F16", "PKV_BF16", "PKV_FP8_E4M3", "PKV_DECODE_FORCE_SIMT",
            "LIB_PATH", "EXPORTED_SYMBOLS"]
 
@@ -25,7 +25,8 @@ PKV_F32, PKV_F16, PKV_BF16, PKV_FP8_E4M3 = 0, 1, 2, 3
 PKV_DECODE_FORCE_SIMT = 1
 
 EXPORTED_SYMBOLS = ("paged_kv_append", "paged_attention_workspace_size",
-                    "paged_attention_decode", "pkv_status_string", "pkv_version")
+                    "paged_attention_decode", "pkv_device_status", "pkv_status_string",
+                    "pkv_version")
 
 _DTYPE_CODES = {torch.float32: PKV_F32, torch.float16: PKV_F16, torch.bfloat16: PKV_BF16,
                 torch.uint8: PKV_FP8_E4M3, torch.float8_e4m3fn: PKV_FP8_E4M3}
@@ -61,6 +62,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pkv_status_string.restype = ctypes.c_char_p
     lib.pkv_version.argtypes = []
     lib.pkv_version.restype = I
+    lib.pkv_device_status.argtypes = [I]
+    lib.pkv_device_status.restype = I
     _lib = lib
     return lib
 
@@ -71,6 +74,11 @@ def pkv_status_string(status: int) -> str:
 
 def pkv_version() -> int:
     return load_library().pkv_version()
+
+
+def pkv_device_status(clear: bool = False) -> int:
+    """0: no bounded wait inside a kernel has expired (since the last clear)."""
+    return load_library().pkv_device_status(1 if clear else 0)
 
 
 def _ptr(t):

@@ -35,23 +35,27 @@ def _deps_mtime():
     return max(os.path.getmtime(f) for f in files)
 
 
-def _compile(src):
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
-    subprocess.check_call([NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj])
+def _compile(src, build_dir, extra):
+    obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
+    subprocess.check_call([NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj])
     return obj
 
 
-def build(force: bool = False) -> str:
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _deps_mtime():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, extra_flags=(), out: str = LIB) -> str:
+    """Compile csrc/*.cu and link `out`. `extra_flags` (e.g. -D tuning macros) go
+    to every nvcc compile; such variants should be linked to a different path."""
+    if not force and not extra_flags and os.path.exists(out) and \
+            os.path.getmtime(out) >= _deps_mtime():
+        return out
+    build_dir = BUILD if not extra_flags else os.path.join(BUILD, "variant_%d" % os.getpid())
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sources()
     with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(_compile, srcs))
-    tmp = LIB + f".tmp{os.getpid()}"
+        objs = list(ex.map(lambda s: _compile(s, build_dir, list(extra_flags)), srcs))
+    tmp = out + f".tmp{os.getpid()}"
     subprocess.check_call([NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static"])
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":

@@ -41,7 +41,15 @@ __device__ int g_tc_timeout = 0;
 namespace tc {
 
 constexpr int kChunk = 64;          // tokens per stage
-constexpr int kConsumerWarps = 4;   // 16 tokens each
+constexpr int kTeamWarps = 4;       // a team takes a chunk: 16 tokens per warp
+#ifndef PKV_TC_TEAMS
+#define PKV_TC_TEAMS 1
+#endif
+constexpr int kTeams = PKV_TC_TEAMS;  // teams take alternate segments
+#ifndef PKV_TC_CTAS_PER_SM
+#define PKV_TC_CTAS_PER_SM 2
+#endif
+constexpr int kConsumerWarps = kTeams * kTeamWarps;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr long long kWaitCycles = 1ll << 31;  // ~1 s at 2 GHz
 
@@ -51,11 +59,12 @@ struct Cfg {
   static constexpr int kQ = 8 * NT * D * 2;        // query rows of one KV head group
   static constexpr int kStage = (2 * kKV + kQ + 1023) / 1024 * 1024;
   static constexpr int kHeads = 8 * NT;
-  static constexpr int kRedO = kConsumerWarps * kHeads * D * 4;
+  static constexpr int kRedO = kConsumerWarps * kHeads * D * 4;   // per team: 4 warps
   static constexpr int kRedML = 2 * kConsumerWarps * kHeads * 4;
-  static constexpr int kBar = 2 * NS * 8;
+  static constexpr int kBar = 2 * NS * 8 + NS * 4;  // full/empty barriers, stage tickets
   static constexpr int kSmem = 1024 + NS * kStage + kRedO + kRedML + kBar +
                                (int)sizeof(SchedShared) + 16;
+  static_assert(kSmem <= 227 * 1024, "shared memory per CTA exceeds 227 KB");
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -103,6 +112,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       }
     }
   }
+}
+
+// Bounded wait until the producer has armed stage `ticket` for chunk kc.
+__device__ __forceinline__ bool wait_ticket(volatile uint32_t* ticket, uint32_t kc,
+                                            volatile int* abort) {
+  if (*abort) return false;
+  const long long t0 = clock64();
+  for (int it = 1; *ticket != kc; ++it) {
+    __nanosleep(32);
+    if ((it & 31) == 0) {
+      if (*abort) return false;
+      if (clock64() - t0 > kWaitCycles) {
+        *abort = 1;
+        atomicExch(&g_tc_timeout, 1);
+        return false;
+      }
+    }
+  }
+  __threadfence_block();
+  return true;
 }
 
 __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
@@ -175,12 +204,12 @@ template <> struct Mma<__half> {
   }
 };
 
-__device__ __forceinline__ void named_sync_consumers() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+__device__ __forceinline__ void named_sync_team(int team) {
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "n"(kTeamWarps * 32) : "memory");
 }
 
-template <typename T, int D, int NT, int NS>
-__global__ void __launch_bounds__(kThreads, 1)
+template <typename T, int D, int NT, int NS, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB)
     decode_tc_kernel(const DecodeParams prm, const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v) {
   using C = Cfg<D, NT, NS>;
@@ -193,13 +222,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* red_l = red_m + kConsumerWarps * C::kHeads;
   uint64_t* full = reinterpret_cast<uint64_t*>(red_l + kConsumerWarps * C::kHeads);
   uint64_t* empty = full + NS;
-  SchedShared* sched = reinterpret_cast<SchedShared*>(empty + NS);
+  // ticket[s] = number of the chunk the producer last armed stage s for. A team
+  // may be several ring laps ahead of the other, so it first waits for the
+  // ticket of its chunk; after that the parity wait on full[s] is unambiguous.
+  volatile uint32_t* ticket = reinterpret_cast<volatile uint32_t*>(empty + NS);
+  SchedShared* sched = reinterpret_cast<SchedShared*>(
+      reinterpret_cast<uint8_t*>(empty + NS) + ((NS * 4 + 7) & ~7));
   volatile int* abort = reinterpret_cast<volatile int*>(sched + 1);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(full + s, 1);
-      mbar_init(empty + s, kConsumerWarps);
+      mbar_init(empty + s, kTeamWarps);  // each chunk is consumed by one team
+      ticket[s] = 0xffffffffu;
     }
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -214,19 +249,36 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------ producer ----
-    int stage = 0;
-    uint32_t phase = 0, armed = 0, last_parity = 0;
+    // Streams the chunks of every segment, in order, into the ring. The block
+    // ids of the next segment are loaded while the current one is issued.
+    uint32_t kc = 0;  // chunk counter: stage kc % NS, phase (kc / NS) & 1
+    uint32_t armed = 0, last_parity = 0;
     bool ok = true;
     const T* qbase = static_cast<const T*>(prm.query);
-    Segment seg;
-    while (walker.next(seg)) {
+    Segment seg, nseg;
+    bool have = walker.next(seg);
+    int cur = 0;
+    if (have) {
+      const int32_t* bt = prm.block_table + (int64_t)seg.seq * prm.max_blocks_per_seq;
+      const int lb0 = seg.t0 / bs, nlb = (seg.t1 + bs - 1) / bs - lb0;
+      cur = lane < nlb ? __ldg(bt + lb0 + lane) : 0;
+    }
+    while (have) {
       const int32_t* bt = prm.block_table + (int64_t)seg.seq * prm.max_blocks_per_seq;
       const int lb0 = seg.t0 / bs;
       const int nlb = (seg.t1 + bs - 1) / bs - lb0;
-      int cur = lane < nlb ? __ldg(bt + lb0 + lane) : 0;
       int nxt = lane + 32 < nlb ? __ldg(bt + lb0 + 32 + lane) : 0;
+      const bool have_next = walker.next(nseg);
+      int ncur = 0;
+      if (have_next) {
+        const int32_t* nbt = prm.block_table + (int64_t)nseg.seq * prm.max_blocks_per_seq;
+        const int nlb0 = nseg.t0 / bs, nnlb = (nseg.t1 + bs - 1) / bs - nlb0;
+        ncur = lane < nnlb ? __ldg(nbt + nlb0 + lane) : 0;
+      }
       int batch = 0;
-      for (int c0 = seg.t0; c0 < seg.t1; c0 += kChunk) {
+      for (int c0 = seg.t0; c0 < seg.t1; c0 += kChunk, ++kc) {
+        const int stage = (int)(kc % NS);
+        const uint32_t phase = (kc / NS) & 1u;
         const int rel = (c0 - seg.t0) / bs;
         if (rel >= batch + 32) {
           cur = nxt;
@@ -246,22 +298,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_load(st + 2 * C::kKV, qbase + ((int64_t)seg.seq * Hq + seg.head * g) * D, qbytes,
                       full + stage);
         }
-        for (int b = 0; b < nblk; ++b) {
-          const int phys = __shfl_sync(0xffffffffu, cur, rel - batch + b);
+        __syncwarp();
+        // Lane rel - batch + b holds the id of the chunk's block b: those lanes
+        // issue their K and V tile copies together.
+        const int b = lane - (rel - batch);
+        if (ok && b >= 0 && b < nblk) {
+          tma_load_5d(st + b * tile, &tmap_k, 0, 0, 0, seg.head, cur, full + stage);
+          tma_load_5d(st + C::kKV + b * tile, &tmap_v, 0, 0, 0, seg.head, cur, full + stage);
+        }
+        if (kTeams > 1) {
+          __syncwarp();
           if (ok && lane == 0) {
-            tma_load_5d(st + b * tile, &tmap_k, 0, 0, 0, seg.head, phys, full + stage);
-            tma_load_5d(st + C::kKV + b * tile, &tmap_v, 0, 0, 0, seg.head, phys, full + stage);
+            __threadfence_block();
+            ticket[stage] = kc;
           }
         }
         if (ok) {
           armed |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
         }
-        if (++stage == NS) {
-          stage = 0;
-          phase ^= 1u;
-        }
       }
+      seg = nseg;
+      cur = ncur;
+      have = have_next;
     }
     // Wait, bounded, for this CTA's copies in flight before leaving.
     if (lane == 0) {
@@ -280,10 +339,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // -------------------------------------------------------------- consumers ----
-  const int w = warp;
+  // Team t takes segments t, t + 2, ...; within a segment its warp tw takes
+  // tokens [16 tw, 16 tw + 16) of every 64-token chunk.
+  const int team = warp / kTeamWarps, tw = warp % kTeamWarps;
+  const int tid_team = threadIdx.x - team * kTeamWarps * 32;
   const int g0 = lane >> 2, cq = lane & 3, x7 = lane & 7;
-  const int kt = 16 * w + ((lane >> 3) & 1) * 8 + x7;  // token row this lane addresses for K
-  const int vt = 16 * w + ((lane >> 4) & 1) * 8 + x7;  // ... and for V
+  const int kt = 16 * tw + ((lane >> 3) & 1) * 8 + x7;  // token row this lane addresses for K
+  const int vt = 16 * tw + ((lane >> 4) & 1) * 8 + x7;  // ... and for V
   const int kj = (lane >> 4) & 1, vj = (lane >> 3) & 1;
   const uint32_t krow = (uint32_t)((kt / bs) * tile + (kt % bs) * 128);
   const uint32_t vrow = (uint32_t)((vt / bs) * tile + (vt % bs) * 128);
@@ -291,11 +353,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t ring_u32 = smem_u32(ring);
   const float sscale = prm.score_scale;
   constexpr int MT = D / 16;
+  float* t_red_o = red_o + team * kTeamWarps * C::kHeads * D;
+  float* t_red_m = red_m + team * kTeamWarps * C::kHeads;
+  float* t_red_l = red_l + team * kTeamWarps * C::kHeads;
 
-  int stage = 0;
-  uint32_t phase = 0;
+  uint32_t kc = 0;
+  int segno = 0;
   Segment seg;
   while (walker.next(seg)) {
+    const int nch = (seg.t1 - seg.t0 + kChunk - 1) / kChunk;
+    if ((segno++ % kTeams) != team) {
+      kc += nch;
+      continue;
+    }
     float m[2 * NT], l[2 * NT];
     float o[MT][NT][4];
     uint32_t bq[MT][NT][2];
@@ -311,8 +381,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
 
-    for (int c0 = seg.t0; c0 < seg.t1; c0 += kChunk) {
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(full + stage, phase, abort));
+    for (int c0 = seg.t0; c0 < seg.t1; c0 += kChunk, ++kc) {
+      const int stage = (int)(kc % NS);
+      const uint32_t phase = (kc / NS) & 1u;
+      const bool ok = __all_sync(
+          0xffffffffu, (kTeams == 1 || wait_ticket(ticket + stage, kc, abort)) &&
+                           mbar_wait(full + stage, phase, abort));
       const uint32_t st = ring_u32 + stage * C::kStage;
       if (ok && c0 == seg.t0) {
         // Q^T fragments: b0b1 = Q[head g0][16ks + 2cq, +1], b2b3 = the same + 8 dims.
@@ -333,21 +407,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      const int nv = min(16, max(0, seg.t1 - (c0 + 16 * w)));
+      const int nv = min(16, max(0, seg.t1 - (c0 + 16 * tw)));
       if (ok && nv > 0) {
-        // S^T = K Q^T for this warp's 16 tokens.
-        float s[NT][4];
+        // S^T = K Q^T for this warp's 16 tokens; two accumulator chains.
+        float s[NT][4], s2[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
+          for (int e = 0; e < 4; ++e) s[nt][e] = s2[nt][e] = 0.f;
 #pragma unroll
         for (int ks = 0; ks < MT; ++ks) {
           uint32_t a[4];
           const int dh = ks >> 2, j = ((ks & 3) << 1) + kj;
           ldsm_x4(a, st + krow + dh * dh_stride + ((j ^ x7) << 4));
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) Mma<T>::run(s[nt], a, bq[ks][nt][0], bq[ks][nt][1]);
+          for (int nt = 0; nt < NT; ++nt) {
+            if (ks & 1)
+              Mma<T>::run(s2[nt], a, bq[ks][nt][0], bq[ks][nt][1]);
+            else
+              Mma<T>::run(s[nt], a, bq[ks][nt][0], bq[ks][nt][1]);
+          }
         }
         const bool v0 = g0 < nv, v1 = g0 + 8 < nv;
         uint32_t bp[NT][2];
@@ -356,8 +435,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           float alpha[2], p[2][2];
 #pragma unroll
           for (int hi = 0; hi < 2; ++hi) {
-            const float s0 = v0 ? s[nt][hi] * sscale : -INFINITY;
-            const float s1 = v1 ? s[nt][2 + hi] * sscale : -INFINITY;
+            const float s0 = v0 ? (s[nt][hi] + s2[nt][hi]) * sscale : -INFINITY;
+            const float s1 = v1 ? (s[nt][2 + hi] + s2[nt][2 + hi]) * sscale : -INFINITY;
             float mx = fmaxf(s0, s1);
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
@@ -375,12 +454,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t P1 = Mma<T>::pack(p[0][1], p[1][1], r10, r11);  // token g0 + 8
           l[nt * 2 + 0] = l[nt * 2 + 0] * alpha[0] + (r00 + r10);
           l[nt * 2 + 1] = l[nt * 2 + 1] * alpha[1] + (r01 + r11);
+          if (alpha[0] != 1.f || alpha[1] != 1.f) {
 #pragma unroll
-          for (int mt = 0; mt < MT; ++mt) {
-            o[mt][nt][0] *= alpha[0];
-            o[mt][nt][1] *= alpha[1];
-            o[mt][nt][2] *= alpha[0];
-            o[mt][nt][3] *= alpha[1];
+            for (int mt = 0; mt < MT; ++mt) {
+              o[mt][nt][0] *= alpha[0];
+              o[mt][nt][1] *= alpha[1];
+              o[mt][nt][2] *= alpha[0];
+              o[mt][nt][3] *= alpha[1];
+            }
           }
           bp[nt][0] = movmatrix_t(P0);
           bp[nt][1] = movmatrix_t(P1);
@@ -407,13 +488,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty + stage);
-      if (++stage == NS) {
-        stage = 0;
-        phase ^= 1u;
-      }
     }
 
-    // ---- segment epilogue: merge the four warps' states ----
+    // ---- segment epilogue: merge the team's four warp states ----
 #pragma unroll
     for (int x = 0; x < 2 * NT; ++x) {
       l[x] += __shfl_xor_sync(0xffffffffu, l[x], 4);
@@ -426,8 +503,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int hi = 0; hi < 2; ++hi) {
           const int head = nt * 8 + 2 * cq + hi;
-          red_m[w * C::kHeads + head] = m[nt * 2 + hi];
-          red_l[w * C::kHeads + head] = l[nt * 2 + hi];
+          t_red_m[tw * C::kHeads + head] = m[nt * 2 + hi];
+          t_red_l[tw * C::kHeads + head] = l[nt * 2 + hi];
         }
     }
 #pragma unroll
@@ -435,26 +512,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int h0 = nt * 8 + 2 * cq, d0 = mt * 16 + g0;
-        float* base = red_o + (w * C::kHeads) * D;
+        float* base = t_red_o + (tw * C::kHeads) * D;
         base[h0 * D + d0] = o[mt][nt][0];
         base[(h0 + 1) * D + d0] = o[mt][nt][1];
         base[h0 * D + d0 + 8] = o[mt][nt][2];
         base[(h0 + 1) * D + d0 + 8] = o[mt][nt][3];
       }
-    named_sync_consumers();
+    named_sync_team(team);
     const bool whole = seg.t0 == 0 && seg.t1 == seg.len;
     const int i = seg.seq, h = seg.head;
-    for (int e = threadIdx.x; e < g * D; e += kConsumerWarps * 32) {
+    for (int e = tid_team; e < g * D; e += kTeamWarps * 32) {
       const int j = e / D, d = e - j * D;
       float M = -INFINITY;
 #pragma unroll
-      for (int x = 0; x < kConsumerWarps; ++x) M = fmaxf(M, red_m[x * C::kHeads + j]);
+      for (int x = 0; x < kTeamWarps; ++x) M = fmaxf(M, t_red_m[x * C::kHeads + j]);
       float L = 0.f, O = 0.f;
 #pragma unroll
-      for (int x = 0; x < kConsumerWarps; ++x) {
-        const float wgt = fast_exp2(red_m[x * C::kHeads + j] - M);
-        L = fmaf(wgt, red_l[x * C::kHeads + j], L);
-        O = fmaf(wgt, red_o[(x * C::kHeads + j) * D + d], O);
+      for (int x = 0; x < kTeamWarps; ++x) {
+        const float wgt = fast_exp2(t_red_m[x * C::kHeads + j] - M);
+        L = fmaf(wgt, t_red_l[x * C::kHeads + j], L);
+        O = fmaf(wgt, t_red_o[(x * C::kHeads + j) * D + d], O);
       }
       const int qh = h * g + j;
       if (whole) {
@@ -465,11 +542,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (d == 0) prm.ws_lse[rowp] = M + fast_log2(L);
       }
     }
-    if (threadIdx.x == 0 && prm.part > 0) {
+    if (tid_team == 0 && prm.part > 0) {
       const int64_t u = (int64_t)i * Hkv + h;
       prm.ws_link[u * prm.max_parts + seg.t0 / prm.part] = (seg.t1 + prm.part - 1) / prm.part;
     }
-    named_sync_consumers();
+    named_sync_team(team);
   }
 }
 
@@ -508,17 +585,30 @@ static bool encode_pool_map(CUtensorMap* map, const void* base, CUtensorMapDataT
   return r == CUDA_SUCCESS;
 }
 
+// Returns the timeout word of the tensor-core kernel (1 if any bounded wait
+// expired), optionally clearing it. Synchronises the device.
+int tc_timeout_flag(bool clear, int* value) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_tc_timeout, sizeof(int)) != cudaSuccess) return -1;
+  if (clear && v) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_tc_timeout, &zero, sizeof(int)) != cudaSuccess) return -1;
+  }
+  *value = v;
+  return 0;
+}
+
 bool tc_supported(int q_dtype, int cache_dtype, int head_dim, int group) {
   return (q_dtype == PKV_BF16 || q_dtype == PKV_F16) && cache_dtype == q_dtype &&
          (head_dim == 64 || head_dim == 128) && group >= 1 && group <= 16;
 }
 
-template <typename T, int D, int NT, int NS>
+template <typename T, int D, int NT, int NS, int MINB>
 static cudaError_t launch_tc_t(const DecodeParams& prm, const CUtensorMap& mk,
                                const CUtensorMap& mv, int max_ctas, int num_sms,
                                cudaStream_t stream) {
   using C = tc::Cfg<D, NT, NS>;
-  auto kernel = tc::decode_tc_kernel<T, D, NT, NS>;
+  auto kernel = tc::decode_tc_kernel<T, D, NT, NS, MINB>;
   static int occ = 0;
   if (occ == 0) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -539,9 +629,13 @@ template <typename T, int D>
 static cudaError_t launch_tc_d(const DecodeParams& prm, const CUtensorMap& mk,
                                const CUtensorMap& mv, int max_ctas, int num_sms,
                                cudaStream_t stream) {
+  // Two CTAs per SM: two producers keep more copies in flight than one.
+  constexpr int kMinB = PKV_TC_CTAS_PER_SM;
+  constexpr int kNS1 = kMinB == 1 ? (D == 128 ? 5 : 8) : (D == 128 ? 2 : 4);
+  constexpr int kNS2 = kMinB == 1 ? (D == 128 ? 4 : 8) : (D == 128 ? 2 : 4);
   const int g = prm.num_heads / prm.num_kv_heads;
-  if (g <= 8) return launch_tc_t<T, D, 1, (D == 128 ? 5 : 8)>(prm, mk, mv, max_ctas, num_sms, stream);
-  return launch_tc_t<T, D, 2, (D == 128 ? 5 : 8)>(prm, mk, mv, max_ctas, num_sms, stream);
+  if (g <= 8) return launch_tc_t<T, D, 1, kNS1, kMinB>(prm, mk, mv, max_ctas, num_sms, stream);
+  return launch_tc_t<T, D, 2, kNS2, kMinB>(prm, mk, mv, max_ctas, num_sms, stream);
 }
 
 cudaError_t launch_decode_tc(const DecodeParams& prm, int q_dtype, int cache_dtype, int max_ctas,

@@ -15,6 +15,7 @@ bool tc_supported(int q_dtype, int cache_dtype, int head_dim, int group);
 cudaError_t launch_decode_tc(const DecodeParams& prm, int q_dtype, int cache_dtype,
                              int max_ctas, int num_sms, cudaStream_t stream);
 cudaError_t launch_merge(const DecodeParams& prm, int q_dtype, int num_sms, cudaStream_t stream);
+int tc_timeout_flag(bool clear, int* value);
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
@@ -61,6 +62,12 @@ using namespace pkv;
 extern "C" {
 
 int pkv_version(void) { return 100; }
+
+int pkv_device_status(int clear) {
+  int v = 0;
+  if (tc_timeout_flag(clear != 0, &v) != 0) return PKV_ERR_CUDA;
+  return v;
+}
 
 const char* pkv_status_string(int status) {
   switch (status) {

@@ -68,6 +68,7 @@ struct SegmentWalker {
   int64_t hi;    // first work offset of the next CTA
   int64_t base;  // work offset of sequence i
   int i, h, L;
+  int Lnext;     // raw seq_lens[i + 1], loaded one sequence ahead
   int64_t p;     // first partition of unit (i, h) still to take
   bool done;
 
@@ -79,7 +80,10 @@ struct SegmentWalker {
         ++i;
         h = 0;
         p = 0;
-        if (i < S) L = clamp_len(load_len(seq_lens + i), cap);
+        if (i < S) {
+          L = clamp_len(Lnext, cap);
+          Lnext = i + 1 < S ? load_len(seq_lens + i + 1) : 0;
+        }
         continue;
       }
       if (p * P >= L) { ++h; p = 0; continue; }  // unit started in an earlier CTA
@@ -190,6 +194,7 @@ __device__ void init_walker(const DecodeParams& prm, SchedShared& sh, SegmentWal
     w.i = S;
     w.h = 0;
     w.L = 0;
+    w.Lnext = 0;
     w.base = W;
     w.p = 0;
     return;
@@ -198,6 +203,7 @@ __device__ void init_walker(const DecodeParams& prm, SchedShared& sh, SegmentWal
   w.i = fi;
   w.base = sh.found_base;
   w.L = clamp_len(__ldg(prm.seq_lens + fi), cap);
+  w.Lnext = fi + 1 < S ? __ldg(prm.seq_lens + fi + 1) : 0;
   const int64_t rel = lo - w.base;
   w.h = (int)(rel / w.L);
   const int64_t r = rel - (int64_t)w.h * w.L;

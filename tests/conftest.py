@@ -41,3 +41,16 @@ def cuda_dev():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+@pytest.fixture(autouse=True)
+def _device_kernels_healthy(request):
+    """After every GPU test: no bounded wait inside a library kernel expired."""
+    yield
+    if request.node.get_closest_marker("gpu") is None:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    import paged_kv_cache_367_b200 as pkv
+    assert pkv.pkv_device_status(clear=True) == 0, "a device-side wait expired"

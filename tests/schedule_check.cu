@@ -24,12 +24,13 @@ static int check(const std::vector<int32_t>& lens, int Hkv, int cap, int part, i
     const int64_t lo = (W * c + G - 1) / G, hi = (W * (c + 1) + G - 1) / G;
     SegmentWalker w;
     w.seq_lens = lens.data(); w.S = S; w.Hkv = Hkv; w.cap = cap; w.P = P; w.hi = hi;
-    w.done = true; w.i = S; w.h = 0; w.L = 0; w.base = W; w.p = 0;
+    w.done = true; w.i = S; w.h = 0; w.L = 0; w.Lnext = 0; w.base = W; w.p = 0;
     int64_t base = 0;
     for (int i = 0; i < S && lo < hi; ++i) {
       const int L = clamp_len(lens[i], cap);
       if (L > 0 && base <= lo && lo < base + (int64_t)L * Hkv) {
         w.done = false; w.i = i; w.base = base; w.L = L;
+        w.Lnext = i + 1 < S ? lens[i + 1] : 0;
         const int64_t rel = lo - base;
         w.h = (int)(rel / L);
         const int64_t r = rel - (int64_t)w.h * L;
