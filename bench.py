@@ -3,8 +3,11 @@
 
 One step = one decode iteration of one attention layer over a batch of
 sequences: paged_kv_append of each sequence's new token, then
-paged_attention_decode (plus its log-sum-exp merge launch when sequences are
-split). Inputs are seeded synthetic tensors already resident in HBM.
+paged_attention_decode (a memset of its split counters and one kernel, which
+also merges split sequences by log-sum-exp). Inputs are seeded synthetic
+tensors already resident in HBM. The timed steps replay a CUDA graph of one
+step; the decode kernel's own time per launch is measured with CUDA events
+around eager launches.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gqa70b]
     python bench.py --impl reference ...    # the fp64 CPU oracle on host cores
@@ -66,6 +69,7 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-graph", action="store_true", help="time eager launches")
     return ap.parse_args()
 
 
@@ -196,8 +200,7 @@ def run_ours(args, rank, world, dev):
                                                   c.head_dim, msl, P)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev) if ws_bytes else None
     out = torch.empty_like(wl.query)
-    stream = torch.cuda.current_stream()
-    launches_per_step = 2 + (1 if P > 0 else 0)
+    launches_per_step = 2  # append kernel + decode kernel (plus a memset when split)
 
     def append(key, value, slot_t):
         pkv.paged_kv_append(key, value, wl.k_cache, wl.v_cache, slot_t, k_scale=ks, v_scale=vs)
@@ -207,31 +210,57 @@ def run_ours(args, rank, world, dev):
                                    scale=c.scale, partition_size=P, workspace=ws, k_scale=ks,
                                    v_scale=vs, max_ctas=args.max_ctas, flags=args.flags)
 
-    for _ in range(max(args.warmup, 3)):
+    def step():
         append(wl.new_key, wl.new_value, slots)
         decode(wl.query, bt, lens, out)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(max(args.warmup, 3)):
+            step()
+    torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
 
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
         t0.record(stream)
-        for k in range(K):
-            append(wl.new_key, wl.new_value, slots)
-            ev[k][0].record(stream)
-            decode(wl.query, bt, lens, out)
-            ev[k][1].record(stream)
+        for _ in range(K):
+            if graph is not None:
+                graph.replay()
+            else:
+                step()
         t1.record(stream)
         torch.cuda.synchronize()
     step_ms = t0.elapsed_time(t1) / K
-    decode_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
     if world > 1:
         torch.distributed.barrier()
+    # The decode kernel alone: CUDA events around eager launches of the same call.
+    KD = min(K, 200)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(KD)]
+    for k in range(KD):
+        append(wl.new_key, wl.new_value, slots)
+        ev[k][0].record(stream)
+        decode(wl.query, bt, lens, out)
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    decode_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    status = pkv.pkv_device_status(clear=True)
+    assert status == 0, f"device wait expired (status {status})"
 
     # End to end: per-step inputs start in pinned host memory, the output ends there.
     KE = args.e2e_steps or min(K, 200)
@@ -288,7 +317,7 @@ def run_ours(args, rank, world, dev):
         "pct_of_8TBs_nominal": round(100 * value / world / NOMINAL_HBM_GBS, 2),
         "decode_ms": round(decode_ms, 5),
         "bytes_per_step": {"decode": dec_b, "append": app_b},
-        "roofline": {"bound": "hbm", "kernel": "paged_attention_decode (decode + merge launches)",
+        "roofline": {"bound": "hbm", "kernel": "paged_attention_decode (counter memset + decode kernel)",
                      "achieved": round(achieved, 2), "peak": peak, "peak_source": peak_src,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": profiled_traffic(c.name)},
@@ -296,6 +325,7 @@ def run_ours(args, rank, world, dev):
                 "ms_per_step": round(e2e_ms, 5), "steps": KE, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": K * launches_per_step,
+        "timing": "CUDA graph replay of one step" if graph is not None else "eager launches",
         "clocks": clk.summary(),
         "source_sha": source_sha(),
     }

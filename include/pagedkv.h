@@ -94,8 +94,9 @@ int paged_kv_append(const void* key, const void* value, void* k_cache, void* v_c
 /*
  * Bytes of workspace paged_attention_decode needs for these sizes: zero when
  * partition_size is 0 (no split); otherwise room for one fp32 partial output
- * row, one log-sum-exp value and one int32 link per (sequence, query head,
- * partition), partitions = ceil(max_seq_len / partition_size).
+ * row and one log-sum-exp value per (sequence, query head, partition), one
+ * int32 link per (sequence, KV head, partition) and one int32 counter per
+ * (sequence, KV head), partitions = ceil(max_seq_len / partition_size).
  * Returns 0 for invalid sizes.
  */
 size_t paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_heads,
@@ -128,9 +129,11 @@ size_t paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_he
  *   partition_size  0: a sequence is never split. > 0 (a multiple of
  *                block_size): a sequence may be split at multiples of this many
  *                tokens; each piece yields a partial (output, log-sum-exp) in the
- *                workspace, and a second kernel merges the pieces by
- *                log-sum-exp. The split points are chosen on the device to
- *                balance work across the GPU.
+ *                workspace, and the CTA that finishes a sequence's last piece
+ *                merges the pieces by log-sum-exp. The split points are chosen
+ *                on the device to balance work across the GPU. The call then
+ *                enqueues a small memset of the workspace's counters and one
+ *                kernel; with partition_size 0, just the kernel.
  *   max_ctas     0: one resident wave of CTAs; > 0: at most this many CTAs (a
  *                tuning and testing knob)
  *   flags        PKV_DECODE_* bits

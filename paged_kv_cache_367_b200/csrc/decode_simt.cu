@@ -11,7 +11,8 @@
 // consecutive dimensions, so one K row is one coalesced 16-lane read. Up to 8
 // query heads are handled per pass over the K/V rows (more passes when g > 8).
 // The 8 half-warps keep separate softmax states, merged through shared memory
-// at the end of each segment. This kernel is the general path (fp32, mixed
+// at the end of each segment; pieces of split units are finished as in
+// schedule.cuh (finish_piece). This kernel is the general path (fp32, mixed
 // dtypes, wide groups); 16-bit caches at head_dim 64/128 use the tensor-core
 // kernel.
 #include "schedule.cuh"
@@ -27,6 +28,7 @@ struct SimtShared {
   float m[8][kSimtHeads];
   float l[8][kSimtHeads];
   float acc[8][kSimtHeads][D];
+  int flag;
 };
 
 template <typename QT, typename KT, int D>
@@ -166,12 +168,16 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(const DecodeP
           if (d == 0) prm.ws_lse[rowp] = M + fast_log2(L);
         }
       }
-      if (threadIdx.x == 0 && prm.part > 0 && hg == 0) {
-        // Link from this segment's first partition to the partition after it.
+      __syncthreads();
+    }
+    if (!(seg.t0 == 0 && seg.t1 == seg.len)) {
+      if (threadIdx.x == 0) {
+        // Link from this piece's first partition to the partition after it.
         const int64_t u = (int64_t)i * Hkv + h;
-        const int pe = (seg.t1 + prm.part - 1) / prm.part;
-        prm.ws_link[u * prm.max_parts + seg.t0 / prm.part] = pe;
+        prm.ws_link[u * prm.max_parts + seg.t0 / prm.part] = (seg.t1 + prm.part - 1) / prm.part;
       }
+      finish_piece<QT>(prm, i, h, seg.len, seg.t0, seg.t1, threadIdx.x, kSimtThreads, &sm.flag,
+                       [] { __syncthreads(); });
       __syncthreads();
     }
   }

@@ -25,7 +25,8 @@
 //    the B operand of O^T += V^T P^T, with V^T fed by ldmatrix.trans.
 //  * At the end of a segment the four warps' softmax states are merged through
 //    shared memory; a whole unit is written out directly, a piece of a split
-//    unit leaves a partial (output row, base-2 log-sum-exp) for the merge kernel.
+//    unit leaves a partial (output row, base-2 log-sum-exp), and the CTA that
+//    finishes a unit's last piece merges them (schedule.cuh, finish_piece).
 //  * Every mbarrier wait is bounded (about a second); on expiry the CTA sets an
 //    error word, skips the rest of its work and still waits, bounded, for its
 //    own copies in flight before it exits.
@@ -229,6 +230,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   SchedShared* sched = reinterpret_cast<SchedShared*>(
       reinterpret_cast<uint8_t*>(empty + NS) + ((NS * 4 + 7) & ~7));
   volatile int* abort = reinterpret_cast<volatile int*>(sched + 1);
+  volatile int* team_flag = abort + 1;  // one per team
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -542,9 +544,13 @@ __global__ void __launch_bounds__(kThreads, MINB)
         if (d == 0) prm.ws_lse[rowp] = M + fast_log2(L);
       }
     }
-    if (tid_team == 0 && prm.part > 0) {
-      const int64_t u = (int64_t)i * Hkv + h;
-      prm.ws_link[u * prm.max_parts + seg.t0 / prm.part] = (seg.t1 + prm.part - 1) / prm.part;
+    if (!whole) {
+      if (tid_team == 0) {
+        const int64_t u = (int64_t)i * Hkv + h;
+        prm.ws_link[u * prm.max_parts + seg.t0 / prm.part] = (seg.t1 + prm.part - 1) / prm.part;
+      }
+      finish_piece<T>(prm, i, h, seg.len, seg.t0, seg.t1, tid_team, kTeamWarps * 32,
+                      team_flag + team, [team] { named_sync_team(team); });
     }
     named_sync_team(team);
   }

@@ -14,7 +14,6 @@ cudaError_t launch_decode_simt(const DecodeParams& prm, int q_dtype, int cache_d
 bool tc_supported(int q_dtype, int cache_dtype, int head_dim, int group);
 cudaError_t launch_decode_tc(const DecodeParams& prm, int q_dtype, int cache_dtype,
                              int max_ctas, int num_sms, cudaStream_t stream);
-cudaError_t launch_merge(const DecodeParams& prm, int q_dtype, int num_sms, cudaStream_t stream);
 int tc_timeout_flag(bool clear, int* value);
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
@@ -35,7 +34,7 @@ static int num_sms_of_current_device(int* out) {
 }
 
 struct WsLayout {
-  size_t o, lse, link, total;
+  size_t o, lse, link, done, total;
 };
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -45,7 +44,8 @@ static WsLayout workspace_layout(int64_t S, int64_t Hq, int64_t Hkv, int64_t D, 
   w.o = 0;
   w.lse = align256(w.o + sizeof(float) * S * Hq * parts * D);
   w.link = align256(w.lse + sizeof(float) * S * Hq * parts);
-  w.total = align256(w.link + sizeof(int32_t) * S * Hkv * parts);
+  w.done = align256(w.link + sizeof(int32_t) * S * Hkv * parts);
+  w.total = align256(w.done + sizeof(int32_t) * S * Hkv);
   if (parts == 0) w.total = 0;
   return w;
 }
@@ -174,19 +174,21 @@ int paged_attention_decode(void* out, const void* query, const void* k_cache,
   prm.ws_o = parts ? reinterpret_cast<float*>(wsb + ws.o) : nullptr;
   prm.ws_lse = parts ? reinterpret_cast<float*>(wsb + ws.lse) : nullptr;
   prm.ws_link = parts ? reinterpret_cast<int*>(wsb + ws.link) : nullptr;
+  prm.ws_done = parts ? reinterpret_cast<int*>(wsb + ws.done) : nullptr;
 
   cudaStream_t st = (cudaStream_t)stream;
   const int group = num_heads / num_kv_heads;
   cudaError_t e;
+  if (parts > 0) {
+    // Per-unit counters of finished split tokens start at zero every call.
+    e = cudaMemsetAsync(prm.ws_done, 0, sizeof(int32_t) * (size_t)num_seqs * num_kv_heads, st);
+    if (e != cudaSuccess) return PKV_ERR_CUDA;
+  }
   if (!(flags & PKV_DECODE_FORCE_SIMT) && tc_supported(q_dtype, cache_dtype, head_dim, group))
     e = launch_decode_tc(prm, q_dtype, cache_dtype, max_ctas, sms, st);
   else
     e = launch_decode_simt(prm, q_dtype, cache_dtype, max_ctas, sms, st);
   if (e != cudaSuccess) return PKV_ERR_CUDA;
-  if (prm.part > 0) {
-    e = launch_merge(prm, q_dtype, sms, st);
-    if (e != cudaSuccess) return PKV_ERR_CUDA;
-  }
   return PKV_OK;
 }
 

@@ -9,7 +9,8 @@
 // of work and a contiguous run of items. Consecutive items of one unit in one
 // CTA form a segment and are processed as a single stream; a unit covered by
 // one segment is finished by that CTA, and a unit cut into several segments
-// leaves one partial (output row, log-sum-exp) per segment for the merge kernel.
+// leaves one partial (output row, log-sum-exp) per segment; the CTA that
+// finishes the last piece of a unit merges its partials (see finish_piece).
 //
 // The split needs no host knowledge of seq_lens: each CTA reads them (they are
 // small and L2-resident) to find its own range.
@@ -37,6 +38,7 @@ struct DecodeParams {
   float* ws_o;        // [num_seqs, num_heads, max_parts, head_dim]
   float* ws_lse;      // [num_seqs, num_heads, max_parts], base-2 log-sum-exp
   int* ws_link;       // [num_seqs, num_kv_heads, max_parts]: partition after a segment
+  int* ws_done;       // [num_seqs, num_kv_heads]: tokens of split units finished (zeroed per call)
 };
 
 constexpr int64_t kNoSplit = int64_t(1) << 30;
@@ -208,6 +210,60 @@ __device__ void init_walker(const DecodeParams& prm, SchedShared& sh, SegmentWal
   w.h = (int)(rel / w.L);
   const int64_t r = rel - (int64_t)w.h * w.L;
   w.p = (r + w.P - 1) / w.P;
+}
+
+// ---- pieces of split units -------------------------------------------------
+//
+// A segment that is not a whole unit writes its partial (per query head: the
+// normalised output row and the base-2 log-sum-exp of its scores) at partition
+// t0 / P, and links that partition to the partition after its last token. It
+// then adds its token count to the unit's counter; the CTA whose addition
+// completes the unit's length merges all pieces of the unit:
+//   M = max_p lse_p,  w_p = 2^(lse_p - M),  out = sum_p w_p o_p / sum_p w_p,
+// the blockwise form of the softmax. No CTA ever waits for another.
+
+// Called by `nthreads` threads (index tid) after they wrote the partial rows of
+// a piece [t0, t1) of unit (i, h) and the link of its first partition. `flag`
+// is a shared int private to these threads; `sync` synchronises them.
+template <typename OT, typename Sync>
+__device__ void finish_piece(const DecodeParams& prm, int i, int h, int L, int t0, int t1,
+                             int tid, int nthreads, volatile int* flag, Sync sync) {
+  __threadfence();
+  sync();
+  const int64_t u = (int64_t)i * prm.num_kv_heads + h;
+  if (tid == 0) {
+    const int before = atomicAdd(prm.ws_done + u, t1 - t0);
+    *flag = before + (t1 - t0) == L;
+  }
+  sync();
+  if (!*flag) return;
+  __threadfence();
+  const int Hq = prm.num_heads, g = Hq / prm.num_kv_heads, D = prm.head_dim;
+  const int MP = prm.max_parts, P = prm.part, nparts = (L + P - 1) / P;
+  const int* link = prm.ws_link + u * MP;
+  for (int e = tid; e < g * D; e += nthreads) {
+    const int j = e / D, d = e - j * D;
+    const int64_t row = ((int64_t)i * Hq + h * g + j) * MP;
+    float M = -INFINITY;
+    int p = 0;
+    for (int guard = 0; guard < nparts && p < nparts; ++guard) {
+      M = fmaxf(M, __ldcg(prm.ws_lse + row + p));
+      const int nx = __ldcg(link + p);
+      if (nx <= p) break;
+      p = nx;
+    }
+    float num = 0.f, den = 0.f;
+    p = 0;
+    for (int guard = 0; guard < nparts && p < nparts; ++guard) {
+      const float w = fast_exp2(__ldcg(prm.ws_lse + row + p) - M);
+      num = fmaf(w, __ldcg(prm.ws_o + (row + p) * D + d), num);
+      den += w;
+      const int nx = __ldcg(link + p);
+      if (nx <= p) break;
+      p = nx;
+    }
+    static_cast<OT*>(prm.out)[((int64_t)i * Hq + h * g + j) * D + d] = from_f32<OT>(num / den);
+  }
 }
 
 }  // namespace pkv
