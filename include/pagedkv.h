@@ -92,11 +92,12 @@ int paged_kv_append(const void* key, const void* value, void* k_cache, void* v_c
                     void* stream);
 
 /*
- * Bytes of workspace paged_attention_decode needs for these sizes: zero when
- * partition_size is 0 (no split); otherwise room for one fp32 partial output
- * row and one log-sum-exp value per (sequence, query head, partition), one
- * int32 link per (sequence, KV head, partition) and one int32 counter per
- * (sequence, KV head), partitions = ceil(max_seq_len / partition_size).
+ * Bytes of workspace paged_attention_decode needs for these sizes: zero when no
+ * sequence can be split (partition_size 0, or max_seq_len <= partition_size);
+ * otherwise room for the partial results of at most two pieces per CTA (up to
+ * 1024 CTAs), each num_heads / num_kv_heads fp32 rows of head_dim plus as many
+ * log-sum-exp values, and one int32 counter per (sequence, KV head). It does
+ * not grow with max_seq_len.
  * Returns 0 for invalid sizes.
  */
 size_t paged_attention_workspace_size(int num_seqs, int num_heads, int num_kv_heads,

@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(const DecodeP
         if (whole) {
           static_cast<QT*>(prm.out)[((int64_t)i * Hq + qh) * D + d] = from_f32<QT>(o);
         } else {
-          const int64_t rowp = ((int64_t)i * Hq + qh) * prm.max_parts + seg.t0 / prm.part;
+          const int64_t rowp = (int64_t)own_piece_slot(blockIdx.x, seg) * g + hg + j;
           prm.ws_o[rowp * D + d] = o;
           if (d == 0) prm.ws_lse[rowp] = M + fast_log2(L);
         }
@@ -171,12 +171,7 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(const DecodeP
       __syncthreads();
     }
     if (!(seg.t0 == 0 && seg.t1 == seg.len)) {
-      if (threadIdx.x == 0) {
-        // Link from this piece's first partition to the partition after it.
-        const int64_t u = (int64_t)i * Hkv + h;
-        prm.ws_link[u * prm.max_parts + seg.t0 / prm.part] = (seg.t1 + prm.part - 1) / prm.part;
-      }
-      finish_piece<QT>(prm, i, h, seg.len, seg.t0, seg.t1, threadIdx.x, kSimtThreads, &sm.flag,
+      finish_piece<QT>(prm, walker, seg, threadIdx.x, kSimtThreads, &sm.flag,
                        [] { __syncthreads(); });
       __syncthreads();
     }
@@ -202,6 +197,7 @@ static cudaError_t launch_simt_t(const DecodeParams& prm, int max_ctas, int num_
   int& occ = prm.head_dim == 64 ? occ64 : occ128;
   if (occ == 0) occ = resident_ctas(kernel, kSimtThreads, 0);
   int grid = occ * num_sms;
+  if (grid > kMaxCtas) grid = kMaxCtas;
   if (max_ctas > 0 && max_ctas < grid) grid = max_ctas;
   kernel<<<grid, kSimtThreads, 0, stream>>>(prm);
   return cudaGetLastError();

@@ -23,10 +23,13 @@
 //    and avoiding per-element conversions and cross-lane dot-product reductions.
 //    P is rounded to the cache dtype, transposed in registers (movmatrix) into
 //    the B operand of O^T += V^T P^T, with V^T fed by ldmatrix.trans.
-//  * At the end of a segment the four warps' softmax states are merged through
-//    shared memory; a whole unit is written out directly, a piece of a split
-//    unit leaves a partial (output row, base-2 log-sum-exp), and the CTA that
-//    finishes a unit's last piece merges them (schedule.cuh, finish_piece).
+//  * At the end of a segment each consumer warp drops its softmax state
+//    (running max, sum, O^T) into one of two shared hand-off buffers and moves
+//    on to the next segment. An epilogue warp combines the four states, writes
+//    the output rows of a whole unit or the partial (output row, base-2
+//    log-sum-exp) of a piece of a split unit, and merges a split unit when its
+//    piece is the last to finish (a per-unit counter of finished tokens; no
+//    CTA waits for another). The epilogue is thus off the streaming path.
 //  * Every mbarrier wait is bounded (about a second); on expiry the CTA sets an
 //    error word, skips the rest of its work and still waits, bounded, for its
 //    own copies in flight before it exits.
@@ -41,30 +44,24 @@ __device__ int g_tc_timeout = 0;
 
 namespace tc {
 
-constexpr int kChunk = 64;          // tokens per stage
-constexpr int kTeamWarps = 4;       // a team takes a chunk: 16 tokens per warp
-#ifndef PKV_TC_TEAMS
-#define PKV_TC_TEAMS 1
-#endif
-constexpr int kTeams = PKV_TC_TEAMS;  // teams take alternate segments
-#ifndef PKV_TC_CTAS_PER_SM
-#define PKV_TC_CTAS_PER_SM 2
-#endif
-constexpr int kConsumerWarps = kTeams * kTeamWarps;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr long long kWaitCycles = 1ll << 31;  // ~1 s at 2 GHz
+constexpr int kChunk = 64;                           // tokens per stage
+constexpr int kConsumerWarps = 4;                    // 16 tokens of a chunk each
+constexpr int kProducerWarp = kConsumerWarps;        // TMA issue
+constexpr int kEpilogueWarp = kConsumerWarps + 1;    // combine, store, merge
+constexpr int kThreads = (kConsumerWarps + 2) * 32;
+constexpr long long kWaitCycles = 1ll << 31;         // ~1 s at 2 GHz
 
 template <int D, int NT, int NS>
 struct Cfg {
-  static constexpr int kKV = kChunk * D * 2;       // bytes of K (or V) per stage
-  static constexpr int kQ = 8 * NT * D * 2;        // query rows of one KV head group
+  static constexpr int kKV = kChunk * D * 2;         // bytes of K (or V) per stage
+  static constexpr int kQ = 8 * NT * D * 2;          // query rows of one KV head group
   static constexpr int kStage = (2 * kKV + kQ + 1023) / 1024 * 1024;
   static constexpr int kHeads = 8 * NT;
-  static constexpr int kRedO = kConsumerWarps * kHeads * D * 4;   // per team: 4 warps
-  static constexpr int kRedML = 2 * kConsumerWarps * kHeads * 4;
-  static constexpr int kBar = 2 * NS * 8 + NS * 4;  // full/empty barriers, stage tickets
-  static constexpr int kSmem = 1024 + NS * kStage + kRedO + kRedML + kBar +
-                               (int)sizeof(SchedShared) + 16;
+  static constexpr int kRedO = kConsumerWarps * kHeads * D;   // floats per hand-off buffer
+  static constexpr int kRed = (kRedO + 2 * kConsumerWarps * kHeads) * 4;
+  static constexpr int kBar = (2 * NS + 4) * 8;
+  static constexpr int kSmem = 1024 + NS * kStage + 2 * kRed + kBar +
+                               (int)sizeof(SchedShared) + 32;
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA exceeds 227 KB");
 };
 
@@ -113,26 +110,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       }
     }
   }
-}
-
-// Bounded wait until the producer has armed stage `ticket` for chunk kc.
-__device__ __forceinline__ bool wait_ticket(volatile uint32_t* ticket, uint32_t kc,
-                                            volatile int* abort) {
-  if (*abort) return false;
-  const long long t0 = clock64();
-  for (int it = 1; *ticket != kc; ++it) {
-    __nanosleep(32);
-    if ((it & 31) == 0) {
-      if (*abort) return false;
-      if (clock64() - t0 > kWaitCycles) {
-        *abort = 1;
-        atomicExch(&g_tc_timeout, 1);
-        return false;
-      }
-    }
-  }
-  __threadfence_block();
-  return true;
 }
 
 __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
@@ -205,8 +182,50 @@ template <> struct Mma<__half> {
   }
 };
 
-__device__ __forceinline__ void named_sync_team(int team) {
-  asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "n"(kTeamWarps * 32) : "memory");
+__device__ __forceinline__ void named_sync_consumers() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+}
+
+// Merge of all pieces of a split unit by one warp: lane j < g owns head j's
+// log-sum-exp bookkeeping, every lane owns D/32 dimensions of every head. The
+// pieces are enumerated from the schedule, so their loads are independent.
+template <typename T, int D, int NT>
+__device__ void warp_merge_unit(const DecodeParams& prm, const SegmentWalker& wk,
+                                const Segment& s, int lane) {
+  constexpr int V = D / 32;
+  const int Hq = prm.num_heads, g = Hq / prm.num_kv_heads;
+  float M = -INFINITY;
+  wk.for_each_piece(s.first, s.len, [&](int slot) {
+    if (lane < g) M = fmaxf(M, __ldcg(prm.ws_lse + (int64_t)slot * g + lane));
+  });
+  float num[8 * NT][V];
+#pragma unroll
+  for (int j = 0; j < 8 * NT; ++j)
+#pragma unroll
+    for (int v = 0; v < V; ++v) num[j][v] = 0.f;
+  float den = 0.f;
+  wk.for_each_piece(s.first, s.len, [&](int slot) {
+    const float w = lane < g ? fast_exp2(__ldcg(prm.ws_lse + (int64_t)slot * g + lane) - M) : 0.f;
+    den += w;
+#pragma unroll
+    for (int j = 0; j < 8 * NT; ++j) {
+      const float wj = __shfl_sync(0xffffffffu, w, j);
+      if (j < g) {
+        const float* src = prm.ws_o + ((int64_t)slot * g + j) * D + lane * V;
+#pragma unroll
+        for (int v = 0; v < V; ++v) num[j][v] = fmaf(wj, __ldcg(src + v), num[j][v]);
+      }
+    }
+  });
+#pragma unroll
+  for (int j = 0; j < 8 * NT; ++j) {
+    const float dj = __shfl_sync(0xffffffffu, den, j);
+    if (j < g) {
+      T* dst = static_cast<T*>(prm.out) + ((int64_t)s.seq * Hq + s.head * g + j) * D + lane * V;
+#pragma unroll
+      for (int v = 0; v < V; ++v) dst[v] = from_f32<T>(num[j][v] / dj);
+    }
+  }
 }
 
 template <typename T, int D, int NT, int NS, int MINB>
@@ -214,29 +233,27 @@ __global__ void __launch_bounds__(kThreads, MINB)
     decode_tc_kernel(const DecodeParams prm, const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v) {
   using C = Cfg<D, NT, NS>;
+  constexpr int H = C::kHeads;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* ring = smem;
-  float* red_o = reinterpret_cast<float*>(smem + NS * C::kStage);
-  float* red_m = red_o + kConsumerWarps * C::kHeads * D;
-  float* red_l = red_m + kConsumerWarps * C::kHeads;
-  uint64_t* full = reinterpret_cast<uint64_t*>(red_l + kConsumerWarps * C::kHeads);
+  float* red = reinterpret_cast<float*>(smem + NS * C::kStage);  // 2 hand-off buffers
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + NS * C::kStage + 2 * C::kRed);
   uint64_t* empty = full + NS;
-  // ticket[s] = number of the chunk the producer last armed stage s for. A team
-  // may be several ring laps ahead of the other, so it first waits for the
-  // ticket of its chunk; after that the parity wait on full[s] is unambiguous.
-  volatile uint32_t* ticket = reinterpret_cast<volatile uint32_t*>(empty + NS);
-  SchedShared* sched = reinterpret_cast<SchedShared*>(
-      reinterpret_cast<uint8_t*>(empty + NS) + ((NS * 4 + 7) & ~7));
+  uint64_t* rfull = empty + NS;    // consumers -> epilogue warp, per hand-off buffer
+  uint64_t* rempty = rfull + 2;    // epilogue warp -> consumers
+  SchedShared* sched = reinterpret_cast<SchedShared*>(rempty + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(sched + 1);
-  volatile int* team_flag = abort + 1;  // one per team
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(full + s, 1);
-      mbar_init(empty + s, kTeamWarps);  // each chunk is consumed by one team
-      ticket[s] = 0xffffffffu;
+      mbar_init(empty + s, kConsumerWarps);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(rfull + b, kConsumerWarps * 32);
+      mbar_init(rempty + b, 32);
     }
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -249,10 +266,11 @@ __global__ void __launch_bounds__(kThreads, MINB)
   const int Hq = prm.num_heads, Hkv = prm.num_kv_heads, g = Hq / Hkv, bs = prm.block_size;
   const int tile = bs * D * 2;  // bytes of one (block, head) tile
 
-  if (warp == kConsumerWarps) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer ----
     // Streams the chunks of every segment, in order, into the ring. The block
-    // ids of the next segment are loaded while the current one is issued.
+    // ids of the next segment are loaded while the current one is issued; the
+    // lane holding a block's id issues that block's K and V tile copies.
     uint32_t kc = 0;  // chunk counter: stage kc % NS, phase (kc / NS) & 1
     uint32_t armed = 0, last_parity = 0;
     bool ok = true;
@@ -301,19 +319,10 @@ __global__ void __launch_bounds__(kThreads, MINB)
                       full + stage);
         }
         __syncwarp();
-        // Lane rel - batch + b holds the id of the chunk's block b: those lanes
-        // issue their K and V tile copies together.
         const int b = lane - (rel - batch);
         if (ok && b >= 0 && b < nblk) {
           tma_load_5d(st + b * tile, &tmap_k, 0, 0, 0, seg.head, cur, full + stage);
           tma_load_5d(st + C::kKV + b * tile, &tmap_v, 0, 0, 0, seg.head, cur, full + stage);
-        }
-        if (kTeams > 1) {
-          __syncwarp();
-          if (ok && lane == 0) {
-            __threadfence_block();
-            ticket[stage] = kc;
-          }
         }
         if (ok) {
           armed |= 1u << stage;
@@ -340,14 +349,93 @@ __global__ void __launch_bounds__(kThreads, MINB)
     return;
   }
 
+  if (warp == kEpilogueWarp) {
+    // ------------------------------------------------------------ epilogue ----
+    // For every segment: combine the four consumer warps' softmax states from
+    // the hand-off buffer, write the output rows (whole unit) or the partial
+    // and link (piece of a split unit), release the buffer, and merge the unit
+    // if this piece completed it.
+    constexpr int V = D / 32;
+    int sidx = 0;
+    Segment seg;
+    while (walker.next(seg)) {
+      const int rb = sidx & 1;
+      const uint32_t use = (uint32_t)(sidx >> 1);
+      ++sidx;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(rfull + rb, use & 1u, abort));
+      const float* ro = red + rb * (C::kRed / 4);
+      const float* rm = ro + C::kRedO;
+      const float* rl = rm + kConsumerWarps * H;
+      const bool whole = seg.t0 == 0 && seg.t1 == seg.len;
+      const int i = seg.seq, h = seg.head;
+      if (ok) {
+        // lane j < g: per-head maximum, warp weights and denominator
+        float M = -INFINITY, wx[kConsumerWarps], Lsum = 0.f;
+        if (lane < g) {
+#pragma unroll
+          for (int x = 0; x < kConsumerWarps; ++x) M = fmaxf(M, rm[x * H + lane]);
+#pragma unroll
+          for (int x = 0; x < kConsumerWarps; ++x) {
+            wx[x] = fast_exp2(rm[x * H + lane] - M);
+            Lsum = fmaf(wx[x], rl[x * H + lane], Lsum);
+          }
+        } else {
+#pragma unroll
+          for (int x = 0; x < kConsumerWarps; ++x) wx[x] = 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < H; ++j) {
+          float w[kConsumerWarps];
+#pragma unroll
+          for (int x = 0; x < kConsumerWarps; ++x) w[x] = __shfl_sync(0xffffffffu, wx[x], j);
+          const float Lj = __shfl_sync(0xffffffffu, Lsum, j);
+          const float Mj = __shfl_sync(0xffffffffu, M, j);
+          if (j < g) {
+            float o[V];
+#pragma unroll
+            for (int v = 0; v < V; ++v) o[v] = 0.f;
+#pragma unroll
+            for (int x = 0; x < kConsumerWarps; ++x) {
+              const float* src = ro + (x * H + j) * D + lane * V;
+#pragma unroll
+              for (int v = 0; v < V; ++v) o[v] = fmaf(w[x], src[v], o[v]);
+            }
+            const int qh = h * g + j;
+            if (whole) {
+              T* dst = static_cast<T*>(prm.out) + ((int64_t)i * Hq + qh) * D + lane * V;
+#pragma unroll
+              for (int v = 0; v < V; ++v) dst[v] = from_f32<T>(o[v] / Lj);
+            } else {
+              const int64_t rowp = (int64_t)own_piece_slot(blockIdx.x, seg) * g + j;
+              float* dst = prm.ws_o + rowp * D + lane * V;
+#pragma unroll
+              for (int v = 0; v < V; ++v) dst[v] = o[v] / Lj;
+              if (lane == 0) prm.ws_lse[rowp] = Mj + fast_log2(Lj);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      mbar_arrive(rempty + rb);  // the hand-off buffer may be refilled
+      if (ok && !whole) {
+        __threadfence();
+        __syncwarp();
+        const int last = lane == 0 ? (int)complete_piece(prm, seg) : 0;
+        if (__shfl_sync(0xffffffffu, last, 0)) {
+          __threadfence();
+          warp_merge_unit<T, D, NT>(prm, walker, seg, lane);
+        }
+      }
+    }
+    return;
+  }
+
   // -------------------------------------------------------------- consumers ----
-  // Team t takes segments t, t + 2, ...; within a segment its warp tw takes
-  // tokens [16 tw, 16 tw + 16) of every 64-token chunk.
-  const int team = warp / kTeamWarps, tw = warp % kTeamWarps;
-  const int tid_team = threadIdx.x - team * kTeamWarps * 32;
+  // Warp w takes tokens [16 w, 16 w + 16) of every 64-token chunk.
+  const int w = warp;
   const int g0 = lane >> 2, cq = lane & 3, x7 = lane & 7;
-  const int kt = 16 * tw + ((lane >> 3) & 1) * 8 + x7;  // token row this lane addresses for K
-  const int vt = 16 * tw + ((lane >> 4) & 1) * 8 + x7;  // ... and for V
+  const int kt = 16 * w + ((lane >> 3) & 1) * 8 + x7;  // token row this lane addresses for K
+  const int vt = 16 * w + ((lane >> 4) & 1) * 8 + x7;  // ... and for V
   const int kj = (lane >> 4) & 1, vj = (lane >> 3) & 1;
   const uint32_t krow = (uint32_t)((kt / bs) * tile + (kt % bs) * 128);
   const uint32_t vrow = (uint32_t)((vt / bs) * tile + (vt % bs) * 128);
@@ -355,19 +443,11 @@ __global__ void __launch_bounds__(kThreads, MINB)
   const uint32_t ring_u32 = smem_u32(ring);
   const float sscale = prm.score_scale;
   constexpr int MT = D / 16;
-  float* t_red_o = red_o + team * kTeamWarps * C::kHeads * D;
-  float* t_red_m = red_m + team * kTeamWarps * C::kHeads;
-  float* t_red_l = red_l + team * kTeamWarps * C::kHeads;
 
   uint32_t kc = 0;
-  int segno = 0;
+  int sidx = 0;
   Segment seg;
   while (walker.next(seg)) {
-    const int nch = (seg.t1 - seg.t0 + kChunk - 1) / kChunk;
-    if ((segno++ % kTeams) != team) {
-      kc += nch;
-      continue;
-    }
     float m[2 * NT], l[2 * NT];
     float o[MT][NT][4];
     uint32_t bq[MT][NT][2];
@@ -386,9 +466,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
     for (int c0 = seg.t0; c0 < seg.t1; c0 += kChunk, ++kc) {
       const int stage = (int)(kc % NS);
       const uint32_t phase = (kc / NS) & 1u;
-      const bool ok = __all_sync(
-          0xffffffffu, (kTeams == 1 || wait_ticket(ticket + stage, kc, abort)) &&
-                           mbar_wait(full + stage, phase, abort));
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(full + stage, phase, abort));
       const uint32_t st = ring_u32 + stage * C::kStage;
       if (ok && c0 == seg.t0) {
         // Q^T fragments: b0b1 = Q[head g0][16ks + 2cq, +1], b2b3 = the same + 8 dims.
@@ -409,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
           }
         }
       }
-      const int nv = min(16, max(0, seg.t1 - (c0 + 16 * tw)));
+      const int nv = min(16, max(0, seg.t1 - (c0 + 16 * w)));
       if (ok && nv > 0) {
         // S^T = K Q^T for this warp's 16 tokens; two accumulator chains.
         float s[NT][4], s2[NT][4];
@@ -492,21 +570,29 @@ __global__ void __launch_bounds__(kThreads, MINB)
       if (lane == 0) mbar_arrive(empty + stage);
     }
 
-    // ---- segment epilogue: merge the team's four warp states ----
+    // ---- hand the warp's state to the epilogue warp ----
 #pragma unroll
     for (int x = 0; x < 2 * NT; ++x) {
       l[x] += __shfl_xor_sync(0xffffffffu, l[x], 4);
       l[x] += __shfl_xor_sync(0xffffffffu, l[x], 8);
       l[x] += __shfl_xor_sync(0xffffffffu, l[x], 16);
     }
+    const int rb = sidx & 1;
+    const uint32_t use = (uint32_t)(sidx >> 1);
+    ++sidx;
+    // The buffer's previous contents (two segments ago) must have been read.
+    mbar_wait(rempty + rb, (use & 1u) ^ 1u, abort);
+    float* ro = red + rb * (C::kRed / 4) + (w * H) * D;
+    float* rm = red + rb * (C::kRed / 4) + C::kRedO;
+    float* rl = rm + kConsumerWarps * H;
     if (g0 == 0) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int hi = 0; hi < 2; ++hi) {
           const int head = nt * 8 + 2 * cq + hi;
-          t_red_m[tw * C::kHeads + head] = m[nt * 2 + hi];
-          t_red_l[tw * C::kHeads + head] = l[nt * 2 + hi];
+          rm[w * H + head] = m[nt * 2 + hi];
+          rl[w * H + head] = l[nt * 2 + hi];
         }
     }
 #pragma unroll
@@ -514,45 +600,12 @@ __global__ void __launch_bounds__(kThreads, MINB)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int h0 = nt * 8 + 2 * cq, d0 = mt * 16 + g0;
-        float* base = t_red_o + (tw * C::kHeads) * D;
-        base[h0 * D + d0] = o[mt][nt][0];
-        base[(h0 + 1) * D + d0] = o[mt][nt][1];
-        base[h0 * D + d0 + 8] = o[mt][nt][2];
-        base[(h0 + 1) * D + d0 + 8] = o[mt][nt][3];
+        ro[h0 * D + d0] = o[mt][nt][0];
+        ro[(h0 + 1) * D + d0] = o[mt][nt][1];
+        ro[h0 * D + d0 + 8] = o[mt][nt][2];
+        ro[(h0 + 1) * D + d0 + 8] = o[mt][nt][3];
       }
-    named_sync_team(team);
-    const bool whole = seg.t0 == 0 && seg.t1 == seg.len;
-    const int i = seg.seq, h = seg.head;
-    for (int e = tid_team; e < g * D; e += kTeamWarps * 32) {
-      const int j = e / D, d = e - j * D;
-      float M = -INFINITY;
-#pragma unroll
-      for (int x = 0; x < kTeamWarps; ++x) M = fmaxf(M, t_red_m[x * C::kHeads + j]);
-      float L = 0.f, O = 0.f;
-#pragma unroll
-      for (int x = 0; x < kTeamWarps; ++x) {
-        const float wgt = fast_exp2(t_red_m[x * C::kHeads + j] - M);
-        L = fmaf(wgt, t_red_l[x * C::kHeads + j], L);
-        O = fmaf(wgt, t_red_o[(x * C::kHeads + j) * D + d], O);
-      }
-      const int qh = h * g + j;
-      if (whole) {
-        static_cast<T*>(prm.out)[((int64_t)i * Hq + qh) * D + d] = from_f32<T>(O / L);
-      } else {
-        const int64_t rowp = ((int64_t)i * Hq + qh) * prm.max_parts + seg.t0 / prm.part;
-        prm.ws_o[rowp * D + d] = O / L;
-        if (d == 0) prm.ws_lse[rowp] = M + fast_log2(L);
-      }
-    }
-    if (!whole) {
-      if (tid_team == 0) {
-        const int64_t u = (int64_t)i * Hkv + h;
-        prm.ws_link[u * prm.max_parts + seg.t0 / prm.part] = (seg.t1 + prm.part - 1) / prm.part;
-      }
-      finish_piece<T>(prm, i, h, seg.len, seg.t0, seg.t1, tid_team, kTeamWarps * 32,
-                      team_flag + team, [team] { named_sync_team(team); });
-    }
-    named_sync_team(team);
+    mbar_arrive(rfull + rb);
   }
 }
 
@@ -626,6 +679,7 @@ static cudaError_t launch_tc_t(const DecodeParams& prm, const CUtensorMap& mk,
     occ = n > 0 ? n : 1;
   }
   int grid = occ * num_sms;
+  if (grid > kMaxCtas) grid = kMaxCtas;
   if (max_ctas > 0 && max_ctas < grid) grid = max_ctas;
   kernel<<<grid, tc::kThreads, C::kSmem, stream>>>(prm, mk, mv);
   return cudaGetLastError();
@@ -635,13 +689,12 @@ template <typename T, int D>
 static cudaError_t launch_tc_d(const DecodeParams& prm, const CUtensorMap& mk,
                                const CUtensorMap& mv, int max_ctas, int num_sms,
                                cudaStream_t stream) {
-  // Two CTAs per SM: two producers keep more copies in flight than one.
-  constexpr int kMinB = PKV_TC_CTAS_PER_SM;
-  constexpr int kNS1 = kMinB == 1 ? (D == 128 ? 5 : 8) : (D == 128 ? 2 : 4);
-  constexpr int kNS2 = kMinB == 1 ? (D == 128 ? 4 : 8) : (D == 128 ? 2 : 4);
+  // Two CTAs per SM (two producers keep more copies in flight than one) where
+  // shared memory allows; head_dim 128 with more than 8 heads per group runs one.
   const int g = prm.num_heads / prm.num_kv_heads;
-  if (g <= 8) return launch_tc_t<T, D, 1, kNS1, kMinB>(prm, mk, mv, max_ctas, num_sms, stream);
-  return launch_tc_t<T, D, 2, kNS2, kMinB>(prm, mk, mv, max_ctas, num_sms, stream);
+  if (g <= 8) return launch_tc_t<T, D, 1, (D == 128 ? 2 : 4), 2>(prm, mk, mv, max_ctas, num_sms, stream);
+  if (D == 64) return launch_tc_t<T, D, 2, 4, 2>(prm, mk, mv, max_ctas, num_sms, stream);
+  return launch_tc_t<T, D, 2, 4, 1>(prm, mk, mv, max_ctas, num_sms, stream);
 }
 
 cudaError_t launch_decode_tc(const DecodeParams& prm, int q_dtype, int cache_dtype, int max_ctas,

@@ -34,19 +34,21 @@ static int num_sms_of_current_device(int* out) {
 }
 
 struct WsLayout {
-  size_t o, lse, link, done, total;
+  size_t o, lse, done, total;
 };
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Partials: two slots per CTA of up to kMaxCtas, each g rows of D floats plus g
+// log-sum-exp values; one counter per (sequence, KV head).
 static WsLayout workspace_layout(int64_t S, int64_t Hq, int64_t Hkv, int64_t D, int64_t parts) {
   WsLayout w;
+  const int64_t g = Hq / Hkv, slots = 2 * (int64_t)kMaxCtas;
   w.o = 0;
-  w.lse = align256(w.o + sizeof(float) * S * Hq * parts * D);
-  w.link = align256(w.lse + sizeof(float) * S * Hq * parts);
-  w.done = align256(w.link + sizeof(int32_t) * S * Hkv * parts);
+  w.lse = align256(w.o + sizeof(float) * slots * g * D);
+  w.done = align256(w.lse + sizeof(float) * slots * g);
   w.total = align256(w.done + sizeof(int32_t) * S * Hkv);
-  if (parts == 0) w.total = 0;
+  if (parts <= 1) w.total = 0;  // no sequence can be cut
   return w;
 }
 
@@ -165,21 +167,20 @@ int paged_attention_decode(void* out, const void* query, const void* k_cache,
   prm.num_blocks = num_blocks;
   const int64_t cap = (int64_t)max_blocks_per_seq * block_size;
   prm.len_cap = (int)(cap < max_seq_len ? cap : max_seq_len);
-  prm.part = parts > 0 ? partition_size : 0;
-  prm.max_parts = (int)parts;
+  prm.part = parts > 1 ? partition_size : 0;
+  prm.unit_cost = 64;  // about one chunk: a segment's set-up and epilogue, in tokens
   prm.score_scale = scale * kLog2e;
   prm.k_scale = k_scale;
   prm.v_scale = v_scale;
   char* wsb = static_cast<char*>(workspace);
-  prm.ws_o = parts ? reinterpret_cast<float*>(wsb + ws.o) : nullptr;
-  prm.ws_lse = parts ? reinterpret_cast<float*>(wsb + ws.lse) : nullptr;
-  prm.ws_link = parts ? reinterpret_cast<int*>(wsb + ws.link) : nullptr;
-  prm.ws_done = parts ? reinterpret_cast<int*>(wsb + ws.done) : nullptr;
+  prm.ws_o = ws.total ? reinterpret_cast<float*>(wsb + ws.o) : nullptr;
+  prm.ws_lse = ws.total ? reinterpret_cast<float*>(wsb + ws.lse) : nullptr;
+  prm.ws_done = ws.total ? reinterpret_cast<int*>(wsb + ws.done) : nullptr;
 
   cudaStream_t st = (cudaStream_t)stream;
   const int group = num_heads / num_kv_heads;
   cudaError_t e;
-  if (parts > 0) {
+  if (ws.total > 0) {
     // Per-unit counters of finished split tokens start at zero every call.
     e = cudaMemsetAsync(prm.ws_done, 0, sizeof(int32_t) * (size_t)num_seqs * num_kv_heads, st);
     if (e != cudaSuccess) return PKV_ERR_CUDA;

@@ -83,8 +83,8 @@ def append(lib, **kw):
     (dict(block_size=64), EUNSUP), (dict(q_dtype=FP8, cache_dtype=FP8), EDTYPE),
     (dict(q_dtype=7), EDTYPE), (dict(q_dtype=BF16, cache_dtype=F16), EDTYPE),
     (dict(out=A + 8), EALIGN), (dict(k_cache=A + 4), EALIGN), (dict(seq_lens=A + 2), EALIGN),
-    (dict(partition_size=512), EWS),
-    (dict(partition_size=512, workspace=A, workspace_bytes=100), EWS),
+    (dict(partition_size=512, max_seq_len=1000), EWS),
+    (dict(partition_size=512, max_seq_len=1000, workspace=A, workspace_bytes=100), EWS),
     (dict(num_seqs=0, out=None), OK),
 ])
 def test_decode_rejects_bad_arguments_on_the_host(lib, kw, code):
@@ -94,10 +94,12 @@ def test_decode_rejects_bad_arguments_on_the_host(lib, kw, code):
 def test_workspace_size(lib):
     ws = lib.paged_attention_workspace_size
     assert ws(4, 8, 2, 128, 128, 0) == 0
-    parts = -(-1000 // 512)
+    assert ws(4, 8, 2, 128, 512, 512) == 0          # nothing can be cut
     need = ws(4, 8, 2, 128, 1000, 512)
-    assert need >= 4 * 8 * parts * (128 + 1) * 4 + 4 * 2 * parts * 4
+    g = 8 // 2
+    assert need >= 2 * 1024 * g * (128 + 1) * 4 + 4 * 2 * 4   # two slots per CTA + counters
     assert need % 256 == 0
+    assert ws(4, 8, 2, 128, 100000, 512) == need     # independent of max_seq_len
     assert ws(-1, 8, 2, 128, 1000, 512) == 0
     assert decode(lib, partition_size=512, max_seq_len=1000, workspace=A + 256,
                   workspace_bytes=need - 1) == EWS
