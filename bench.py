@@ -171,6 +171,18 @@ def workload_config(wl, partition_size):
             "parallelism": "replicas: one independent workload per GPU, no collective"}
 
 
+def max_over_ranks(values, device):
+    """Element-wise maximum of per-rank timings (all ranks call it)."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def replica_seed(base_seed: int, rank: int) -> int:
+    """Seed of rank `rank`'s replica of a workload (distinct per rank)."""
+    return base_seed + 7919 * rank
+
+
 def step_bytes(wl):
     c = wl.cfg
     eq, ekv = W.ELEM_BYTES[c.q_dtype], W.ELEM_BYTES[c.cache_dtype]
@@ -184,7 +196,7 @@ def step_bytes(wl):
 
 def run_ours(args, rank, world, dev):
     cfg = W.CONFIGS[args.workload]
-    cfg = cfg.replace(seed=cfg.seed + 7919 * rank)
+    cfg = cfg.replace(seed=replica_seed(cfg.seed, rank))
     P = cfg.partition_size if args.partition_size is None else args.partition_size
     wl = W.make_workload(cfg, device=dev)
     c = wl.cfg
@@ -298,9 +310,7 @@ def run_ours(args, rank, world, dev):
     assert torch.isfinite(h_out.float()).all(), "non-finite decode output"
 
     if world > 1:
-        t = torch.tensor([step_ms, decode_ms, e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        step_ms, decode_ms, e2e_ms = t.tolist()
+        step_ms, decode_ms, e2e_ms = max_over_ranks([step_ms, decode_ms, e2e_ms], dev)
 
     dec_b, app_b = step_bytes(wl)
     peak, peak_src = measured_hbm_peak()
