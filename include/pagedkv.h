@@ -157,6 +157,34 @@ int paged_attention_decode(void* out, const void* query, const void* k_cache,
                            void* stream);
 
 /*
+ * paged_attention_decode_static — paged_attention_decode without a caller
+ * workspace, for callers that cannot allocate device memory (code inside a
+ * framework that owns all device allocations, loops where cudaMalloc's implicit
+ * synchronisation is not acceptable, bindings with no device-memory API). The
+ * pages have no counterpart: it is a packaging of the same decode.
+ *
+ * Arguments and results are those of paged_attention_decode without
+ * `workspace` and `workspace_bytes`. The split-sequence scratch is a fixed
+ * 16 MiB array of device memory inside this library, present on every device
+ * where the library's device code is loaded until the process exits. Sizes whose
+ * paged_attention_workspace_size() exceeds 16 MiB are rejected with
+ * PKV_ERR_WORKSPACE before anything is enqueued. The call allocates nothing.
+ * Its first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make it before any stream
+ * capture. Every call shares the array, and each call clears what must start at
+ * zero; calls whose work overlaps on the GPU (several streams or host threads)
+ * race on the array and must be serialised by the caller.
+ */
+int paged_attention_decode_static(void* out, const void* query, const void* k_cache,
+                                  const void* v_cache, const int32_t* block_table,
+                                  const int32_t* seq_lens, int num_seqs, int num_heads,
+                                  int num_kv_heads, int head_dim, int block_size,
+                                  int max_blocks_per_seq, int64_t num_blocks, int max_seq_len,
+                                  float scale, int q_dtype, int cache_dtype,
+                                  const float* k_scale, const float* v_scale, int partition_size,
+                                  int max_ctas, unsigned flags, void* stream);
+
+/*
  * Health word of the device kernels. Every wait inside a kernel is bounded
  * (about one second); a wait that expires makes its CTA skip the rest of its
  * work and sets this word, so a wrong result is reported instead of a hung GPU.

@@ -15,6 +15,7 @@ import os
 import torch
 
 __all__ = ["paged_kv_append", "paged_attention_decode", "paged_attention_workspace_size",
+           "paged_attention_decode_static",
            "pkv_device_status", "pkv_status_string", "pkv_version", "load_library", "PagedKVError",
            "PKV_F32", "PKV_F16", "PKV_BF16", "PKV_FP8_E4M3", "PKV_DECODE_FORCE_SIMT",
            "LIB_PATH", "EXPORTED_SYMBOLS"]
@@ -25,8 +26,8 @@ PKV_F32, PKV_F16, PKV_BF16, PKV_FP8_E4M3 = 0, 1, 2, 3
 PKV_DECODE_FORCE_SIMT = 1
 
 EXPORTED_SYMBOLS = ("paged_kv_append", "paged_attention_workspace_size",
-                    "paged_attention_decode", "pkv_device_status", "pkv_status_string",
-                    "pkv_version")
+                    "paged_attention_decode", "paged_attention_decode_static",
+                    "pkv_device_status", "pkv_status_string", "pkv_version")
 
 _DTYPE_CODES = {torch.float32: PKV_F32, torch.float16: PKV_F16, torch.bfloat16: PKV_BF16,
                 torch.uint8: PKV_FP8_E4M3, torch.float8_e4m3fn: PKV_FP8_E4M3}
@@ -64,6 +65,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pkv_version.restype = I
     lib.pkv_device_status.argtypes = [I]
     lib.pkv_device_status.restype = I
+    lib.paged_attention_decode_static.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I64, I, F,
+                                                  I, I, P, P, I, I, U, P]
+    lib.paged_attention_decode_static.restype = I
     _lib = lib
     return lib
 
@@ -142,3 +146,24 @@ def paged_attention_decode(out, query, k_cache, v_cache, block_table, seq_lens, 
                                     _ptr(workspace), ws_bytes, _stream(stream))
     if st != 0:
         raise PagedKVError("paged_attention_decode", st)
+
+
+def paged_attention_decode_static(out, query, k_cache, v_cache, block_table, seq_lens, *,
+                                  max_seq_len, scale, partition_size=0, k_scale=None,
+                                  v_scale=None, max_ctas=0, flags=0, stream=None) -> None:
+    """paged_attention_decode with the library's own fixed scratch instead of a
+    caller workspace, for callers that cannot allocate device memory; see
+    paged_attention_decode_static in include/pagedkv.h (16 MiB limit, calls that
+    overlap on the GPU race)."""
+    lib = load_library()
+    S, Hq, D = query.shape
+    nb, bs, Hkv, _ = k_cache.shape
+    mbps = block_table.shape[1]
+    st = lib.paged_attention_decode_static(_ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache),
+                                           _ptr(block_table), _ptr(seq_lens), S, Hq, Hkv, D, bs,
+                                           mbps, nb, int(max_seq_len), float(scale),
+                                           _dtype_code(query), _dtype_code(k_cache),
+                                           _ptr(k_scale), _ptr(v_scale), int(partition_size),
+                                           int(max_ctas), int(flags), _stream(stream))
+    if st != 0:
+        raise PagedKVError("paged_attention_decode_static", st)
