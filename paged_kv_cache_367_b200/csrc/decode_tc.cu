@@ -34,6 +34,7 @@
 //    error word, skips the rest of its work and still waits, bounded, for its
 //    own copies in flight before it exits.
 #include <cuda.h>
+#include <type_traits>
 #include <cudaTypedefs.h>
 
 #include "schedule.cuh"
@@ -51,9 +52,9 @@ constexpr int kEpilogueWarp = kConsumerWarps + 1;    // combine, store, merge
 constexpr int kThreads = (kConsumerWarps + 2) * 32;
 constexpr long long kWaitCycles = 1ll << 31;         // ~1 s at 2 GHz
 
-template <int D, int NT, int NS>
+template <int D, int NT, int NS, int EKV>
 struct Cfg {
-  static constexpr int kKV = kChunk * D * 2;         // bytes of K (or V) per stage
+  static constexpr int kKV = kChunk * D * EKV;       // bytes of K (or V) per stage
   static constexpr int kQ = 8 * NT * D * 2;          // query rows of one KV head group
   static constexpr int kStage = (2 * kKV + kQ + 1023) / 1024 * 1024;
   static constexpr int kHeads = 8 * NT;
@@ -142,6 +143,22 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
                : "r"(addr));
 }
 
+// Two E4M3 codes (low byte first) to an f16x2 pair.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"((unsigned short)(two_codes & 0xffffu)));
+  return d;
+}
+
+// bf16x2 or f16x2 bits to f16x2 bits.
+template <typename T> __device__ __forceinline__ uint32_t to_f16x2(uint32_t v);
+template <> __device__ __forceinline__ uint32_t to_f16x2<__half>(uint32_t v) { return v; }
+template <> __device__ __forceinline__ uint32_t to_f16x2<__nv_bfloat16>(uint32_t v) {
+  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v));
+  __half2 h = __floats2half2_rn(f.x, f.y);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
   uint32_t d;
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
@@ -228,11 +245,16 @@ __device__ void warp_merge_unit(const DecodeParams& prm, const SegmentWalker& wk
   }
 }
 
-template <typename T, int D, int NT, int NS, int MINB>
+// T: query/output type (bf16 or f16). F8: the cache holds E4M3 codes; the
+// products then run in f16 (exact for E4M3 values) with k_scale folded into the
+// score scale and v_scale applied to the output.
+template <typename T, int D, int NT, int NS, int MINB, bool F8>
 __global__ void __launch_bounds__(kThreads, MINB)
     decode_tc_kernel(const DecodeParams prm, const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v) {
-  using C = Cfg<D, NT, NS>;
+  constexpr int EKV = F8 ? 1 : 2;  // cache element bytes
+  using C = Cfg<D, NT, NS, EKV>;
+  using M = typename std::conditional<F8, __half, T>::type;  // MMA operand type
   constexpr int H = C::kHeads;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -264,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Hq = prm.num_heads, Hkv = prm.num_kv_heads, g = Hq / Hkv, bs = prm.block_size;
-  const int tile = bs * D * 2;  // bytes of one (block, head) tile
+  const int tile = bs * D * EKV;  // bytes of one (block, head) tile
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer ----
@@ -356,6 +378,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
     // and link (piece of a split unit), release the buffer, and merge the unit
     // if this piece completed it.
     constexpr int V = D / 32;
+    const float vscale = F8 ? __ldg(prm.v_scale) : 1.f;
     int sidx = 0;
     Segment seg;
     while (walker.next(seg)) {
@@ -388,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
           float w[kConsumerWarps];
 #pragma unroll
           for (int x = 0; x < kConsumerWarps; ++x) w[x] = __shfl_sync(0xffffffffu, wx[x], j);
-          const float Lj = __shfl_sync(0xffffffffu, Lsum, j);
+          const float Lj = __shfl_sync(0xffffffffu, Lsum, j) / vscale;
           const float Mj = __shfl_sync(0xffffffffu, M, j);
           if (j < g) {
             float o[V];
@@ -410,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
               float* dst = prm.ws_o + rowp * D + lane * V;
 #pragma unroll
               for (int v = 0; v < V; ++v) dst[v] = o[v] / Lj;
-              if (lane == 0) prm.ws_lse[rowp] = Mj + fast_log2(Lj);
+              if (lane == 0) prm.ws_lse[rowp] = Mj + fast_log2(Lj * vscale);
             }
           }
         }
@@ -441,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
   const uint32_t vrow = (uint32_t)((vt / bs) * tile + (vt % bs) * 128);
   const uint32_t dh_stride = (uint32_t)(bs * 128);
   const uint32_t ring_u32 = smem_u32(ring);
-  const float sscale = prm.score_scale;
+  const float sscale = prm.score_scale * (F8 ? __ldg(prm.k_scale) : 1.f);
   constexpr int MT = D / 16;
 
   uint32_t kc = 0;
@@ -479,8 +502,16 @@ __global__ void __launch_bounds__(kThreads, MINB)
             uint32_t b0 = 0, b1 = 0;
             if (head < g) {
               const uint32_t* row = reinterpret_cast<const uint32_t*>(qs + head * D * 2);
-              b0 = row[(16 * ks + 2 * cq) / 2];
-              b1 = row[(16 * ks + 8 + 2 * cq) / 2];
+              if constexpr (F8) {
+                // E4M3 K rows give each lane 4 consecutive dimensions of a
+                // 16-wide step; the contraction index is permuted to match:
+                // logical (2cq, 2cq+1) <- dims 4cq, 4cq+1; (2cq+8, +9) <- 4cq+2, +3.
+                b0 = to_f16x2<T>(row[(16 * ks + 4 * cq) / 2]);
+                b1 = to_f16x2<T>(row[(16 * ks + 4 * cq + 2) / 2]);
+              } else {
+                b0 = row[(16 * ks + 2 * cq) / 2];
+                b1 = row[(16 * ks + 8 + 2 * cq) / 2];
+              }
             }
             bq[ks][nt][0] = b0;
             bq[ks][nt][1] = b1;
@@ -495,17 +526,41 @@ __global__ void __launch_bounds__(kThreads, MINB)
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
           for (int e = 0; e < 4; ++e) s[nt][e] = s2[nt][e] = 0.f;
+        if constexpr (F8) {
+          // One ldmatrix.x4 brings 16 tokens x 32 dimensions (two 16-wide steps).
 #pragma unroll
-        for (int ks = 0; ks < MT; ++ks) {
-          uint32_t a[4];
-          const int dh = ks >> 2, j = ((ks & 3) << 1) + kj;
-          ldsm_x4(a, st + krow + dh * dh_stride + ((j ^ x7) << 4));
+          for (int q2 = 0; q2 < MT / 2; ++q2) {
+            uint32_t r[4];
+            const int j = 2 * q2 + kj;
+            ldsm_x4(r, st + krow + ((j ^ x7) << 4));
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            if (ks & 1)
-              Mma<T>::run(s2[nt], a, bq[ks][nt][0], bq[ks][nt][1]);
-            else
-              Mma<T>::run(s[nt], a, bq[ks][nt][0], bq[ks][nt][1]);
+            for (int half = 0; half < 2; ++half) {
+              const int ks = 2 * q2 + half;
+              const uint32_t a[4] = {e4m3x2_to_f16x2(r[2 * half]), e4m3x2_to_f16x2(r[2 * half + 1]),
+                                     e4m3x2_to_f16x2(r[2 * half] >> 16),
+                                     e4m3x2_to_f16x2(r[2 * half + 1] >> 16)};
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                if (half)
+                  Mma<M>::run(s2[nt], a, bq[ks][nt][0], bq[ks][nt][1]);
+                else
+                  Mma<M>::run(s[nt], a, bq[ks][nt][0], bq[ks][nt][1]);
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < MT; ++ks) {
+            uint32_t a[4];
+            const int dh = ks >> 2, j = ((ks & 3) << 1) + kj;
+            ldsm_x4(a, st + krow + dh * dh_stride + ((j ^ x7) << 4));
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              if (ks & 1)
+                Mma<M>::run(s2[nt], a, bq[ks][nt][0], bq[ks][nt][1]);
+              else
+                Mma<M>::run(s[nt], a, bq[ks][nt][0], bq[ks][nt][1]);
+            }
           }
         }
         const bool v0 = g0 < nv, v1 = g0 + 8 < nv;
@@ -530,8 +585,8 @@ __global__ void __launch_bounds__(kThreads, MINB)
             p[hi][1] = fast_exp2(s1 - mu);
           }
           float r00, r01, r10, r11;
-          const uint32_t P0 = Mma<T>::pack(p[0][0], p[1][0], r00, r01);  // token g0, heads 2cq, 2cq+1
-          const uint32_t P1 = Mma<T>::pack(p[0][1], p[1][1], r10, r11);  // token g0 + 8
+          const uint32_t P0 = Mma<M>::pack(p[0][0], p[1][0], r00, r01);  // token g0, heads 2cq, 2cq+1
+          const uint32_t P1 = Mma<M>::pack(p[0][1], p[1][1], r10, r11);  // token g0 + 8
           l[nt * 2 + 0] = l[nt * 2 + 0] * alpha[0] + (r00 + r10);
           l[nt * 2 + 1] = l[nt * 2 + 1] * alpha[1] + (r01 + r11);
           if (alpha[0] != 1.f || alpha[1] != 1.f) {
@@ -553,17 +608,45 @@ __global__ void __launch_bounds__(kThreads, MINB)
           mlo = (2 * cq < nv ? 0x0000ffffu : 0u) | (2 * cq + 1 < nv ? 0xffff0000u : 0u);
           mhi = (2 * cq + 8 < nv ? 0x0000ffffu : 0u) | (2 * cq + 9 < nv ? 0xffff0000u : 0u);
         }
+        if constexpr (F8) {
+          // ldmatrix.trans on E4M3 rows gives each lane, per 8x16-byte matrix,
+          // dims (2g0, 2g0+1) of tokens (2cq, 2cq+1). One byte permute splits
+          // them into an even-dimension and an odd-dimension pair of tokens, so
+          // M-row g0 of the product is dim 16mt + 2g0 and row g0+8 is dim
+          // 16mt + 2g0 + 1.
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          uint32_t a[4];
-          const int dh = mt >> 2, j = ((mt & 3) << 1) + vj;
-          ldsm_x4_t(a, st + C::kKV + vrow + dh * dh_stride + ((j ^ x7) << 4));
-          a[0] &= mlo;
-          a[1] &= mlo;
-          a[2] &= mhi;
-          a[3] &= mhi;
+          for (int q2 = 0; q2 < MT / 2; ++q2) {
+            uint32_t r[4];
+            const int j = 2 * q2 + kj;
+            ldsm_x4_t(r, st + C::kKV + krow + ((j ^ x7) << 4));
+            r[0] &= mlo;
+            r[1] &= mhi;
+            r[2] &= mlo;
+            r[3] &= mhi;
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) Mma<T>::run(o[mt][nt], a, bp[nt][0], bp[nt][1]);
+            for (int half = 0; half < 2; ++half) {
+              const uint32_t lo = __byte_perm(r[2 * half], 0, 0x3120);      // tokens 2cq, 2cq+1
+              const uint32_t hi8 = __byte_perm(r[2 * half + 1], 0, 0x3120); // tokens 8+2cq, +1
+              const uint32_t a[4] = {e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(lo >> 16),
+                                     e4m3x2_to_f16x2(hi8), e4m3x2_to_f16x2(hi8 >> 16)};
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                Mma<M>::run(o[2 * q2 + half][nt], a, bp[nt][0], bp[nt][1]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            uint32_t a[4];
+            const int dh = mt >> 2, j = ((mt & 3) << 1) + vj;
+            ldsm_x4_t(a, st + C::kKV + vrow + dh * dh_stride + ((j ^ x7) << 4));
+            a[0] &= mlo;
+            a[1] &= mlo;
+            a[2] &= mhi;
+            a[3] &= mhi;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) Mma<M>::run(o[mt][nt], a, bp[nt][0], bp[nt][1]);
+          }
         }
       }
       __syncwarp();
@@ -599,11 +682,14 @@ __global__ void __launch_bounds__(kThreads, MINB)
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const int h0 = nt * 8 + 2 * cq, d0 = mt * 16 + g0;
+        // Rows g0 and g0 + 8 of m-tile mt: dims (16mt + g0, + 8), or for E4M3
+        // caches (16mt + 2g0, + 1).
+        const int h0 = nt * 8 + 2 * cq;
+        const int d0 = F8 ? mt * 16 + 2 * g0 : mt * 16 + g0, d1 = F8 ? d0 + 1 : d0 + 8;
         ro[h0 * D + d0] = o[mt][nt][0];
         ro[(h0 + 1) * D + d0] = o[mt][nt][1];
-        ro[h0 * D + d0 + 8] = o[mt][nt][2];
-        ro[(h0 + 1) * D + d0 + 8] = o[mt][nt][3];
+        ro[h0 * D + d1] = o[mt][nt][2];
+        ro[(h0 + 1) * D + d1] = o[mt][nt][3];
       }
     mbar_arrive(rfull + rb);
   }
@@ -626,17 +712,18 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 5-D view of a [num_blocks, bs, Hkv, D] 16-bit pool: (d_lo 64, token bs, d_hi D/64,
-// head Hkv, block num_blocks); one box is a whole (block, head) tile.
-static bool encode_pool_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int D,
-                            int bs, int Hkv, int64_t nb) {
+// 5-D view of a [num_blocks, bs, Hkv, D] pool of e-byte elements: (d_lo 128/e,
+// token bs, d_hi D*e/128, head Hkv, block num_blocks); one box is a whole
+// (block, head) tile, landing as 128-byte rows with the 128B swizzle.
+static bool encode_pool_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int e,
+                            int D, int bs, int Hkv, int64_t nb) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
-  const cuuint64_t e = 2;
-  cuuint64_t dims[5] = {64, (cuuint64_t)bs, (cuuint64_t)(D / 64), (cuuint64_t)Hkv, (cuuint64_t)nb};
-  cuuint64_t strides[4] = {(cuuint64_t)Hkv * D * e, 64 * e, (cuuint64_t)D * e,
+  const cuuint64_t row = 128 / e;  // elements per 128-byte row
+  cuuint64_t dims[5] = {row, (cuuint64_t)bs, (cuuint64_t)(D / row), (cuuint64_t)Hkv, (cuuint64_t)nb};
+  cuuint64_t strides[4] = {(cuuint64_t)Hkv * D * e, 128, (cuuint64_t)D * e,
                            (cuuint64_t)bs * Hkv * D * e};
-  cuuint32_t box[5] = {64, (cuuint32_t)bs, (cuuint32_t)(D / 64), 1, 1};
+  cuuint32_t box[5] = {(cuuint32_t)row, (cuuint32_t)bs, (cuuint32_t)(D / row), 1, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = enc(map, dt, 5, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -658,16 +745,18 @@ int tc_timeout_flag(bool clear, int* value) {
 }
 
 bool tc_supported(int q_dtype, int cache_dtype, int head_dim, int group) {
-  return (q_dtype == PKV_BF16 || q_dtype == PKV_F16) && cache_dtype == q_dtype &&
-         (head_dim == 64 || head_dim == 128) && group >= 1 && group <= 16;
+  if (q_dtype != PKV_BF16 && q_dtype != PKV_F16) return false;
+  if (group < 1 || group > 16) return false;
+  if (cache_dtype == q_dtype) return head_dim == 64 || head_dim == 128;
+  return cache_dtype == PKV_FP8_E4M3 && head_dim == 128;
 }
 
-template <typename T, int D, int NT, int NS, int MINB>
+template <typename T, int D, int NT, int NS, int MINB, bool F8>
 static cudaError_t launch_tc_t(const DecodeParams& prm, const CUtensorMap& mk,
                                const CUtensorMap& mv, int max_ctas, int num_sms,
                                cudaStream_t stream) {
-  using C = tc::Cfg<D, NT, NS>;
-  auto kernel = tc::decode_tc_kernel<T, D, NT, NS, MINB>;
+  using C = tc::Cfg<D, NT, NS, F8 ? 1 : 2>;
+  auto kernel = tc::decode_tc_kernel<T, D, NT, NS, MINB, F8>;
   static int occ = 0;
   if (occ == 0) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -685,36 +774,45 @@ static cudaError_t launch_tc_t(const DecodeParams& prm, const CUtensorMap& mk,
   return cudaGetLastError();
 }
 
-template <typename T, int D>
+template <typename T, int D, bool F8>
 static cudaError_t launch_tc_d(const DecodeParams& prm, const CUtensorMap& mk,
                                const CUtensorMap& mv, int max_ctas, int num_sms,
                                cudaStream_t stream) {
   // Two CTAs per SM (two producers keep more copies in flight than one) where
   // shared memory allows; head_dim 128 with more than 8 heads per group runs one.
   const int g = prm.num_heads / prm.num_kv_heads;
-  if (g <= 8) return launch_tc_t<T, D, 1, (D == 128 ? 2 : 4), 2>(prm, mk, mv, max_ctas, num_sms, stream);
-  if (D == 64) return launch_tc_t<T, D, 2, 4, 2>(prm, mk, mv, max_ctas, num_sms, stream);
-  return launch_tc_t<T, D, 2, 4, 1>(prm, mk, mv, max_ctas, num_sms, stream);
+  // E4M3 stages are half the size: four of them per CTA.
+  constexpr int kNS = F8 ? 4 : (D == 128 ? 2 : 4);
+  if (g <= 8) return launch_tc_t<T, D, 1, kNS, 2, F8>(prm, mk, mv, max_ctas, num_sms, stream);
+  if (D == 64 || F8) return launch_tc_t<T, D, 2, 4, 2, F8>(prm, mk, mv, max_ctas, num_sms, stream);
+  return launch_tc_t<T, D, 2, 4, 1, F8>(prm, mk, mv, max_ctas, num_sms, stream);
 }
 
 cudaError_t launch_decode_tc(const DecodeParams& prm, int q_dtype, int cache_dtype, int max_ctas,
                              int num_sms, cudaStream_t stream) {
-  (void)cache_dtype;
-  const CUtensorMapDataType dt =
-      q_dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const bool f8 = cache_dtype == PKV_FP8_E4M3;
+  const CUtensorMapDataType dt = f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : q_dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const int e = f8 ? 1 : 2;
   CUtensorMap mk, mv;
-  if (!encode_pool_map(&mk, prm.k_cache, dt, prm.head_dim, prm.block_size, prm.num_kv_heads,
+  if (!encode_pool_map(&mk, prm.k_cache, dt, e, prm.head_dim, prm.block_size, prm.num_kv_heads,
                        prm.num_blocks) ||
-      !encode_pool_map(&mv, prm.v_cache, dt, prm.head_dim, prm.block_size, prm.num_kv_heads,
+      !encode_pool_map(&mv, prm.v_cache, dt, e, prm.head_dim, prm.block_size, prm.num_kv_heads,
                        prm.num_blocks))
     return cudaErrorInvalidValue;
+  if (f8) {
+    return q_dtype == PKV_BF16
+               ? launch_tc_d<__nv_bfloat16, 128, true>(prm, mk, mv, max_ctas, num_sms, stream)
+               : launch_tc_d<__half, 128, true>(prm, mk, mv, max_ctas, num_sms, stream);
+  }
   if (q_dtype == PKV_BF16) {
     return prm.head_dim == 128
-               ? launch_tc_d<__nv_bfloat16, 128>(prm, mk, mv, max_ctas, num_sms, stream)
-               : launch_tc_d<__nv_bfloat16, 64>(prm, mk, mv, max_ctas, num_sms, stream);
+               ? launch_tc_d<__nv_bfloat16, 128, false>(prm, mk, mv, max_ctas, num_sms, stream)
+               : launch_tc_d<__nv_bfloat16, 64, false>(prm, mk, mv, max_ctas, num_sms, stream);
   }
-  return prm.head_dim == 128 ? launch_tc_d<__half, 128>(prm, mk, mv, max_ctas, num_sms, stream)
-                             : launch_tc_d<__half, 64>(prm, mk, mv, max_ctas, num_sms, stream);
+  return prm.head_dim == 128 ? launch_tc_d<__half, 128, false>(prm, mk, mv, max_ctas, num_sms, stream)
+                             : launch_tc_d<__half, 64, false>(prm, mk, mv, max_ctas, num_sms, stream);
 }
 
 }  // namespace pkv

@@ -162,3 +162,13 @@ def test_block_ids_outside_the_pool_read_as_zeros(cuda_dev):
         out = gpu_step(wl, cuda_dev, append=False, block_table=bt, flags=flags)
         want = oracle_decode(wl, kc, vc, block_table=bt)
         assert_close(to_f64(out), want, cfg)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (32, 8), (64, 8), (16, 1)])
+@pytest.mark.parametrize("qdt", ["bf16", "f16"])
+@pytest.mark.parametrize("flags", FLAGS)
+def test_fp8_cache_group_sizes(cuda_dev, Hq, Hkv, qdt, flags):
+    cfg = C["fp8_prefix"].replace(num_seqs=5, num_heads=Hq, num_kv_heads=Hkv, q_dtype=qdt,
+                                  lens=("uniform", 1, 400), prefix_len=0, partition_size=64,
+                                  seed=91)
+    _check(cfg, cuda_dev, flags=flags)
