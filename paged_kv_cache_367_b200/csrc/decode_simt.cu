@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(const DecodeP
       __syncthreads();
     }
     if (!(seg.t0 == 0 && seg.t1 == seg.len)) {
-      finish_piece<QT>(prm, walker, seg, threadIdx.x, kSimtThreads, &sm.flag,
+      finish_piece<QT>(prm, walker.cuts, walker.P, seg, threadIdx.x, kSimtThreads, &sm.flag,
                        [] { __syncthreads(); });
       __syncthreads();
     }
@@ -197,14 +197,16 @@ static cudaError_t launch_simt_t(const DecodeParams& prm, int max_ctas, int num_
   int& occ = prm.head_dim == 64 ? occ64 : occ128;
   if (occ == 0) occ = resident_ctas(kernel, kSimtThreads, 0);
   int grid = occ * num_sms;
-  if (grid > kMaxCtas) grid = kMaxCtas;
+  if (grid > kMaxRanges) grid = kMaxRanges;
   if (max_ctas > 0 && max_ctas < grid) grid = max_ctas;
   kernel<<<grid, kSimtThreads, 0, stream>>>(prm);
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode_simt(const DecodeParams& prm, int q_dtype, int cache_dtype,
+cudaError_t launch_decode_simt(const DecodeParams& prm_in, int q_dtype, int cache_dtype,
                                int max_ctas, int num_sms, cudaStream_t stream) {
+  DecodeParams prm = prm_in;
+  prm.dyn_ranges = 0;  // static ranges only: one per CTA
   const bool fp8 = cache_dtype == PKV_FP8_E4M3;
   switch (q_dtype) {
     case PKV_F32:

@@ -60,7 +60,7 @@ struct Cfg {
   static constexpr int kHeads = 8 * NT;
   static constexpr int kRedO = kConsumerWarps * kHeads * D;   // floats per hand-off buffer
   static constexpr int kRed = (kRedO + 2 * kConsumerWarps * kHeads) * 4;
-  static constexpr int kBar = (2 * NS + 4) * 8;
+  static constexpr int kBar = (2 * NS + 4) * 8 + (NS + 2) * 48;  // barriers, descriptors
   static constexpr int kSmem = 1024 + NS * kStage + 2 * kRed + kBar +
                                (int)sizeof(SchedShared) + 32;
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA exceeds 227 KB");
@@ -207,12 +207,12 @@ __device__ __forceinline__ void named_sync_consumers() {
 // log-sum-exp bookkeeping, every lane owns D/32 dimensions of every head. The
 // pieces are enumerated from the schedule, so their loads are independent.
 template <typename T, int D, int NT>
-__device__ void warp_merge_unit(const DecodeParams& prm, const SegmentWalker& wk,
+__device__ void warp_merge_unit(const DecodeParams& prm, const Cuts& cu, int64_t P,
                                 const Segment& s, int lane) {
   constexpr int V = D / 32;
   const int Hq = prm.num_heads, g = Hq / prm.num_kv_heads;
   float M = -INFINITY;
-  wk.for_each_piece(s.first, s.len, [&](int slot) {
+  for_each_piece(cu, P, s.first, s.len, [&](int slot) {
     if (lane < g) M = fmaxf(M, __ldcg(prm.ws_lse + (int64_t)slot * g + lane));
   });
   float num[8 * NT][V];
@@ -221,7 +221,7 @@ __device__ void warp_merge_unit(const DecodeParams& prm, const SegmentWalker& wk
 #pragma unroll
     for (int v = 0; v < V; ++v) num[j][v] = 0.f;
   float den = 0.f;
-  wk.for_each_piece(s.first, s.len, [&](int slot) {
+  for_each_piece(cu, P, s.first, s.len, [&](int slot) {
     const float w = lane < g ? fast_exp2(__ldcg(prm.ws_lse + (int64_t)slot * g + lane) - M) : 0.f;
     den += w;
 #pragma unroll
@@ -245,6 +245,17 @@ __device__ void warp_merge_unit(const DecodeParams& prm, const SegmentWalker& wk
   }
 }
 
+// What the producer tells the other warps about the chunk in a stage (and the
+// consumers tell the epilogue warp about a finished segment).
+struct ChunkDesc {
+  int64_t first;             // work offset of the unit's partition 0
+  int seq, head, t0, t1, len;  // the segment
+  int c0;                    // first token of the chunk
+  int range;                 // range the segment belongs to
+  int flags;
+};
+constexpr int kFirst = 1, kLast = 2, kEnd = 4;
+
 // T: query/output type (bf16 or f16). F8: the cache holds E4M3 codes; the
 // products then run in f16 (exact for E4M3 values) with k_scale folded into the
 // score scale and v_scale applied to the output.
@@ -265,7 +276,9 @@ __global__ void __launch_bounds__(kThreads, MINB)
   uint64_t* empty = full + NS;
   uint64_t* rfull = empty + NS;    // consumers -> epilogue warp, per hand-off buffer
   uint64_t* rempty = rfull + 2;    // epilogue warp -> consumers
-  SchedShared* sched = reinterpret_cast<SchedShared*>(rempty + 2);
+  ChunkDesc* desc = reinterpret_cast<ChunkDesc*>(rempty + 2);  // per stage
+  ChunkDesc* hdesc = desc + NS;                                 // per hand-off buffer
+  SchedShared* sched = reinterpret_cast<SchedShared*>(hdesc + 2);
   volatile int* abort = reinterpret_cast<volatile int*>(sched + 1);
 
   if (threadIdx.x == 0) {
@@ -287,75 +300,102 @@ __global__ void __launch_bounds__(kThreads, MINB)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Hq = prm.num_heads, Hkv = prm.num_kv_heads, g = Hq / Hkv, bs = prm.block_size;
   const int tile = bs * D * EKV;  // bytes of one (block, head) tile
+  const Cuts cuts = sched->cuts;
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer ----
-    // Streams the chunks of every segment, in order, into the ring. The block
-    // ids of the next segment are loaded while the current one is issued; the
-    // lane holding a block's id issues that block's K and V tile copies.
+    // Streams the chunks of every segment of this CTA's static range, then of
+    // each dynamic range it takes, in order, into the ring, with a descriptor
+    // per chunk. The block ids of the next segment are loaded while the current
+    // one is issued; the lane holding a block's id issues that block's K and V
+    // tile copies. A final descriptor marks the end.
     uint32_t kc = 0;  // chunk counter: stage kc % NS, phase (kc / NS) & 1
     uint32_t armed = 0, last_parity = 0;
     bool ok = true;
     const T* qbase = static_cast<const T*>(prm.query);
-    Segment seg, nseg;
-    bool have = walker.next(seg);
-    int cur = 0;
-    if (have) {
-      const int32_t* bt = prm.block_table + (int64_t)seg.seq * prm.max_blocks_per_seq;
-      const int lb0 = seg.t0 / bs, nlb = (seg.t1 + bs - 1) / bs - lb0;
-      cur = lane < nlb ? __ldg(bt + lb0 + lane) : 0;
-    }
-    while (have) {
-      const int32_t* bt = prm.block_table + (int64_t)seg.seq * prm.max_blocks_per_seq;
-      const int lb0 = seg.t0 / bs;
-      const int nlb = (seg.t1 + bs - 1) / bs - lb0;
-      int nxt = lane + 32 < nlb ? __ldg(bt + lb0 + 32 + lane) : 0;
-      const bool have_next = walker.next(nseg);
-      int ncur = 0;
-      if (have_next) {
-        const int32_t* nbt = prm.block_table + (int64_t)nseg.seq * prm.max_blocks_per_seq;
-        const int nlb0 = nseg.t0 / bs, nnlb = (nseg.t1 + bs - 1) / bs - nlb0;
-        ncur = lane < nnlb ? __ldg(nbt + nlb0 + lane) : 0;
+    int64_t r = blockIdx.x;
+    int ci = sched->d_i;            // forward cursor for dynamic ranges
+    int64_t cbase = sched->d_base;
+    int* const dyn_counter = prm.ws_done + (int64_t)prm.num_seqs * Hkv;
+    for (;;) {
+      Segment seg, nseg;
+      bool have = walker.next(seg);
+      int cur = 0;
+      if (have) {
+        const int32_t* bt = prm.block_table + (int64_t)seg.seq * prm.max_blocks_per_seq;
+        const int lb0 = seg.t0 / bs, nlb = (seg.t1 + bs - 1) / bs - lb0;
+        cur = lane < nlb ? __ldg(bt + lb0 + lane) : 0;
       }
-      int batch = 0;
-      for (int c0 = seg.t0; c0 < seg.t1; c0 += kChunk, ++kc) {
-        const int stage = (int)(kc % NS);
-        const uint32_t phase = (kc / NS) & 1u;
-        const int rel = (c0 - seg.t0) / bs;
-        if (rel >= batch + 32) {
-          cur = nxt;
-          batch += 32;
-          nxt = lane + batch + 32 < nlb ? __ldg(bt + lb0 + batch + 32 + lane) : 0;
+      while (have && ok) {
+        const int32_t* bt = prm.block_table + (int64_t)seg.seq * prm.max_blocks_per_seq;
+        const int lb0 = seg.t0 / bs;
+        const int nlb = (seg.t1 + bs - 1) / bs - lb0;
+        int nxt = lane + 32 < nlb ? __ldg(bt + lb0 + 32 + lane) : 0;
+        const bool have_next = walker.next(nseg);
+        int ncur = 0;
+        if (have_next) {
+          const int32_t* nbt = prm.block_table + (int64_t)nseg.seq * prm.max_blocks_per_seq;
+          const int nlb0 = nseg.t0 / bs, nnlb = (nseg.t1 + bs - 1) / bs - nlb0;
+          ncur = lane < nnlb ? __ldg(nbt + nlb0 + lane) : 0;
         }
-        const int ntok = min(kChunk, seg.t1 - c0);
-        const int nblk = (ntok + bs - 1) / bs;
-        const bool first = c0 == seg.t0;
-        if (lane == 0 && ok) ok = mbar_wait(empty + stage, phase ^ 1u, abort);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        uint8_t* st = ring + stage * C::kStage;
-        if (ok && lane == 0) {
-          const uint32_t qbytes = first ? (uint32_t)(g * D * 2) : 0u;
-          mbar_expect_tx(full + stage, (uint32_t)(2 * nblk * tile) + qbytes);
-          if (first)
-            bulk_load(st + 2 * C::kKV, qbase + ((int64_t)seg.seq * Hq + seg.head * g) * D, qbytes,
-                      full + stage);
+        int batch = 0;
+        for (int c0 = seg.t0; c0 < seg.t1; c0 += kChunk, ++kc) {
+          const int stage = (int)(kc % NS);
+          const uint32_t phase = (kc / NS) & 1u;
+          const int rel = (c0 - seg.t0) / bs;
+          if (rel >= batch + 32) {
+            cur = nxt;
+            batch += 32;
+            nxt = lane + batch + 32 < nlb ? __ldg(bt + lb0 + batch + 32 + lane) : 0;
+          }
+          const int ntok = min(kChunk, seg.t1 - c0);
+          const int nblk = (ntok + bs - 1) / bs;
+          const bool first = c0 == seg.t0;
+          if (lane == 0 && ok) ok = mbar_wait(empty + stage, phase ^ 1u, abort);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          uint8_t* st = ring + stage * C::kStage;
+          if (ok && lane == 0) {
+            ChunkDesc& dd = desc[stage];
+            dd.first = seg.first;
+            dd.seq = seg.seq;
+            dd.head = seg.head;
+            dd.t0 = seg.t0;
+            dd.t1 = seg.t1;
+            dd.len = seg.len;
+            dd.c0 = c0;
+            dd.range = (int)r;
+            dd.flags = (first ? kFirst : 0) | (c0 + kChunk >= seg.t1 ? kLast : 0);
+            const uint32_t qbytes = first ? (uint32_t)(g * D * 2) : 0u;
+            mbar_expect_tx(full + stage, (uint32_t)(2 * nblk * tile) + qbytes);  // releases dd
+            if (first)
+              bulk_load(st + 2 * C::kKV, qbase + ((int64_t)seg.seq * Hq + seg.head * g) * D,
+                        qbytes, full + stage);
+          }
+          __syncwarp();
+          const int b = lane - (rel - batch);
+          if (ok && b >= 0 && b < nblk) {
+            tma_load_5d(st + b * tile, &tmap_k, 0, 0, 0, seg.head, cur, full + stage);
+            tma_load_5d(st + C::kKV + b * tile, &tmap_v, 0, 0, 0, seg.head, cur, full + stage);
+          }
+          if (ok) {
+            armed |= 1u << stage;
+            last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          }
         }
-        __syncwarp();
-        const int b = lane - (rel - batch);
-        if (ok && b >= 0 && b < nblk) {
-          tma_load_5d(st + b * tile, &tmap_k, 0, 0, 0, seg.head, cur, full + stage);
-          tma_load_5d(st + C::kKV + b * tile, &tmap_v, 0, 0, 0, seg.head, cur, full + stage);
-        }
-        if (ok) {
-          armed |= 1u << stage;
-          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-        }
+        seg = nseg;
+        cur = ncur;
+        have = have_next;
       }
-      seg = nseg;
-      cur = ncur;
-      have = have_next;
+      if (!ok || cuts.Rd == 0) break;
+      int64_t nr = 0;
+      if (lane == 0) nr = cuts.G + atomicAdd(dyn_counter, 1);
+      nr = __shfl_sync(0xffffffffu, nr, 0);
+      if (nr >= cuts.R()) break;
+      r = nr;
+      warp_start_range(prm, walker, r, ci, cbase);  // an empty range leaves the walker done
     }
-    // Wait, bounded, for this CTA's copies in flight before leaving.
+    // Wait, bounded, for this CTA's copies in flight (before the end marker,
+    // which moves a stage's barrier on to another phase).
     if (lane == 0) {
       for (int s = 0; s < NS; ++s) {
         if (!(armed >> s & 1u)) continue;
@@ -368,6 +408,16 @@ __global__ void __launch_bounds__(kThreads, MINB)
         }
       }
     }
+    // End marker.
+    {
+      const int stage = (int)(kc % NS);
+      const uint32_t phase = (kc / NS) & 1u;
+      if (lane == 0 && ok) ok = mbar_wait(empty + stage, phase ^ 1u, abort);
+      if (lane == 0 && ok) {
+        desc[stage].flags = kEnd;
+        mbar_arrive(full + stage);
+      }
+    }
     return;
   }
 
@@ -375,23 +425,31 @@ __global__ void __launch_bounds__(kThreads, MINB)
     // ------------------------------------------------------------ epilogue ----
     // For every segment: combine the four consumer warps' softmax states from
     // the hand-off buffer, write the output rows (whole unit) or the partial
-    // and link (piece of a split unit), release the buffer, and merge the unit
-    // if this piece completed it.
+    // (piece of a split unit), release the buffer, and merge the unit if this
+    // piece completed it.
     constexpr int V = D / 32;
     const float vscale = F8 ? __ldg(prm.v_scale) : 1.f;
     int sidx = 0;
-    Segment seg;
-    while (walker.next(seg)) {
+    for (;;) {
       const int rb = sidx & 1;
       const uint32_t use = (uint32_t)(sidx >> 1);
       ++sidx;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(rfull + rb, use & 1u, abort));
+      const ChunkDesc d = hdesc[rb];
+      if (!ok || (d.flags & kEnd)) break;
+      Segment seg;
+      seg.seq = d.seq;
+      seg.head = d.head;
+      seg.t0 = d.t0;
+      seg.t1 = d.t1;
+      seg.len = d.len;
+      seg.first = d.first;
       const float* ro = red + rb * (C::kRed / 4);
       const float* rm = ro + C::kRedO;
       const float* rl = rm + kConsumerWarps * H;
       const bool whole = seg.t0 == 0 && seg.t1 == seg.len;
       const int i = seg.seq, h = seg.head;
-      if (ok) {
+      {
         // lane j < g: per-head maximum, warp weights and denominator
         float M = -INFINITY, wx[kConsumerWarps], Lsum = 0.f;
         if (lane < g) {
@@ -429,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
 #pragma unroll
               for (int v = 0; v < V; ++v) dst[v] = from_f32<T>(o[v] / Lj);
             } else {
-              const int64_t rowp = (int64_t)own_piece_slot(blockIdx.x, seg) * g + j;
+              const int64_t rowp = (int64_t)own_piece_slot(d.range, seg) * g + j;
               float* dst = prm.ws_o + rowp * D + lane * V;
 #pragma unroll
               for (int v = 0; v < V; ++v) dst[v] = o[v] / Lj;
@@ -440,13 +498,13 @@ __global__ void __launch_bounds__(kThreads, MINB)
       }
       __syncwarp();
       mbar_arrive(rempty + rb);  // the hand-off buffer may be refilled
-      if (ok && !whole) {
+      if (!whole) {
         __threadfence();
         __syncwarp();
         const int last = lane == 0 ? (int)complete_piece(prm, seg) : 0;
         if (__shfl_sync(0xffffffffu, last, 0)) {
           __threadfence();
-          warp_merge_unit<T, D, NT>(prm, walker, seg, lane);
+          warp_merge_unit<T, D, NT>(prm, cuts, walker.P, seg, lane);
         }
       }
     }
@@ -469,29 +527,32 @@ __global__ void __launch_bounds__(kThreads, MINB)
 
   uint32_t kc = 0;
   int sidx = 0;
-  Segment seg;
-  while (walker.next(seg)) {
-    float m[2 * NT], l[2 * NT];
-    float o[MT][NT][4];
-    uint32_t bq[MT][NT][2];
+  float m[2 * NT], l[2 * NT];
+  float o[MT][NT][4];
+  uint32_t bq[MT][NT][2];
+  for (;;) {
+    const int stage = (int)(kc % NS);
+    const uint32_t phase = (kc / NS) & 1u;
+    ++kc;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(full + stage, phase, abort));
+    if (!ok) break;
+    const ChunkDesc d = desc[stage];
+    if (d.flags & kEnd) break;
+    const uint32_t st = ring_u32 + stage * C::kStage;
+    if (d.flags & kFirst) {
 #pragma unroll
-    for (int x = 0; x < 2 * NT; ++x) {
-      m[x] = -INFINITY;
-      l[x] = 0.f;
+      for (int x = 0; x < 2 * NT; ++x) {
+        m[x] = -INFINITY;
+        l[x] = 0.f;
+      }
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
     }
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
-
-    for (int c0 = seg.t0; c0 < seg.t1; c0 += kChunk, ++kc) {
-      const int stage = (int)(kc % NS);
-      const uint32_t phase = (kc / NS) & 1u;
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(full + stage, phase, abort));
-      const uint32_t st = ring_u32 + stage * C::kStage;
-      if (ok && c0 == seg.t0) {
+      if (d.flags & kFirst) {
         // Q^T fragments: b0b1 = Q[head g0][16ks + 2cq, +1], b2b3 = the same + 8 dims.
         const uint8_t* qs = ring + stage * C::kStage + 2 * C::kKV;
 #pragma unroll
@@ -518,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
           }
         }
       }
-      const int nv = min(16, max(0, seg.t1 - (c0 + 16 * w)));
+      const int nv = min(16, max(0, d.t1 - (d.c0 + 16 * w)));
       if (ok && nv > 0) {
         // S^T = K Q^T for this warp's 16 tokens; two accumulator chains.
         float s[NT][4], s2[NT][4];
@@ -650,47 +711,56 @@ __global__ void __launch_bounds__(kThreads, MINB)
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(empty + stage);
+    if (lane == 0) mbar_arrive(empty + stage);
+    if (d.flags & kLast) {
+      // ---- hand the warp's state to the epilogue warp ----
+  #pragma unroll
+      for (int x = 0; x < 2 * NT; ++x) {
+        l[x] += __shfl_xor_sync(0xffffffffu, l[x], 4);
+        l[x] += __shfl_xor_sync(0xffffffffu, l[x], 8);
+        l[x] += __shfl_xor_sync(0xffffffffu, l[x], 16);
+      }
+      const int rb = sidx & 1;
+      const uint32_t use = (uint32_t)(sidx >> 1);
+      ++sidx;
+      // The buffer's previous contents (two segments ago) must have been read.
+      mbar_wait(rempty + rb, (use & 1u) ^ 1u, abort);
+      if (w == 0 && lane == 0) hdesc[rb] = d;
+      float* ro = red + rb * (C::kRed / 4) + (w * H) * D;
+      float* rm = red + rb * (C::kRed / 4) + C::kRedO;
+      float* rl = rm + kConsumerWarps * H;
+      if (g0 == 0) {
+  #pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+  #pragma unroll
+          for (int hi = 0; hi < 2; ++hi) {
+            const int head = nt * 8 + 2 * cq + hi;
+            rm[w * H + head] = m[nt * 2 + hi];
+            rl[w * H + head] = l[nt * 2 + hi];
+          }
+      }
+  #pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+  #pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          // Rows g0 and g0 + 8 of m-tile mt: dims (16mt + g0, + 8), or for E4M3
+          // caches (16mt + 2g0, + 1).
+          const int h0 = nt * 8 + 2 * cq;
+          const int d0 = F8 ? mt * 16 + 2 * g0 : mt * 16 + g0, d1 = F8 ? d0 + 1 : d0 + 8;
+          ro[h0 * D + d0] = o[mt][nt][0];
+          ro[(h0 + 1) * D + d0] = o[mt][nt][1];
+          ro[h0 * D + d1] = o[mt][nt][2];
+          ro[(h0 + 1) * D + d1] = o[mt][nt][3];
+        }
+    mbar_arrive(rfull + rb);
     }
-
-    // ---- hand the warp's state to the epilogue warp ----
-#pragma unroll
-    for (int x = 0; x < 2 * NT; ++x) {
-      l[x] += __shfl_xor_sync(0xffffffffu, l[x], 4);
-      l[x] += __shfl_xor_sync(0xffffffffu, l[x], 8);
-      l[x] += __shfl_xor_sync(0xffffffffu, l[x], 16);
-    }
+  }
+  // Tell the epilogue warp there is nothing more.
+  {
     const int rb = sidx & 1;
     const uint32_t use = (uint32_t)(sidx >> 1);
-    ++sidx;
-    // The buffer's previous contents (two segments ago) must have been read.
     mbar_wait(rempty + rb, (use & 1u) ^ 1u, abort);
-    float* ro = red + rb * (C::kRed / 4) + (w * H) * D;
-    float* rm = red + rb * (C::kRed / 4) + C::kRedO;
-    float* rl = rm + kConsumerWarps * H;
-    if (g0 == 0) {
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int hi = 0; hi < 2; ++hi) {
-          const int head = nt * 8 + 2 * cq + hi;
-          rm[w * H + head] = m[nt * 2 + hi];
-          rl[w * H + head] = l[nt * 2 + hi];
-        }
-    }
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        // Rows g0 and g0 + 8 of m-tile mt: dims (16mt + g0, + 8), or for E4M3
-        // caches (16mt + 2g0, + 1).
-        const int h0 = nt * 8 + 2 * cq;
-        const int d0 = F8 ? mt * 16 + 2 * g0 : mt * 16 + g0, d1 = F8 ? d0 + 1 : d0 + 8;
-        ro[h0 * D + d0] = o[mt][nt][0];
-        ro[(h0 + 1) * D + d0] = o[mt][nt][1];
-        ro[h0 * D + d1] = o[mt][nt][2];
-        ro[(h0 + 1) * D + d1] = o[mt][nt][3];
-      }
+    if (w == 0 && lane == 0) hdesc[rb].flags = kEnd;
     mbar_arrive(rfull + rb);
   }
 }
@@ -768,9 +838,19 @@ static cudaError_t launch_tc_t(const DecodeParams& prm, const CUtensorMap& mk,
     occ = n > 0 ? n : 1;
   }
   int grid = occ * num_sms;
-  if (grid > kMaxCtas) grid = kMaxCtas;
+  if (grid > kMaxRanges) grid = kMaxRanges;
   if (max_ctas > 0 && max_ctas < grid) grid = max_ctas;
-  kernel<<<grid, tc::kThreads, C::kSmem, stream>>>(prm, mk, mv);
+  // Dynamic ranges (work handed out at run time to whichever CTA is free) are
+  // supported by the kernel but off: on the measured workloads the extra pieces
+  // they cut, with their merges and per-range start-up, cost more than the
+  // tail they save. kDynRanges > 0 turns them on (up to kMaxRanges in total).
+  constexpr int kDynRanges = 0;
+  DecodeParams p = prm;
+  p.dyn_ranges = prm.ws_done && kDynRanges > 0
+                     ? (kDynRanges < kMaxRanges - grid ? kDynRanges : kMaxRanges - grid)
+                     : 0;
+  p.static_share = 870;
+  kernel<<<grid, tc::kThreads, C::kSmem, stream>>>(p, mk, mv);
   return cudaGetLastError();
 }
 

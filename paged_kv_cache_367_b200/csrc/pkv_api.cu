@@ -39,15 +39,16 @@ struct WsLayout {
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Partials: two slots per CTA of up to kMaxCtas, each g rows of D floats plus g
-// log-sum-exp values; one counter per (sequence, KV head).
+// Partials: two slots per range, up to kMaxRanges ranges, each g rows of D
+// floats plus g log-sum-exp values; one counter per (sequence, KV head) and the
+// dynamic-range counter.
 static WsLayout workspace_layout(int64_t S, int64_t Hq, int64_t Hkv, int64_t D, int64_t parts) {
   WsLayout w;
-  const int64_t g = Hq / Hkv, slots = 2 * (int64_t)kMaxCtas;
+  const int64_t g = Hq / Hkv, slots = 2 * (int64_t)kMaxRanges;
   w.o = 0;
   w.lse = align256(w.o + sizeof(float) * slots * g * D);
   w.done = align256(w.lse + sizeof(float) * slots * g);
-  w.total = align256(w.done + sizeof(int32_t) * S * Hkv);
+  w.total = align256(w.done + sizeof(int32_t) * (S * Hkv + 1));
   if (parts <= 1) w.total = 0;  // no sequence can be cut
   return w;
 }
@@ -169,6 +170,8 @@ int paged_attention_decode(void* out, const void* query, const void* k_cache,
   prm.len_cap = (int)(cap < max_seq_len ? cap : max_seq_len);
   prm.part = parts > 1 ? partition_size : 0;
   prm.unit_cost = 64;  // about one chunk: a segment's set-up and epilogue, in tokens
+  prm.dyn_ranges = 0;  // the tensor-core launcher enables dynamic ranges
+  prm.static_share = 1024;
   prm.score_scale = scale * kLog2e;
   prm.k_scale = k_scale;
   prm.v_scale = v_scale;
@@ -181,8 +184,10 @@ int paged_attention_decode(void* out, const void* query, const void* k_cache,
   const int group = num_heads / num_kv_heads;
   cudaError_t e;
   if (ws.total > 0) {
-    // Per-unit counters of finished split tokens start at zero every call.
-    e = cudaMemsetAsync(prm.ws_done, 0, sizeof(int32_t) * (size_t)num_seqs * num_kv_heads, st);
+    // Per-unit counters of finished split tokens and the dynamic-range counter
+    // start at zero every call.
+    e = cudaMemsetAsync(prm.ws_done, 0, sizeof(int32_t) * ((size_t)num_seqs * num_kv_heads + 1),
+                        st);
     if (e != cudaSuccess) return PKV_ERR_CUDA;
   }
   if (!(flags & PKV_DECODE_FORCE_SIMT) && tc_supported(q_dtype, cache_dtype, head_dim, group))

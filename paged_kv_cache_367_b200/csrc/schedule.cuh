@@ -5,26 +5,29 @@
 // tokens). Units are laid end to end in (sequence, head) order, giving every
 // unit a work range in [0, W), W = sum over units of (cost + L). Partition p of
 // a unit (tokens [p P, (p + 1) P)) is an item at work offset
-//   first + p P,   first = unit start + cost,
-// and belongs to CTA floor(offset G / W) of a grid of G CTAs. So every CTA gets
-// about W / G of work and a contiguous run of items; a unit may be cut only at
-// multiples of the partition size P (never, when P = 0). Consecutive items of
-// one unit in one CTA form a segment, processed as one stream. A unit covered
-// by one segment is finished by that CTA. A unit cut into several segments
-// ("pieces") leaves one partial per piece, and the CTA that finishes the last
-// piece merges them. The split needs no host knowledge of seq_lens: each CTA
-// reads them (small, L2-resident) to find its own range.
+//   first + p P,   first = unit start + cost.
+// [0, W) is cut into ranges (Cuts): G "static" ranges of equal size cover
+// [0, Ws) and are taken by CTA r = blockIdx.x; Rd "dynamic" ranges of equal size
+// cover [Ws, W) and are handed out, in order, to whichever CTA asks next (a
+// global counter), so CTAs that run faster take more of the tail. An item
+// belongs to the range its offset falls in; a unit may be cut only at multiples
+// of the partition size P (never, when P = 0). Consecutive items of one unit in
+// one range form a segment, processed as one stream. A unit covered by one
+// segment is finished there. A unit cut into several segments ("pieces")
+// leaves one partial per piece, and the CTA that finishes the last piece merges
+// them. No host knowledge of seq_lens is needed: CTAs read them (small,
+// L2-resident) to find their ranges.
 //
-// Partials live in the workspace in two slots per CTA: slot 2c holds CTA c's
-// piece that starts inside a unit (only its first segment can), slot 2c + 1
-// its piece that starts a unit and ends inside it (only its last segment can).
+// Partials live in the workspace in two slots per range: slot 2r holds range
+// r's piece that starts inside a unit (only its first segment can), slot
+// 2r + 1 its piece that starts a unit and ends inside it (only its last can).
 #pragma once
 
 #include "common.cuh"
 
 namespace pkv {
 
-constexpr int kMaxCtas = 1024;  // grid size bound (two partial slots per CTA)
+constexpr int kMaxRanges = 1024;  // ranges per launch (two partial slots each)
 
 struct DecodeParams {
   void* out;
@@ -38,12 +41,15 @@ struct DecodeParams {
   int len_cap;        // seq_lens are clamped to [0, len_cap]
   int part;           // partition size in tokens, 0 = never split
   int unit_cost;      // work charged per non-empty unit, in tokens
+  int dyn_ranges;     // number of dynamic ranges (0: every range is static)
+  int static_share;   // share of the work in static ranges, in 1/1024 (when dyn_ranges > 0)
   float score_scale;  // scale * log2(e): scores are kept in the base-2 domain
   const float* k_scale;
   const float* v_scale;
-  float* ws_o;        // [2 * kMaxCtas, g, head_dim]: normalised partial output rows
-  float* ws_lse;      // [2 * kMaxCtas, g]: base-2 log-sum-exp of each partial
-  int* ws_done;       // [num_seqs, num_kv_heads]: finished tokens of split units (zeroed per call)
+  float* ws_o;        // [2 * kMaxRanges, g, head_dim]: normalised partial output rows
+  float* ws_lse;      // [2 * kMaxRanges, g]: base-2 log-sum-exp of each partial
+  int* ws_done;       // [num_seqs * num_kv_heads + 1]: finished tokens of split units, then
+                      // the dynamic-range counter (zeroed per call)
 };
 
 constexpr int64_t kNoSplit = int64_t(1) << 30;
@@ -60,6 +66,34 @@ __host__ __device__ __forceinline__ int load_len(const int32_t* p) {
 #endif
 }
 
+// The cut of [0, W) into G static ranges over [0, Ws) and Rd dynamic ranges
+// over [Ws, W) (Rd = 0 means Ws = W).
+struct Cuts {
+  int64_t W, Ws, G, Rd;
+
+  __host__ __device__ int64_t R() const { return G + Rd; }
+  // First work offset of range r (r in [0, R]).
+  __host__ __device__ int64_t lo(int64_t r) const {
+    if (r <= G) return (Ws * r + G - 1) / G;
+    return Ws + ((W - Ws) * (r - G) + Rd - 1) / Rd;
+  }
+  // Range holding offset off (0 <= off < W).
+  __host__ __device__ int64_t owner(int64_t off) const {
+    if (off < Ws) return off * G / Ws;
+    return G + (off - Ws) * Rd / (W - Ws);
+  }
+};
+
+__host__ __device__ __forceinline__ Cuts make_cuts(int64_t W, int64_t G, int64_t Rd,
+                                                   int static_share) {
+  Cuts c;
+  c.W = W;
+  c.G = G;
+  c.Rd = Rd;
+  c.Ws = Rd > 0 ? W * static_share / 1024 : W;
+  return c;
+}
+
 struct Segment {
   int seq, head;
   int t0, t1;       // token range [t0, t1) of the unit
@@ -67,39 +101,47 @@ struct Segment {
   int64_t first;    // work offset of the unit's partition 0
 };
 
-// First work offset owned by CTA c.
-__host__ __device__ __forceinline__ int64_t cta_lo(int64_t c, int64_t W, int64_t G) {
-  return (W * c + G - 1) / G;
-}
-
 // Index of the first partition of a unit (partition 0 at offset `first`) that
-// CTA c owns or would own: every partition before it belongs to earlier CTAs.
-__host__ __device__ __forceinline__ int64_t cta_first_part(int64_t c, int64_t first, int64_t P,
-                                                           int64_t W, int64_t G) {
-  const int64_t lo = cta_lo(c, W, G);
+// range r owns or would own: every partition before it belongs to earlier ranges.
+__host__ __device__ __forceinline__ int64_t range_first_part(const Cuts& cu, int64_t r,
+                                                             int64_t first, int64_t P) {
+  const int64_t lo = cu.lo(r);
   return lo <= first ? 0 : (lo - first + P - 1) / P;
 }
 
-// Workspace slot of the piece of a unit held by CTA c; c0 owns partition 0.
-__host__ __device__ __forceinline__ int piece_slot(int64_t c, int64_t c0) {
-  return (int)(2 * c + (c == c0 ? 1 : 0));
+// Workspace slot of the piece of a unit held by range r; r0 owns partition 0.
+__host__ __device__ __forceinline__ int piece_slot(int64_t r, int64_t r0) {
+  return (int)(2 * r + (r == r0 ? 1 : 0));
 }
 
-// Slot of the piece `s` produced by CTA c (the producing side of piece_slot).
-__host__ __device__ __forceinline__ int own_piece_slot(int64_t c, const Segment& s) {
-  return (int)(2 * c + (s.t0 == 0 ? 1 : 0));
+// Slot of the piece `s` produced by range r (the producing side of piece_slot).
+__host__ __device__ __forceinline__ int own_piece_slot(int64_t r, const Segment& s) {
+  return (int)(2 * r + (s.t0 == 0 ? 1 : 0));
 }
 
-// Walks the segments of one CTA's range. Each role of a CTA holds its own copy
-// and advances it independently; all copies see the same sequence. If the range
-// ends inside a unit that starts in it, that piece (the "tail") comes first and
-// the walk from the range's start stops short of it: its partial is then ready
-// early, and the CTA ends on work that needs no merge.
+// Pieces of a split unit (L tokens, partition 0 at `first`): f(slot) for each,
+// in token order.
+template <typename F>
+__host__ __device__ void for_each_piece(const Cuts& cu, int64_t P, int64_t first, int L, F f) {
+  const int64_t nparts = (L + P - 1) / P;
+  const int64_t r0 = cu.owner(first);
+  const int64_t r1 = cu.owner(first + (nparts - 1) * P);
+  for (int64_t r = r0; r <= r1; ++r) {
+    const int64_t s0 = r == r0 ? 0 : range_first_part(cu, r, first, P);
+    const int64_t s1 = r == r1 ? nparts : range_first_part(cu, r + 1, first, P);
+    if (s0 < s1) f(piece_slot(r, r0));
+  }
+}
+
+// Walks the segments of one range. If the range ends inside a unit that starts
+// in it, that piece (the "tail") comes first and the walk from the range's start
+// stops short of it: its partial is then ready early, and the range ends on
+// work that needs no merge.
 struct SegmentWalker {
   const int32_t* seq_lens;
   int S, Hkv, cap, cost;
   int64_t P;     // partition size, kNoSplit when the unit is never cut
-  int64_t W, G;  // total work, grid size
+  Cuts cuts;
   int64_t hi;    // where the walk from the range's start stops
   int64_t base;  // work offset of sequence i
   int i, h, L;
@@ -128,7 +170,7 @@ struct SegmentWalker {
         }
         continue;
       }
-      if (p * P >= L) { ++h; p = 0; continue; }  // unit's rest belongs to earlier CTAs
+      if (p * P >= L) { ++h; p = 0; continue; }  // unit's rest belongs to earlier ranges
       const int64_t first = base + (int64_t)h * (L + cost) + cost;
       if (first + p * P >= hi) { done = true; break; }
       const int64_t nparts = (L + P - 1) / P;
@@ -141,7 +183,7 @@ struct SegmentWalker {
       s.t0 = (int)(p * P);
       s.t1 = (int)((q + 1) * P < L ? (q + 1) * P : L);
       if (s.t1 < L) {
-        done = true;  // the rest of this unit belongs to the next CTA
+        done = true;  // the rest of this unit belongs to the next range
       } else {
         ++h;
         p = 0;
@@ -150,20 +192,54 @@ struct SegmentWalker {
     }
     return false;
   }
-
-  // Pieces of a split unit: calls f(slot) for each, in token order.
-  template <typename F>
-  __host__ __device__ void for_each_piece(int64_t first, int L, F f) const {
-    const int64_t nparts = (L + P - 1) / P;
-    const int64_t c0 = first * G / W;
-    const int64_t c1 = (first + (nparts - 1) * P) * G / W;
-    for (int64_t c = c0; c <= c1; ++c) {
-      const int64_t s0 = c == c0 ? 0 : cta_first_part(c, first, P, W, G);
-      const int64_t s1 = c == c1 ? nparts : cta_first_part(c + 1, first, P, W, G);
-      if (s0 < s1) f(piece_slot(c, c0));
-    }
-  }
 };
+
+// Sets up `w` for the range [lo, hi): `fi`/`fbase`/`fL` locate the sequence
+// holding offset lo (fi < 0: empty range), `li`/`lbase`/`lL` the one holding
+// hi - 1, and `fLnext` is the raw length of sequence fi + 1.
+__host__ __device__ __forceinline__ void start_range(SegmentWalker& w, int64_t lo, int64_t hi,
+                                                     int fi, int64_t fbase, int fL, int fLnext,
+                                                     int li, int64_t lbase, int lL) {
+  w.hi = hi;
+  w.tail_pending = false;
+  if (lo >= hi || fi < 0 || fL <= 0) {
+    w.done = true;
+    w.i = w.S;
+    w.h = 0;
+    w.L = 0;
+    w.Lnext = 0;
+    w.base = w.cuts.W;
+    w.p = 0;
+    return;
+  }
+  w.done = false;
+  w.i = fi;
+  w.base = fbase;
+  w.L = fL;
+  w.Lnext = fLnext;
+  const int64_t rel = lo - fbase;
+  w.h = (int)(rel / (fL + w.cost));
+  const int64_t r = rel - (int64_t)w.h * (fL + w.cost);  // offset inside unit (fi, h)
+  w.p = r <= w.cost ? 0 : (r - w.cost + w.P - 1) / w.P;
+  // The tail: the last item lies in a unit that starts at or after lo and
+  // continues past hi.
+  if (li < 0 || lL <= 0) return;
+  const int64_t lrel = (hi - 1) - lbase;
+  const int hh = (int)(lrel / (lL + w.cost));
+  const int64_t first = lbase + (int64_t)hh * (lL + w.cost) + w.cost;
+  if (hi - 1 < first || first < lo) return;
+  const int64_t nparts = (lL + w.P - 1) / w.P;
+  const int64_t q = (hi - 1 - first) / w.P;
+  if (q >= nparts - 1) return;  // the unit ends inside the range
+  w.tail.seq = li;
+  w.tail.head = hh;
+  w.tail.len = lL;
+  w.tail.first = first;
+  w.tail.t0 = 0;
+  w.tail.t1 = (int)((q + 1) * w.P);
+  w.tail_pending = true;
+  w.hi = first;  // the walk from lo stops before the tail unit
+}
 
 // Block-wide inclusive scan of one int64 per thread (blockDim.x <= 1024).
 __device__ __forceinline__ int64_t block_inclusive_scan(int64_t v, int64_t* sm32, int64_t& total) {
@@ -193,37 +269,16 @@ __device__ __forceinline__ int64_t block_inclusive_scan(int64_t v, int64_t* sm32
 
 struct SchedShared {
   int64_t scan[32];
-  int64_t found_base, last_base;
-  int64_t total;
-  int found_i, last_i;
+  int64_t f_base, l_base, d_base;
+  Cuts cuts;
+  int f_i, l_i, d_i;
 };
 
-// Sets the tail of a walker whose range [lo, hi) has its last offset in
-// sequence li (work offset lbase): if the last item lies in a unit that starts
-// at or after lo and continues past hi, that piece becomes the tail.
-__host__ __device__ __forceinline__ void set_tail(SegmentWalker& w, int li, int64_t lbase, int Lli,
-                                                  int64_t lo) {
-  w.tail_pending = false;
-  if (li < 0 || Lli <= 0) return;
-  const int64_t rel = (w.hi - 1) - lbase;
-  const int hh = (int)(rel / (Lli + w.cost));
-  const int64_t first = lbase + (int64_t)hh * (Lli + w.cost) + w.cost;
-  if (w.hi - 1 < first || first < lo) return;  // last item in an earlier unit, or unit began earlier
-  const int64_t nparts = (Lli + w.P - 1) / w.P;
-  const int64_t q = (w.hi - 1 - first) / w.P;
-  if (q >= nparts - 1) return;                  // the unit ends inside the range
-  w.tail.seq = li;
-  w.tail.head = hh;
-  w.tail.len = Lli;
-  w.tail.first = first;
-  w.tail.t0 = 0;
-  w.tail.t1 = (int)((q + 1) * w.P);
-  w.tail_pending = true;
-  w.hi = first;  // the walk from lo stops before the tail unit
-}
-
-// Sets up this CTA's walker (all threads must call it). Also zero-fills the
-// output rows of zero-length sequences i with i % gridDim.x == blockIdx.x.
+// Sets up this CTA's walker for its static range r = blockIdx.x (all threads
+// must call it; ends with __syncthreads), leaves the cuts in sh.cuts and the
+// sequence holding the start of the dynamic ranges in sh.d_i / sh.d_base. Also
+// zero-fills the output rows of zero-length sequences i with
+// i % gridDim.x == blockIdx.x.
 template <typename OT>
 __device__ void init_walker(const DecodeParams& prm, SchedShared& sh, SegmentWalker& w) {
   const int S = prm.num_seqs, Hkv = prm.num_kv_heads, cap = prm.len_cap, cost = prm.unit_cost;
@@ -240,32 +295,41 @@ __device__ void init_walker(const DecodeParams& prm, SchedShared& sh, SegmentWal
   }
   int64_t W;
   block_inclusive_scan(sum, sh.scan, W);
-  const int64_t lo = cta_lo(c, W, G);
-  const int64_t hi = cta_lo(c + 1, W, G);
-  // Pass 2: the sequences whose work ranges contain offsets lo and hi - 1.
+  const Cuts cu = make_cuts(W, G, prm.dyn_ranges, prm.static_share);
+  const int64_t lo = cu.lo(c), hi = cu.lo(c + 1), ws = cu.Ws;
+  // Pass 2: the sequences holding offsets lo, hi - 1 and Ws.
   if (threadIdx.x == 0) {
-    sh.found_i = -1;
-    sh.last_i = -1;
+    sh.f_i = -1;
+    sh.l_i = -1;
+    sh.d_i = S;
+    sh.d_base = W;
+    sh.cuts = cu;
   }
   __syncthreads();
   int64_t carry = 0;
-  for (int i0 = 0; i0 < S && lo < hi; i0 += blockDim.x) {
+  for (int i0 = 0; i0 < S; i0 += blockDim.x) {
     const int i = i0 + threadIdx.x;
     const int L = i < S ? clamp_len(__ldg(prm.seq_lens + i), cap) : 0;
     const int64_t wi = L > 0 ? (int64_t)Hkv * (L + cost) : 0;
     int64_t chunk_tot;
     const int64_t incl = block_inclusive_scan(wi, sh.scan, chunk_tot);
     const int64_t b = carry + incl - wi;
-    if (wi > 0 && b <= lo && lo < b + wi) {
-      sh.found_i = i;
-      sh.found_base = b;
+    if (wi > 0 && b <= lo && lo < b + wi && lo < hi) {
+      sh.f_i = i;
+      sh.f_base = b;
     }
-    if (wi > 0 && b <= hi - 1 && hi - 1 < b + wi) {
-      sh.last_i = i;
-      sh.last_base = b;
+    if (wi > 0 && b <= hi - 1 && hi - 1 < b + wi && lo < hi) {
+      sh.l_i = i;
+      sh.l_base = b;
+    }
+    if (wi > 0 && b <= ws && ws < b + wi) {
+      sh.d_i = i;
+      sh.d_base = b;
     }
     __syncthreads();
-    if (sh.last_i >= 0) break;
+    const bool have_range = lo >= hi || sh.l_i >= 0;
+    const bool have_dyn = ws >= W || sh.d_i < S;
+    if (have_range && have_dyn) break;
     carry += chunk_tot;
   }
   __syncthreads();
@@ -275,32 +339,61 @@ __device__ void init_walker(const DecodeParams& prm, SchedShared& sh, SegmentWal
   w.cap = cap;
   w.cost = cost;
   w.P = prm.part > 0 ? prm.part : kNoSplit;
-  w.W = W;
-  w.G = G;
-  w.hi = hi;
-  w.tail_pending = false;
-  const int fi = sh.found_i;
-  if (lo >= hi || fi < 0) {
-    w.done = true;
-    w.i = S;
-    w.h = 0;
-    w.L = 0;
-    w.Lnext = 0;
-    w.base = W;
-    w.p = 0;
-    return;
+  w.cuts = cu;
+  const int fi = sh.f_i, li = sh.l_i;
+  const int fL = fi >= 0 ? clamp_len(__ldg(prm.seq_lens + fi), cap) : 0;
+  const int fLn = fi >= 0 && fi + 1 < S ? __ldg(prm.seq_lens + fi + 1) : 0;
+  const int lL = li >= 0 ? clamp_len(__ldg(prm.seq_lens + li), cap) : 0;
+  start_range(w, lo, hi, fi, sh.f_base, fL, fLn, li, sh.l_base, lL);
+}
+
+// Warp-wide forward search: the sequence whose work range holds offset x,
+// starting from sequence *i at work offset *base (all lanes hold the same
+// cursor, which only moves forward). On success the cursor points at it and
+// *L is its clamped length; returns false if x lies past the last sequence.
+__device__ __forceinline__ bool warp_find_seq(const DecodeParams& prm, int64_t x, int& i,
+                                              int64_t& base, int& L) {
+  const int lane = threadIdx.x & 31;
+  const int S = prm.num_seqs, Hkv = prm.num_kv_heads, cap = prm.len_cap, cost = prm.unit_cost;
+  while (i < S) {
+    const int idx = i + lane;
+    const int Li = idx < S ? clamp_len(__ldg(prm.seq_lens + idx), cap) : 0;
+    const int64_t wi = Li > 0 ? (int64_t)Hkv * (Li + cost) : 0;
+    int64_t incl = wi;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    const int64_t excl = incl - wi;
+    const unsigned hit = __ballot_sync(0xffffffffu, wi > 0 && base + excl <= x && x < base + incl);
+    if (hit) {
+      const int k = __ffs(hit) - 1;
+      base += __shfl_sync(0xffffffffu, excl, k);
+      L = __shfl_sync(0xffffffffu, Li, k);
+      i += k;
+      return true;
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+    i += 32;
   }
-  w.done = false;
-  w.i = fi;
-  w.base = sh.found_base;
-  w.L = clamp_len(__ldg(prm.seq_lens + fi), cap);
-  w.Lnext = fi + 1 < S ? __ldg(prm.seq_lens + fi + 1) : 0;
-  const int64_t rel = lo - w.base;
-  w.h = (int)(rel / (w.L + cost));
-  const int64_t r = rel - (int64_t)w.h * (w.L + cost);  // offset inside unit (fi, h)
-  w.p = r <= cost ? 0 : (r - cost + w.P - 1) / w.P;
-  const int li = sh.last_i;
-  set_tail(w, li, sh.last_base, li >= 0 ? clamp_len(__ldg(prm.seq_lens + li), cap) : 0, lo);
+  return false;
+}
+
+// Warp-wide: sets up `w` (whose constant fields are already set) for range r,
+// moving the cursor (ci, cbase) forward. Returns false for an empty range.
+__device__ __forceinline__ bool warp_start_range(const DecodeParams& prm, SegmentWalker& w,
+                                                 int64_t r, int& ci, int64_t& cbase) {
+  const int64_t lo = w.cuts.lo(r), hi = w.cuts.lo(r + 1);
+  if (lo >= hi) return false;
+  int L = 0;
+  if (!warp_find_seq(prm, lo, ci, cbase, L)) return false;
+  int li = ci, lL = L;
+  int64_t lbase = cbase;
+  warp_find_seq(prm, hi - 1, li, lbase, lL);
+  const int fLn = ci + 1 < w.S ? __ldg(prm.seq_lens + ci + 1) : 0;
+  start_range(w, lo, hi, ci, cbase, L, fLn, li, lbase, lL);
+  return !w.done || w.tail_pending;
 }
 
 // ---- pieces of split units -------------------------------------------------
@@ -324,7 +417,7 @@ __device__ __forceinline__ bool complete_piece(const DecodeParams& prm, const Se
 // partial of their piece `s`. `flag` is a shared int private to these
 // threads; `sync` synchronises them.
 template <typename OT, typename Sync>
-__device__ void finish_piece(const DecodeParams& prm, const SegmentWalker& w, const Segment& s,
+__device__ void finish_piece(const DecodeParams& prm, const Cuts& cu, int64_t P, const Segment& s,
                              int tid, int nthreads, volatile int* flag, Sync sync) {
   __threadfence();
   sync();
@@ -336,11 +429,11 @@ __device__ void finish_piece(const DecodeParams& prm, const SegmentWalker& w, co
   for (int e = tid; e < g * D; e += nthreads) {
     const int j = e / D, d = e - j * D;
     float M = -INFINITY;
-    w.for_each_piece(s.first, s.len, [&](int slot) {
+    for_each_piece(cu, P, s.first, s.len, [&](int slot) {
       M = fmaxf(M, __ldcg(prm.ws_lse + (int64_t)slot * g + j));
     });
     float num = 0.f, den = 0.f;
-    w.for_each_piece(s.first, s.len, [&](int slot) {
+    for_each_piece(cu, P, s.first, s.len, [&](int slot) {
       const float wt = fast_exp2(__ldcg(prm.ws_lse + (int64_t)slot * g + j) - M);
       num = fmaf(wt, __ldcg(prm.ws_o + ((int64_t)slot * g + j) * D + d), num);
       den += wt;
