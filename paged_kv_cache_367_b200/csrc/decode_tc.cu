@@ -62,7 +62,7 @@ struct Cfg {
   static constexpr int kRed = (kRedO + 2 * kConsumerWarps * kHeads) * 4;
   static constexpr int kBar = (2 * NS + 4) * 8 + (NS + 2) * 48;  // barriers, descriptors
   static constexpr int kSmem = 1024 + NS * kStage + 2 * kRed + kBar +
-                               (int)sizeof(SchedShared) + 32;
+                               (int)sizeof(SchedShared) + (32 * 16 + 16) * 4 + 32 * 4 + 32;
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA exceeds 227 KB");
 };
 
@@ -203,44 +203,158 @@ __device__ __forceinline__ void named_sync_consumers() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
 }
 
-// Merge of all pieces of a split unit by one warp: lane j < g owns head j's
-// log-sum-exp bookkeeping, every lane owns D/32 dimensions of every head. The
-// pieces are enumerated from the schedule, so their loads are independent.
+// Merge of all pieces of a split unit by one warp. The pieces are listed 32
+// ranges at a time (a lane per range; a ballot numbers the non-empty ones, in
+// token order) into `wslot`, and taken 32 at a time, one per lane: each lane
+// reads its piece's log-sum-exp values, the warp reduces the per-head maxima,
+// the maxima and the pieces' weights go to shared scratch (`msc`, 16 floats;
+// `wsc`, 32 x 16 floats). Every lane then accumulates its D/32 columns of 8
+// heads at a time over the pieces, with the rows of several pieces loaded
+// before any is used, so that the merge costs about one memory latency per
+// group of pieces rather than one per piece and head.
 template <typename T, int D, int NT>
 __device__ void warp_merge_unit(const DecodeParams& prm, const Cuts& cu, int64_t P,
-                                const Segment& s, int lane) {
-  constexpr int V = D / 32;
+                                const Segment& s, int lane, float* wsc, float* msc,
+                                int* wslot) {
+  constexpr int V = D / 32, H = 8 * NT, HG = 8;
+  constexpr int PPS = 32 / (HG * V);  // pieces whose rows are in flight together
+  static_assert(V == 2 || V == 4, "rows are moved as float2 or float4");
   const int Hq = prm.num_heads, g = Hq / prm.num_kv_heads;
-  float M = -INFINITY;
-  for_each_piece(cu, P, s.first, s.len, [&](int slot) {
-    if (lane < g) M = fmaxf(M, __ldcg(prm.ws_lse + (int64_t)slot * g + lane));
-  });
-  float num[8 * NT][V];
-#pragma unroll
-  for (int j = 0; j < 8 * NT; ++j)
-#pragma unroll
-    for (int v = 0; v < V; ++v) num[j][v] = 0.f;
-  float den = 0.f;
-  for_each_piece(cu, P, s.first, s.len, [&](int slot) {
-    const float w = lane < g ? fast_exp2(__ldcg(prm.ws_lse + (int64_t)slot * g + lane) - M) : 0.f;
-    den += w;
-#pragma unroll
-    for (int j = 0; j < 8 * NT; ++j) {
-      const float wj = __shfl_sync(0xffffffffu, w, j);
-      if (j < g) {
-        const float* src = prm.ws_o + ((int64_t)slot * g + j) * D + lane * V;
-#pragma unroll
-        for (int v = 0; v < V; ++v) num[j][v] = fmaf(wj, __ldcg(src + v), num[j][v]);
+  const int64_t nparts = (s.len + P - 1) / P;
+  const int64_t r0 = cu.owner(s.first);
+  const int64_t r1 = cu.owner(s.first + (nparts - 1) * P);
+  // Writes the slots of pieces [b0, b0 + 32) to wslot; returns the piece count.
+  auto list = [&](int b0) {
+    int k = 0;
+    for (int64_t rb = r0; rb <= r1; rb += 32) {
+      const int64_t r = rb + lane;
+      bool has = false;
+      if (r <= r1) {
+        const int64_t s0 = r == r0 ? 0 : range_first_part(cu, r, s.first, P);
+        const int64_t s1 = r == r1 ? nparts : range_first_part(cu, r + 1, s.first, P);
+        has = s0 < s1;
       }
+      const unsigned m = __ballot_sync(0xffffffffu, has);
+      const int idx = k + __popc(m & ((1u << lane) - 1u)) - b0;
+      if (has && idx >= 0 && idx < 32) wslot[idx] = piece_slot(r, r0);
+      k += __popc(m);
     }
-  });
+    __syncwarp();
+    return k;
+  };
+  auto load_lse = [&](int b0, int n, float (&lk)[H]) {
 #pragma unroll
-  for (int j = 0; j < 8 * NT; ++j) {
-    const float dj = __shfl_sync(0xffffffffu, den, j);
-    if (j < g) {
-      T* dst = static_cast<T*>(prm.out) + ((int64_t)s.seq * Hq + s.head * g + j) * D + lane * V;
+    for (int j = 0; j < H; ++j) lk[j] = -INFINITY;
+    if (b0 + lane < n) {
+      const float* src = prm.ws_lse + (int64_t)wslot[lane] * g;
 #pragma unroll
-      for (int v = 0; v < V; ++v) dst[v] = from_f32<T>(num[j][v] / dj);
+      for (int j = 0; j < H; ++j)
+        if (j < g) lk[j] = __ldcg(src + j);
+    }
+  };
+  const int n = list(0);
+  float lk[H], M[H];
+#pragma unroll
+  for (int j = 0; j < H; ++j) M[j] = -INFINITY;
+  for (int b0 = 0; b0 < n; b0 += 32) {
+    if (b0 > 0) {
+      __syncwarp();
+      list(b0);
+    }
+    load_lse(b0, n, lk);
+#pragma unroll
+    for (int j = 0; j < H; ++j) M[j] = fmaxf(M[j], lk[j]);
+  }
+#pragma unroll
+  for (int j = 0; j < H; ++j)
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) M[j] = fmaxf(M[j], __shfl_xor_sync(0xffffffffu, M[j], o));
+  if (lane == 0) {
+#pragma unroll
+    for (int j = 0; j < H; ++j) msc[j] = M[j];
+  }
+  // Weights of pieces [b0, b0 + 32) for every head, from this lane's lk.
+  auto weights = [&](int b0) {
+    if (b0 + lane < n) {
+#pragma unroll
+      for (int j = 0; j < H; ++j) wsc[lane * H + j] = j < g ? fast_exp2(lk[j] - msc[j]) : 0.f;
+    }
+  };
+  if (n > 32) {
+    __syncwarp();
+    list(0);
+    load_lse(0, n, lk);
+  }
+  __syncwarp();
+  weights(0);
+  // Heads are accumulated 8 at a time; each group walks all pieces.
+  for (int h0 = 0; h0 < g; h0 += HG) {
+    float num[HG][V], den[HG];
+#pragma unroll
+    for (int j = 0; j < HG; ++j) {
+      den[j] = 0.f;
+#pragma unroll
+      for (int v = 0; v < V; ++v) num[j][v] = 0.f;
+    }
+    for (int b0 = 0; b0 < n; b0 += 32) {
+      if (n > 32 && (b0 > 0 || h0 > 0)) {  // the list and weights held another batch
+        list(b0);
+        load_lse(b0, n, lk);
+        weights(b0);
+      }
+      __syncwarp();
+      const int nb = min(32, n - b0);
+      for (int q = 0; q < nb; q += PPS) {
+        float r[PPS][HG][V];
+#pragma unroll
+        for (int p = 0; p < PPS; ++p) {
+          const int slot = wslot[min(q + p, nb - 1)];
+#pragma unroll
+          for (int j = 0; j < HG; ++j) {
+            if (h0 + j < g) {
+              const float* src = prm.ws_o + ((int64_t)slot * g + h0 + j) * D + lane * V;
+              if constexpr (V == 4) {
+                const float4 t = __ldcg(reinterpret_cast<const float4*>(src));
+                r[p][j][0] = t.x; r[p][j][1] = t.y; r[p][j][2] = t.z; r[p][j][3] = t.w;
+              } else {
+                const float2 t = __ldcg(reinterpret_cast<const float2*>(src));
+                r[p][j][0] = t.x; r[p][j][1] = t.y;
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int p = 0; p < PPS; ++p) {
+#pragma unroll
+          for (int j = 0; j < HG; ++j) {
+            if (h0 + j < g) {
+              const float wt = q + p < nb ? wsc[(q + p) * H + h0 + j] : 0.f;
+              den[j] += wt;
+#pragma unroll
+              for (int v = 0; v < V; ++v) num[j][v] = fmaf(wt, r[p][j][v], num[j][v]);
+            }
+          }
+        }
+      }
+      __syncwarp();
+    }
+#pragma unroll
+    for (int j = 0; j < HG; ++j) {
+      if (h0 + j < g) {
+        const float inv = 1.f / den[j];
+        float a, b;
+        T* dst = static_cast<T*>(prm.out) + ((int64_t)s.seq * Hq + s.head * g + h0 + j) * D +
+                 lane * V;
+        if constexpr (V == 4) {
+          uint2 w;
+          w.x = Mma<T>::pack(num[j][0] * inv, num[j][1] * inv, a, b);
+          w.y = Mma<T>::pack(num[j][2] * inv, num[j][3] * inv, a, b);
+          *reinterpret_cast<uint2*>(dst) = w;
+        } else {
+          *reinterpret_cast<uint32_t*>(dst) =
+              Mma<T>::pack(num[j][0] * inv, num[j][1] * inv, a, b);
+        }
+      }
     }
   }
 }
@@ -279,7 +393,10 @@ __global__ void __launch_bounds__(kThreads, MINB)
   ChunkDesc* desc = reinterpret_cast<ChunkDesc*>(rempty + 2);  // per stage
   ChunkDesc* hdesc = desc + NS;                                 // per hand-off buffer
   SchedShared* sched = reinterpret_cast<SchedShared*>(hdesc + 2);
-  volatile int* abort = reinterpret_cast<volatile int*>(sched + 1);
+  float* merge_scratch = reinterpret_cast<float*>(sched + 1);  // 32 x 16 floats, epilogue warp
+  float* merge_max = merge_scratch + 32 * 16;                         // 16, epilogue warp
+  int* merge_slots = reinterpret_cast<int*>(merge_max + 16);          // 32, epilogue warp
+  volatile int* abort = reinterpret_cast<volatile int*>(merge_slots + 32);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -450,62 +567,86 @@ __global__ void __launch_bounds__(kThreads, MINB)
       const bool whole = seg.t0 == 0 && seg.t1 == seg.len;
       const int i = seg.seq, h = seg.head;
       {
-        // lane j < g: per-head maximum, warp weights and denominator
-        float M = -INFINITY, wx[kConsumerWarps], Lsum = 0.f;
+        // Lanes j < g: per-head maximum, warp weights and 1/denominator, into
+        // the shared scratch (each head: 4 weights, the reciprocal, the lse).
         if (lane < g) {
+          float mx = -INFINITY;
 #pragma unroll
-          for (int x = 0; x < kConsumerWarps; ++x) M = fmaxf(M, rm[x * H + lane]);
+          for (int x = 0; x < kConsumerWarps; ++x) mx = fmaxf(mx, rm[x * H + lane]);
+          float lsum = 0.f;
 #pragma unroll
           for (int x = 0; x < kConsumerWarps; ++x) {
-            wx[x] = fast_exp2(rm[x * H + lane] - M);
-            Lsum = fmaf(wx[x], rl[x * H + lane], Lsum);
+            const float wt = fast_exp2(rm[x * H + lane] - mx);
+            merge_scratch[lane * 8 + x] = wt;
+            lsum = fmaf(wt, rl[x * H + lane], lsum);
           }
-        } else {
-#pragma unroll
-          for (int x = 0; x < kConsumerWarps; ++x) wx[x] = 0.f;
+          merge_scratch[lane * 8 + 4] = vscale / lsum;
+          if (!whole) {
+            const int64_t rowp = (int64_t)own_piece_slot(d.range, seg) * g + lane;
+            prm.ws_lse[rowp] = mx + fast_log2(lsum);
+          }
         }
+        __syncwarp();
 #pragma unroll
         for (int j = 0; j < H; ++j) {
-          float w[kConsumerWarps];
-#pragma unroll
-          for (int x = 0; x < kConsumerWarps; ++x) w[x] = __shfl_sync(0xffffffffu, wx[x], j);
-          const float Lj = __shfl_sync(0xffffffffu, Lsum, j) / vscale;
-          const float Mj = __shfl_sync(0xffffffffu, M, j);
           if (j < g) {
+            const float* sc = merge_scratch + j * 8;
             float o[V];
 #pragma unroll
             for (int v = 0; v < V; ++v) o[v] = 0.f;
 #pragma unroll
             for (int x = 0; x < kConsumerWarps; ++x) {
+              const float wt = sc[x];
               const float* src = ro + (x * H + j) * D + lane * V;
+              if constexpr (V == 4) {
+                const float4 r = *reinterpret_cast<const float4*>(src);
+                o[0] = fmaf(wt, r.x, o[0]);
+                o[1] = fmaf(wt, r.y, o[1]);
+                o[2] = fmaf(wt, r.z, o[2]);
+                o[3] = fmaf(wt, r.w, o[3]);
+              } else {
 #pragma unroll
-              for (int v = 0; v < V; ++v) o[v] = fmaf(w[x], src[v], o[v]);
+                for (int v = 0; v < V; ++v) o[v] = fmaf(wt, src[v], o[v]);
+              }
             }
+            const float inv = sc[4];
+#pragma unroll
+            for (int v = 0; v < V; ++v) o[v] *= inv;
             const int qh = h * g + j;
             if (whole) {
               T* dst = static_cast<T*>(prm.out) + ((int64_t)i * Hq + qh) * D + lane * V;
+              if constexpr (V == 4) {
+                uint2 pk;
+                float r0, r1;
+                pk.x = Mma<T>::pack(o[0], o[1], r0, r1);
+                pk.y = Mma<T>::pack(o[2], o[3], r0, r1);
+                *reinterpret_cast<uint2*>(dst) = pk;
+              } else {
 #pragma unroll
-              for (int v = 0; v < V; ++v) dst[v] = from_f32<T>(o[v] / Lj);
+                for (int v = 0; v < V; ++v) dst[v] = from_f32<T>(o[v]);
+              }
             } else {
               const int64_t rowp = (int64_t)own_piece_slot(d.range, seg) * g + j;
               float* dst = prm.ws_o + rowp * D + lane * V;
+              if constexpr (V == 4) {
+                *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+              } else {
 #pragma unroll
-              for (int v = 0; v < V; ++v) dst[v] = o[v] / Lj;
-              if (lane == 0) prm.ws_lse[rowp] = Mj + fast_log2(Lj * vscale);
+                for (int v = 0; v < V; ++v) dst[v] = o[v];
+              }
             }
           }
         }
+        __syncwarp();  // the scratch is rewritten by the next segment
       }
       __syncwarp();
       mbar_arrive(rempty + rb);  // the hand-off buffer may be refilled
       if (!whole) {
-        __threadfence();
-        __syncwarp();
+        __syncwarp();  // orders the lanes' partial stores before lane 0's release
         const int last = lane == 0 ? (int)complete_piece(prm, seg) : 0;
-        if (__shfl_sync(0xffffffffu, last, 0)) {
-          __threadfence();
-          warp_merge_unit<T, D, NT>(prm, cuts, walker.P, seg, lane);
-        }
+        if (__shfl_sync(0xffffffffu, last, 0))  // lane 0 acquired the other pieces
+          warp_merge_unit<T, D, NT>(prm, cuts, walker.P, seg, lane, merge_scratch,
+                                    merge_max, merge_slots);
       }
     }
     return;

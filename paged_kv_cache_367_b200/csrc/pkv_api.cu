@@ -169,7 +169,8 @@ int paged_attention_decode(void* out, const void* query, const void* k_cache,
   const int64_t cap = (int64_t)max_blocks_per_seq * block_size;
   prm.len_cap = (int)(cap < max_seq_len ? cap : max_seq_len);
   prm.part = parts > 1 ? partition_size : 0;
-  prm.unit_cost = 64;  // about one chunk: a segment's set-up and epilogue, in tokens
+  prm.unit_cost = 24;  // a segment's set-up and hand-off, in tokens (measured)
+  prm.unit_round = 64;  // the tensor-core kernel streams 64-token chunks
   prm.dyn_ranges = 0;  // the tensor-core launcher enables dynamic ranges
   prm.static_share = 1024;
   prm.score_scale = scale * kLog2e;

@@ -1,10 +1,12 @@
 // Device-side work split for paged decode.
 //
 // A unit is one (sequence, KV head) pair; its work is the sequence's tokens
-// plus a fixed per-unit cost (the set-up and epilogue a unit costs, counted in
-// tokens). Units are laid end to end in (sequence, head) order, giving every
-// unit a work range in [0, W), W = sum over units of (cost + L). Partition p of
-// a unit (tokens [p P, (p + 1) P)) is an item at work offset
+// rounded up to the kernel's chunk (a kernel streams whole chunks, so a partly
+// filled chunk costs like a full one) plus a fixed per-unit cost (set-up and
+// epilogue, counted in tokens). Units are laid end to end in (sequence, head)
+// order, giving every unit a work range in [0, W), W = sum over units of
+// (cost + Lw), Lw = L rounded up to the chunk. Partition p of a unit (tokens
+// [p P, (p + 1) P)) is an item at work offset
 //   first + p P,   first = unit start + cost.
 // [0, W) is cut into ranges (Cuts): G "static" ranges of equal size cover
 // [0, Ws) and are taken by CTA r = blockIdx.x; Rd "dynamic" ranges of equal size
@@ -41,6 +43,7 @@ struct DecodeParams {
   int len_cap;        // seq_lens are clamped to [0, len_cap]
   int part;           // partition size in tokens, 0 = never split
   int unit_cost;      // work charged per non-empty unit, in tokens
+  int unit_round;     // unit lengths are rounded up to a multiple of this (the chunk)
   int dyn_ranges;     // number of dynamic ranges (0: every range is static)
   int static_share;   // share of the work in static ranges, in 1/1024 (when dyn_ranges > 0)
   float score_scale;  // scale * log2(e): scores are kept in the base-2 domain
@@ -56,6 +59,11 @@ constexpr int64_t kNoSplit = int64_t(1) << 30;
 
 __host__ __device__ __forceinline__ int clamp_len(int L, int cap) {
   return L < 0 ? 0 : (L > cap ? cap : L);
+}
+
+// Work of a unit of L tokens (0 for an empty unit).
+__host__ __device__ __forceinline__ int64_t unit_work(int L, int cost, int round) {
+  return L > 0 ? (int64_t)(L + round - 1) / round * round + cost : 0;
 }
 
 __host__ __device__ __forceinline__ int load_len(const int32_t* p) {
@@ -134,12 +142,14 @@ __host__ __device__ void for_each_piece(const Cuts& cu, int64_t P, int64_t first
 }
 
 // Walks the segments of one range. If the range ends inside a unit that starts
-// in it, that piece (the "tail") comes first and the walk from the range's start
-// stops short of it: its partial is then ready early, and the range ends on
-// work that needs no merge.
+// in it, that piece (the "tail") is taken early: right after the range's first
+// segment when that segment is itself a piece of a unit begun in an earlier
+// range (a "head"), else first; the walk from the range's start stops short of
+// it. Pieces, whose partials need merging, thus come before whole units, and a
+// range ends on work that needs no merge.
 struct SegmentWalker {
   const int32_t* seq_lens;
-  int S, Hkv, cap, cost;
+  int S, Hkv, cap, cost, round;
   int64_t P;     // partition size, kNoSplit when the unit is never cut
   Cuts cuts;
   int64_t hi;    // where the walk from the range's start stops
@@ -149,18 +159,23 @@ struct SegmentWalker {
   int64_t p;     // first partition of unit (i, h) still to take
   bool done;
   bool tail_pending;
+  bool started;   // a segment has been returned
+  bool has_head;  // the walk from the range's start begins inside a unit
   Segment tail;
 
   __host__ __device__ bool next(Segment& s) {
-    if (tail_pending) {
+    // The tail goes first, unless the range begins with a head piece (a unit
+    // begun in an earlier range, p > 0): then right after it.
+    if (tail_pending && (started || !has_head)) {
       tail_pending = false;
+      started = true;
       s = tail;
       return true;
     }
     while (!done) {
       if (i >= S) { done = true; break; }
       if (h >= Hkv || L == 0) {
-        base += L > 0 ? (int64_t)Hkv * (L + cost) : 0;
+        base += (int64_t)Hkv * unit_work(L, cost, round);
         ++i;
         h = 0;
         p = 0;
@@ -171,7 +186,7 @@ struct SegmentWalker {
         continue;
       }
       if (p * P >= L) { ++h; p = 0; continue; }  // unit's rest belongs to earlier ranges
-      const int64_t first = base + (int64_t)h * (L + cost) + cost;
+      const int64_t first = base + (int64_t)h * unit_work(L, cost, round) + cost;
       if (first + p * P >= hi) { done = true; break; }
       const int64_t nparts = (L + P - 1) / P;
       int64_t q = (hi - 1 - first) / P;
@@ -188,6 +203,13 @@ struct SegmentWalker {
         ++h;
         p = 0;
       }
+      started = true;
+      return true;
+    }
+    if (tail_pending) {
+      tail_pending = false;
+      started = true;
+      s = tail;
       return true;
     }
     return false;
@@ -202,6 +224,8 @@ __host__ __device__ __forceinline__ void start_range(SegmentWalker& w, int64_t l
                                                      int li, int64_t lbase, int lL) {
   w.hi = hi;
   w.tail_pending = false;
+  w.started = false;
+  w.has_head = false;
   if (lo >= hi || fi < 0 || fL <= 0) {
     w.done = true;
     w.i = w.S;
@@ -217,16 +241,19 @@ __host__ __device__ __forceinline__ void start_range(SegmentWalker& w, int64_t l
   w.base = fbase;
   w.L = fL;
   w.Lnext = fLnext;
+  const int64_t fw = unit_work(fL, w.cost, w.round);
   const int64_t rel = lo - fbase;
-  w.h = (int)(rel / (fL + w.cost));
-  const int64_t r = rel - (int64_t)w.h * (fL + w.cost);  // offset inside unit (fi, h)
+  w.h = (int)(rel / fw);
+  const int64_t r = rel - (int64_t)w.h * fw;  // offset inside unit (fi, h)
   w.p = r <= w.cost ? 0 : (r - w.cost + w.P - 1) / w.P;
+  w.has_head = w.p > 0 && w.p * w.P < fL && fbase + (int64_t)w.h * fw + w.cost + w.p * w.P < hi;
   // The tail: the last item lies in a unit that starts at or after lo and
   // continues past hi.
   if (li < 0 || lL <= 0) return;
+  const int64_t lw = unit_work(lL, w.cost, w.round);
   const int64_t lrel = (hi - 1) - lbase;
-  const int hh = (int)(lrel / (lL + w.cost));
-  const int64_t first = lbase + (int64_t)hh * (lL + w.cost) + w.cost;
+  const int hh = (int)(lrel / lw);
+  const int64_t first = lbase + (int64_t)hh * lw + w.cost;
   if (hi - 1 < first || first < lo) return;
   const int64_t nparts = (lL + w.P - 1) / w.P;
   const int64_t q = (hi - 1 - first) / w.P;
@@ -282,12 +309,13 @@ struct SchedShared {
 template <typename OT>
 __device__ void init_walker(const DecodeParams& prm, SchedShared& sh, SegmentWalker& w) {
   const int S = prm.num_seqs, Hkv = prm.num_kv_heads, cap = prm.len_cap, cost = prm.unit_cost;
+  const int round = prm.unit_round;
   const int G = gridDim.x, c = blockIdx.x;
   // Pass 1: total work; zero rows of empty sequences.
   int64_t sum = 0;
   for (int i = threadIdx.x; i < S; i += blockDim.x) {
     const int L = clamp_len(__ldg(prm.seq_lens + i), cap);
-    sum += L > 0 ? (int64_t)Hkv * (L + cost) : 0;
+    sum += (int64_t)Hkv * unit_work(L, cost, round);
     if (L == 0 && i % G == c) {
       OT* o = static_cast<OT*>(prm.out) + (int64_t)i * prm.num_heads * prm.head_dim;
       for (int e = 0; e < prm.num_heads * prm.head_dim; ++e) o[e] = from_f32<OT>(0.f);
@@ -310,7 +338,7 @@ __device__ void init_walker(const DecodeParams& prm, SchedShared& sh, SegmentWal
   for (int i0 = 0; i0 < S; i0 += blockDim.x) {
     const int i = i0 + threadIdx.x;
     const int L = i < S ? clamp_len(__ldg(prm.seq_lens + i), cap) : 0;
-    const int64_t wi = L > 0 ? (int64_t)Hkv * (L + cost) : 0;
+    const int64_t wi = (int64_t)Hkv * unit_work(L, cost, round);
     int64_t chunk_tot;
     const int64_t incl = block_inclusive_scan(wi, sh.scan, chunk_tot);
     const int64_t b = carry + incl - wi;
@@ -338,6 +366,7 @@ __device__ void init_walker(const DecodeParams& prm, SchedShared& sh, SegmentWal
   w.Hkv = Hkv;
   w.cap = cap;
   w.cost = cost;
+  w.round = round;
   w.P = prm.part > 0 ? prm.part : kNoSplit;
   w.cuts = cu;
   const int fi = sh.f_i, li = sh.l_i;
@@ -358,7 +387,7 @@ __device__ __forceinline__ bool warp_find_seq(const DecodeParams& prm, int64_t x
   while (i < S) {
     const int idx = i + lane;
     const int Li = idx < S ? clamp_len(__ldg(prm.seq_lens + idx), cap) : 0;
-    const int64_t wi = Li > 0 ? (int64_t)Hkv * (Li + cost) : 0;
+    const int64_t wi = (int64_t)Hkv * unit_work(Li, cost, prm.unit_round);
     int64_t incl = wi;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -406,10 +435,16 @@ __device__ __forceinline__ bool warp_start_range(const DecodeParams& prm, Segmen
 // the blockwise form of the softmax. No CTA ever waits for another.
 
 // Adds piece `s` to its unit's counter; true for the piece that completes it.
-// Call from one thread, after the piece's partial is written and fenced.
+// Call from one thread once the piece's partial is written by the threads it is
+// synchronised with: the addition releases those writes and acquires the other
+// pieces' (acq_rel at GPU scope).
 __device__ __forceinline__ bool complete_piece(const DecodeParams& prm, const Segment& s) {
   const int64_t u = (int64_t)s.seq * prm.num_kv_heads + s.head;
-  const int before = atomicAdd(prm.ws_done + u, s.t1 - s.t0);
+  int before;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;"
+               : "=r"(before)
+               : "l"(prm.ws_done + u), "r"(s.t1 - s.t0)
+               : "memory");
   return before + (s.t1 - s.t0) == s.len;
 }
 

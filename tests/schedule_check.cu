@@ -21,12 +21,12 @@
 using namespace pkv;
 
 // Sequential search: the sequence holding offset x (-1 if none).
-static int find_seq(const std::vector<int32_t>& lens, int Hkv, int cap, int cost, int64_t x,
-                    int64_t* base_out, int* L_out) {
+static int find_seq(const std::vector<int32_t>& lens, int Hkv, int cap, int cost, int round,
+                    int64_t x, int64_t* base_out, int* L_out) {
   int64_t base = 0;
   for (int i = 0; i < (int)lens.size(); ++i) {
     const int L = clamp_len(lens[i], cap);
-    const int64_t wi = L > 0 ? (int64_t)Hkv * (L + cost) : 0;
+    const int64_t wi = (int64_t)Hkv * unit_work(L, cost, round);
     if (wi > 0 && base <= x && x < base + wi) {
       *base_out = base;
       *L_out = L;
@@ -37,14 +37,11 @@ static int find_seq(const std::vector<int32_t>& lens, int Hkv, int cap, int cost
   return -1;
 }
 
-static int check(const std::vector<int32_t>& lens, int Hkv, int cap, int part, int cost, int G,
-                 int Rd, int share) {
+static int check(const std::vector<int32_t>& lens, int Hkv, int cap, int part, int cost, int round,
+                 int G, int Rd, int share) {
   const int S = (int)lens.size();
   int64_t W = 0;
-  for (int L : lens) {
-    const int c = clamp_len(L, cap);
-    W += c > 0 ? (int64_t)Hkv * (c + cost) : 0;
-  }
+  for (int L : lens) W += (int64_t)Hkv * unit_work(clamp_len(L, cap), cost, round);
   if (W == 0) return 0;
   const int64_t P = part > 0 ? part : kNoSplit;
   const Cuts cu = make_cuts(W, G, Rd, share);
@@ -62,14 +59,15 @@ static int check(const std::vector<int32_t>& lens, int Hkv, int cap, int part, i
       if (lo < hi && cu.owner(off) != r) return 13;
     SegmentWalker w;
     w.seq_lens = lens.data(); w.S = S; w.Hkv = Hkv; w.cap = cap; w.cost = cost; w.P = P;
+    w.round = round;
     w.cuts = cu;
     int64_t fbase = 0, lbase = 0;
     int fL = 0, lL = 0;
-    const int fi = lo < hi ? find_seq(lens, Hkv, cap, cost, lo, &fbase, &fL) : -1;
-    const int li = lo < hi ? find_seq(lens, Hkv, cap, cost, hi - 1, &lbase, &lL) : -1;
+    const int fi = lo < hi ? find_seq(lens, Hkv, cap, cost, round, lo, &fbase, &fL) : -1;
+    const int li = lo < hi ? find_seq(lens, Hkv, cap, cost, round, hi - 1, &lbase, &lL) : -1;
     const int fLn = fi >= 0 && fi + 1 < S ? lens[fi + 1] : 0;
     start_range(w, lo, hi, fi, fbase, fL, fLn, li, lbase, lL);
-    bool first_seg = true;
+    bool first_seg = true, prev_head = false, seen_whole = false;
     Segment s;
     while (w.next(s)) {
       if (s.t0 >= s.t1 || s.t1 > s.len) return 1;
@@ -78,8 +76,12 @@ static int check(const std::vector<int32_t>& lens, int Hkv, int cap, int part, i
       // ownership: the segment's first partition lies in this range
       const int64_t off = s.first + s.t0;
       if (off < lo || off >= hi) return 6;
-      // a piece that starts its unit and ends inside it comes first
-      if (s.t0 == 0 && s.t1 < s.len && !first_seg) return 10;
+      // pieces come before whole units: a piece that starts its unit and ends
+      // inside it is first or follows a piece that starts inside its unit
+      if (s.t0 == 0 && s.t1 < s.len && !(first_seg || prev_head)) return 10;
+      if (!(s.t0 == 0 && s.t1 == s.len) && seen_whole) return 14;
+      seen_whole = seen_whole || (s.t0 == 0 && s.t1 == s.len);
+      prev_head = first_seg && s.t0 > 0;
       first_seg = false;
       std::vector<char>& v = seen[s.seq * Hkv + s.head];
       for (int t = s.t0; t < s.t1; ++t) {
@@ -130,10 +132,11 @@ int main() {
     const int G = 1 + rand() % 600;
     const int Rd = (rand() % 2) ? 0 : rand() % (2 * G + 1);
     const int share = rand() % 1025;
-    const int r = check(lens, Hkv, cap, part, cost, G, Rd, share);
+    const int round = (rand() % 2) ? 1 : (8 << (rand() % 4));
+    const int r = check(lens, Hkv, cap, part, cost, round, G, Rd, share);
     if (r) {
-      printf("FAIL code %d: S=%d Hkv=%d cap=%d part=%d cost=%d G=%d Rd=%d share=%d\n", r, S,
-             Hkv, cap, part, cost, G, Rd, share);
+      printf("FAIL code %d: S=%d Hkv=%d cap=%d part=%d cost=%d round=%d G=%d Rd=%d share=%d\n",
+             r, S, Hkv, cap, part, cost, round, G, Rd, share);
       return 1;
     }
     ++cases;
