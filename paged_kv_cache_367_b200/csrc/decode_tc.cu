@@ -203,23 +203,36 @@ __device__ __forceinline__ void named_sync_consumers() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
 }
 
+// 16-byte copy global -> shared that completes asynchronously (cp.async).
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
+               : "memory");
+}
+// Waits for this thread's cp.async copies.
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // Merge of all pieces of a split unit by one warp. The pieces are listed 32
 // ranges at a time (a lane per range; a ballot numbers the non-empty ones, in
 // token order) into `wslot`, and taken 32 at a time, one per lane: each lane
 // reads its piece's log-sum-exp values, the warp reduces the per-head maxima,
-// the maxima and the pieces' weights go to shared scratch (`msc`, 16 floats;
-// `wsc`, 32 x 16 floats). Every lane then accumulates its D/32 columns of 8
-// heads at a time over the pieces, with the rows of several pieces loaded
-// before any is used, so that the merge costs about one memory latency per
-// group of pieces rather than one per piece and head.
+// and the maxima and the pieces' weights go to shared scratch (`msc`, 16
+// floats; `wsc`, 32 x 16 floats). The pieces' partial rows are then brought
+// into `stage` (stage_floats floats of shared memory the warp owns meanwhile)
+// as many pieces at a time as fit, by asynchronous 16-byte copies that are all
+// in flight together, and each lane accumulates its D/32 columns of every head
+// from there: a merge costs one memory latency per staging round rather than
+// one per piece and head.
 template <typename T, int D, int NT>
 __device__ void warp_merge_unit(const DecodeParams& prm, const Cuts& cu, int64_t P,
-                                const Segment& s, int lane, float* wsc, float* msc,
-                                int* wslot) {
-  constexpr int V = D / 32, H = 8 * NT, HG = 8;
-  constexpr int PPS = 32 / (HG * V);  // pieces whose rows are in flight together
-  static_assert(V == 2 || V == 4, "rows are moved as float2 or float4");
+                                const Segment& s, int lane, float* wsc, float* msc, int* wslot,
+                                float* stage, int stage_floats) {
+  constexpr int V = D / 32, H = 8 * NT;
+  static_assert(V == 2 || V == 4, "rows are read as float2 or float4");
   const int Hq = prm.num_heads, g = Hq / prm.num_kv_heads;
+  const int rowf = g * D;                 // floats of one piece's partial rows
+  const int B = stage_floats / rowf;      // pieces per staging round (>= 4)
   const int64_t nparts = (s.len + P - 1) / P;
   const int64_t r0 = cu.owner(s.first);
   const int64_t r1 = cu.owner(s.first + (nparts - 1) * P);
@@ -252,7 +265,19 @@ __device__ void warp_merge_unit(const DecodeParams& prm, const Cuts& cu, int64_t
         if (j < g) lk[j] = __ldcg(src + j);
     }
   };
+  // Copies the partial rows of pieces [q, q + nq) of the listed batch into the
+  // stage (not waited for).
+  auto stage_rows = [&](int q, int nq) {
+    for (int p = 0; p < nq; ++p) {
+      const float* src = prm.ws_o + (int64_t)wslot[q + p] * rowf;
+      for (int e = lane * 4; e < rowf; e += 128) cp_async16(stage + p * rowf + e, src + e);
+    }
+  };
   const int n = list(0);
+  // The first staging round's copies are issued before the log-sum-exp loads,
+  // so both wait out one memory latency together.
+  const int B0 = min(B, min(32, n));
+  stage_rows(0, B0);
   float lk[H], M[H];
 #pragma unroll
   for (int j = 0; j < H; ++j) M[j] = -INFINITY;
@@ -273,87 +298,67 @@ __device__ void warp_merge_unit(const DecodeParams& prm, const Cuts& cu, int64_t
 #pragma unroll
     for (int j = 0; j < H; ++j) msc[j] = M[j];
   }
-  // Weights of pieces [b0, b0 + 32) for every head, from this lane's lk.
-  auto weights = [&](int b0) {
+  float num[H][V], den[H];
+#pragma unroll
+  for (int j = 0; j < H; ++j) {
+    den[j] = 0.f;
+#pragma unroll
+    for (int v = 0; v < V; ++v) num[j][v] = 0.f;
+  }
+  for (int b0 = 0; b0 < n; b0 += 32) {
+    __syncwarp();
+    if (n > 32) {  // the list and log-sum-exp values held another batch
+      list(b0);
+      load_lse(b0, n, lk);
+    }
     if (b0 + lane < n) {
 #pragma unroll
       for (int j = 0; j < H; ++j) wsc[lane * H + j] = j < g ? fast_exp2(lk[j] - msc[j]) : 0.f;
     }
-  };
-  if (n > 32) {
     __syncwarp();
-    list(0);
-    load_lse(0, n, lk);
+    const int nb = min(32, n - b0);
+    for (int q = 0; q < nb; q += B) {
+      const int nq = min(B, nb - q);
+      if (b0 > 0 || q > 0) stage_rows(q, nq);  // the first round is in flight already
+      cp_async_wait_all();
+      __syncwarp();
+      for (int p = 0; p < nq; ++p) {
+#pragma unroll
+        for (int j = 0; j < H; ++j) {
+          if (j < g) {
+            const float wt = wsc[(q + p) * H + j];
+            const float* x = stage + p * rowf + j * D + lane * V;
+            den[j] += wt;
+            if constexpr (V == 4) {
+              const float4 t = *reinterpret_cast<const float4*>(x);
+              num[j][0] = fmaf(wt, t.x, num[j][0]);
+              num[j][1] = fmaf(wt, t.y, num[j][1]);
+              num[j][2] = fmaf(wt, t.z, num[j][2]);
+              num[j][3] = fmaf(wt, t.w, num[j][3]);
+            } else {
+              const float2 t = *reinterpret_cast<const float2*>(x);
+              num[j][0] = fmaf(wt, t.x, num[j][0]);
+              num[j][1] = fmaf(wt, t.y, num[j][1]);
+            }
+          }
+        }
+      }
+      __syncwarp();  // the stage is refilled next round
+    }
   }
-  __syncwarp();
-  weights(0);
-  // Heads are accumulated 8 at a time; each group walks all pieces.
-  for (int h0 = 0; h0 < g; h0 += HG) {
-    float num[HG][V], den[HG];
 #pragma unroll
-    for (int j = 0; j < HG; ++j) {
-      den[j] = 0.f;
-#pragma unroll
-      for (int v = 0; v < V; ++v) num[j][v] = 0.f;
-    }
-    for (int b0 = 0; b0 < n; b0 += 32) {
-      if (n > 32 && (b0 > 0 || h0 > 0)) {  // the list and weights held another batch
-        list(b0);
-        load_lse(b0, n, lk);
-        weights(b0);
-      }
-      __syncwarp();
-      const int nb = min(32, n - b0);
-      for (int q = 0; q < nb; q += PPS) {
-        float r[PPS][HG][V];
-#pragma unroll
-        for (int p = 0; p < PPS; ++p) {
-          const int slot = wslot[min(q + p, nb - 1)];
-#pragma unroll
-          for (int j = 0; j < HG; ++j) {
-            if (h0 + j < g) {
-              const float* src = prm.ws_o + ((int64_t)slot * g + h0 + j) * D + lane * V;
-              if constexpr (V == 4) {
-                const float4 t = __ldcg(reinterpret_cast<const float4*>(src));
-                r[p][j][0] = t.x; r[p][j][1] = t.y; r[p][j][2] = t.z; r[p][j][3] = t.w;
-              } else {
-                const float2 t = __ldcg(reinterpret_cast<const float2*>(src));
-                r[p][j][0] = t.x; r[p][j][1] = t.y;
-              }
-            }
-          }
-        }
-#pragma unroll
-        for (int p = 0; p < PPS; ++p) {
-#pragma unroll
-          for (int j = 0; j < HG; ++j) {
-            if (h0 + j < g) {
-              const float wt = q + p < nb ? wsc[(q + p) * H + h0 + j] : 0.f;
-              den[j] += wt;
-#pragma unroll
-              for (int v = 0; v < V; ++v) num[j][v] = fmaf(wt, r[p][j][v], num[j][v]);
-            }
-          }
-        }
-      }
-      __syncwarp();
-    }
-#pragma unroll
-    for (int j = 0; j < HG; ++j) {
-      if (h0 + j < g) {
-        const float inv = 1.f / den[j];
-        float a, b;
-        T* dst = static_cast<T*>(prm.out) + ((int64_t)s.seq * Hq + s.head * g + h0 + j) * D +
-                 lane * V;
-        if constexpr (V == 4) {
-          uint2 w;
-          w.x = Mma<T>::pack(num[j][0] * inv, num[j][1] * inv, a, b);
-          w.y = Mma<T>::pack(num[j][2] * inv, num[j][3] * inv, a, b);
-          *reinterpret_cast<uint2*>(dst) = w;
-        } else {
-          *reinterpret_cast<uint32_t*>(dst) =
-              Mma<T>::pack(num[j][0] * inv, num[j][1] * inv, a, b);
-        }
+  for (int j = 0; j < H; ++j) {
+    if (j < g) {
+      const float inv = 1.f / den[j];
+      float a, b;
+      T* dst = static_cast<T*>(prm.out) + ((int64_t)s.seq * Hq + s.head * g + j) * D + lane * V;
+      if constexpr (V == 4) {
+        uint2 w;
+        w.x = Mma<T>::pack(num[j][0] * inv, num[j][1] * inv, a, b);
+        w.y = Mma<T>::pack(num[j][2] * inv, num[j][3] * inv, a, b);
+        *reinterpret_cast<uint2*>(dst) = w;
+      } else {
+        *reinterpret_cast<uint32_t*>(dst) = Mma<T>::pack(num[j][0] * inv, num[j][1] * inv, a, b);
       }
     }
   }
@@ -639,15 +644,14 @@ __global__ void __launch_bounds__(kThreads, MINB)
         }
         __syncwarp();  // the scratch is rewritten by the next segment
       }
-      __syncwarp();
-      mbar_arrive(rempty + rb);  // the hand-off buffer may be refilled
+      __syncwarp();  // also orders the lanes' partial stores before lane 0's release
       if (!whole) {
-        __syncwarp();  // orders the lanes' partial stores before lane 0's release
         const int last = lane == 0 ? (int)complete_piece(prm, seg) : 0;
         if (__shfl_sync(0xffffffffu, last, 0))  // lane 0 acquired the other pieces
-          warp_merge_unit<T, D, NT>(prm, cuts, walker.P, seg, lane, merge_scratch,
-                                    merge_max, merge_slots);
+          warp_merge_unit<T, D, NT>(prm, cuts, walker.P, seg, lane, merge_scratch, merge_max,
+                                    merge_slots, red + rb * (C::kRed / 4), C::kRed / 4);
       }
+      mbar_arrive(rempty + rb);  // the hand-off buffer (the merge's stage) may be refilled
     }
     return;
   }

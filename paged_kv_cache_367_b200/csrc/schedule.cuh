@@ -294,12 +294,40 @@ __device__ __forceinline__ int64_t block_inclusive_scan(int64_t v, int64_t* sm32
   return v;
 }
 
+constexpr int kInitLens = 256;  // batches of at most this many sequences are set up in one pass
+
 struct SchedShared {
   int64_t scan[32];
   int64_t f_base, l_base, d_base;
   Cuts cuts;
   int f_i, l_i, d_i;
+  int lens[kInitLens];  // raw seq_lens, in the one-pass set-up
 };
+
+// Zero rows of sequence i if it is empty and this CTA owns it (i % G == c).
+template <typename OT>
+__device__ __forceinline__ void zero_empty_rows(const DecodeParams& prm, int i, int L, int G,
+                                                int c) {
+  if (i < prm.num_seqs && L == 0 && i % G == c) {
+    OT* o = static_cast<OT*>(prm.out) + (int64_t)i * prm.num_heads * prm.head_dim;
+    for (int e = 0; e < prm.num_heads * prm.head_dim; ++e) o[e] = from_f32<OT>(0.f);
+  }
+}
+
+// Records sequence i (work [b, b + wi)) if it holds offset lo, hi - 1 or Ws.
+__device__ __forceinline__ void mark_range_seqs(SchedShared& sh, int i, int64_t b, int64_t wi,
+                                                int64_t lo, int64_t hi, int64_t ws) {
+  if (wi <= 0) return;
+  if (lo < hi && b <= lo && lo < b + wi) {
+    sh.f_i = i;
+    sh.f_base = b;
+  }
+  if (lo < hi && b <= hi - 1 && hi - 1 < b + wi) {
+    sh.l_i = i;
+    sh.l_base = b;
+  }
+  if (b <= ws && ws < b + wi) sh.d_i = i;
+}
 
 // Sets up this CTA's walker for its static range r = blockIdx.x (all threads
 // must call it; ends with __syncthreads), leaves the cuts in sh.cuts and the
@@ -311,56 +339,72 @@ __device__ void init_walker(const DecodeParams& prm, SchedShared& sh, SegmentWal
   const int S = prm.num_seqs, Hkv = prm.num_kv_heads, cap = prm.len_cap, cost = prm.unit_cost;
   const int round = prm.unit_round;
   const int G = gridDim.x, c = blockIdx.x;
-  // Pass 1: total work; zero rows of empty sequences.
-  int64_t sum = 0;
-  for (int i = threadIdx.x; i < S; i += blockDim.x) {
-    const int L = clamp_len(__ldg(prm.seq_lens + i), cap);
-    sum += (int64_t)Hkv * unit_work(L, cost, round);
-    if (L == 0 && i % G == c) {
-      OT* o = static_cast<OT*>(prm.out) + (int64_t)i * prm.num_heads * prm.head_dim;
-      for (int e = 0; e < prm.num_heads * prm.head_dim; ++e) o[e] = from_f32<OT>(0.f);
-    }
-  }
-  int64_t W;
-  block_inclusive_scan(sum, sh.scan, W);
-  const Cuts cu = make_cuts(W, G, prm.dyn_ranges, prm.static_share);
-  const int64_t lo = cu.lo(c), hi = cu.lo(c + 1), ws = cu.Ws;
-  // Pass 2: the sequences holding offsets lo, hi - 1 and Ws.
+  int64_t W, lo, hi, ws;
+  Cuts cu;
   if (threadIdx.x == 0) {
     sh.f_i = -1;
     sh.l_i = -1;
     sh.d_i = S;
-    sh.d_base = W;
-    sh.cuts = cu;
   }
-  __syncthreads();
-  int64_t carry = 0;
-  for (int i0 = 0; i0 < S; i0 += blockDim.x) {
-    const int i = i0 + threadIdx.x;
-    const int L = i < S ? clamp_len(__ldg(prm.seq_lens + i), cap) : 0;
-    const int64_t wi = (int64_t)Hkv * unit_work(L, cost, round);
-    int64_t chunk_tot;
-    const int64_t incl = block_inclusive_scan(wi, sh.scan, chunk_tot);
-    const int64_t b = carry + incl - wi;
-    if (wi > 0 && b <= lo && lo < b + wi && lo < hi) {
-      sh.f_i = i;
-      sh.f_base = b;
-    }
-    if (wi > 0 && b <= hi - 1 && hi - 1 < b + wi && lo < hi) {
-      sh.l_i = i;
-      sh.l_base = b;
-    }
-    if (wi > 0 && b <= ws && ws < b + wi) {
-      sh.d_i = i;
-      sh.d_base = b;
+  if (S <= (int)blockDim.x && S <= kInitLens) {
+    // One pass: each thread holds one sequence; a single scan gives both the
+    // total work and every sequence's work offset.
+    const int i = threadIdx.x;
+    const int raw = i < S ? __ldg(prm.seq_lens + i) : 0;
+    const int L = clamp_len(raw, cap);
+    if (i < S) sh.lens[i] = raw;
+    zero_empty_rows<OT>(prm, i, L, G, c);
+    const int64_t wi = i < S ? (int64_t)Hkv * unit_work(L, cost, round) : 0;
+    const int64_t incl = block_inclusive_scan(wi, sh.scan, W);  // syncs: defaults above are set
+    cu = make_cuts(W, G, prm.dyn_ranges, prm.static_share);
+    lo = cu.lo(c);
+    hi = cu.lo(c + 1);
+    ws = cu.Ws;
+    mark_range_seqs(sh, i, incl - wi, wi, lo, hi, ws);
+    if (threadIdx.x == 0) {
+      sh.d_base = W;
+      sh.cuts = cu;
     }
     __syncthreads();
-    const bool have_range = lo >= hi || sh.l_i >= 0;
-    const bool have_dyn = ws >= W || sh.d_i < S;
-    if (have_range && have_dyn) break;
-    carry += chunk_tot;
+    if (sh.d_i == i) sh.d_base = incl - wi;  // d_base defaults to W, written above
+    __syncthreads();
+  } else {
+    // Pass 1: total work; zero rows of empty sequences.
+    int64_t sum = 0;
+    for (int i = threadIdx.x; i < S; i += blockDim.x) {
+      const int L = clamp_len(__ldg(prm.seq_lens + i), cap);
+      sum += (int64_t)Hkv * unit_work(L, cost, round);
+      zero_empty_rows<OT>(prm, i, L, G, c);
+    }
+    block_inclusive_scan(sum, sh.scan, W);
+    cu = make_cuts(W, G, prm.dyn_ranges, prm.static_share);
+    lo = cu.lo(c);
+    hi = cu.lo(c + 1);
+    ws = cu.Ws;
+    // Pass 2: the sequences holding offsets lo, hi - 1 and Ws.
+    if (threadIdx.x == 0) {
+      sh.d_base = W;
+      sh.cuts = cu;
+    }
+    __syncthreads();
+    int64_t carry = 0;
+    for (int i0 = 0; i0 < S; i0 += blockDim.x) {
+      const int i = i0 + threadIdx.x;
+      const int L = i < S ? clamp_len(__ldg(prm.seq_lens + i), cap) : 0;
+      const int64_t wi = (int64_t)Hkv * unit_work(L, cost, round);
+      int64_t chunk_tot;
+      const int64_t incl = block_inclusive_scan(wi, sh.scan, chunk_tot);
+      const int64_t b = carry + incl - wi;
+      mark_range_seqs(sh, i, b, wi, lo, hi, ws);
+      if (wi > 0 && b <= ws && ws < b + wi) sh.d_base = b;
+      __syncthreads();
+      const bool have_range = lo >= hi || sh.l_i >= 0;
+      const bool have_dyn = ws >= W || sh.d_i < S;
+      if (have_range && have_dyn) break;
+      carry += chunk_tot;
+    }
+    __syncthreads();
   }
-  __syncthreads();
   w.seq_lens = prm.seq_lens;
   w.S = S;
   w.Hkv = Hkv;
@@ -370,9 +414,11 @@ __device__ void init_walker(const DecodeParams& prm, SchedShared& sh, SegmentWal
   w.P = prm.part > 0 ? prm.part : kNoSplit;
   w.cuts = cu;
   const int fi = sh.f_i, li = sh.l_i;
-  const int fL = fi >= 0 ? clamp_len(__ldg(prm.seq_lens + fi), cap) : 0;
-  const int fLn = fi >= 0 && fi + 1 < S ? __ldg(prm.seq_lens + fi + 1) : 0;
-  const int lL = li >= 0 ? clamp_len(__ldg(prm.seq_lens + li), cap) : 0;
+  const bool one_pass = S <= (int)blockDim.x && S <= kInitLens;
+  auto raw_len = [&](int i) { return one_pass ? sh.lens[i] : __ldg(prm.seq_lens + i); };
+  const int fL = fi >= 0 ? clamp_len(raw_len(fi), cap) : 0;
+  const int fLn = fi >= 0 && fi + 1 < S ? raw_len(fi + 1) : 0;
+  const int lL = li >= 0 ? clamp_len(raw_len(li), cap) : 0;
   start_range(w, lo, hi, fi, sh.f_base, fL, fLn, li, sh.l_base, lL);
 }
 

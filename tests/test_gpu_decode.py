@@ -64,6 +64,25 @@ def test_group_sizes(cuda_dev, Hq, Hkv, dt):
     _check(cfg, cuda_dev)
 
 
+@pytest.mark.parametrize("S", [150, 192, 193, 256, 257, 600])
+@pytest.mark.parametrize("flags", FLAGS)
+def test_many_sequences(cuda_dev, S, flags):
+    # Batches larger than a CTA (one sequence per thread) take the multi-pass
+    # schedule set-up; zero lengths are mixed in.
+    cfg = C["gqa70b"].replace(num_seqs=S, lens=("uniform", 0, 200), partition_size=64, seed=S)
+    _check(cfg, cuda_dev, flags=flags)
+
+
+@pytest.mark.parametrize("L,P", [(40000, 64), (9000, 32), (3000, 16)])
+@pytest.mark.parametrize("flags", FLAGS)
+def test_unit_split_into_many_pieces(cuda_dev, L, P, flags):
+    # One sequence with one KV head spread over every CTA: the merge of its
+    # partials takes more pieces than a warp has lanes.
+    cfg = C["gqa70b"].replace(num_seqs=1, num_heads=8, num_kv_heads=1, lens=("fixed", [L]),
+                              partition_size=P, seed=5)
+    _check(cfg, cuda_dev, flags=flags)
+
+
 def test_permutation_of_physical_blocks_is_bit_identical(cuda_dev):
     cfg = SMALL["gqa70b"]
     wl = W.make_workload(cfg, device=cuda_dev)
