@@ -70,15 +70,21 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-graph", action="store_true", help="time eager launches")
+    ap.add_argument("--op", default="decode", choices=["decode", "blocks"],
+                    help="blocks: time the block copies (copy-on-write, swap) and the host "
+                         "block manager instead of the decode step (one JSON line each)")
     return ap.parse_args()
 
 
+DECODE_SOURCES = ("common.cuh", "schedule.cuh", "decode_tc.cu", "decode_simt.cu", "pkv_api.cu")
+
+
 def source_sha() -> str:
+    """Hash of the sources the decode kernels and their launch are built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_367_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, name), "rb").read())
+    for name in DECODE_SOURCES:
+        h.update(open(os.path.join(csrc, name), "rb").read())
     h.update(open(os.path.join(ROOT, "include", "pagedkv.h"), "rb").read())
     return h.hexdigest()[:12]
 
@@ -425,6 +431,110 @@ def run_reference(args):
                     "d2h_bytes_per_step": 0}}
 
 
+def _event_time_ms(fn, steps, warmup, flush=None):
+    """Mean device time of fn() over `steps` calls (CUDA events on the current
+    stream), after `warmup` calls; `flush` runs untimed before each call."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    total = 0.0
+    for _ in range(steps):
+        if flush is not None:
+            flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        total += a.elapsed_time(b)
+    return total / steps
+
+
+def run_block_ops(args, dev):
+    """Block copies and the host block manager, each as one JSON line."""
+    from paged_kv_cache_367_b200.blocks import BlockManager
+    peak, peak_src = measured_hbm_peak()
+    steps, warmup = max(args.steps // 50, 10), max(args.warmup, 3)
+    bs, Hkv, D = 16, 8, 128                      # the 70B-class GQA pool: 32 KB per K block
+    nb = 16384                                   # 1 GiB of K+V
+    gen = torch.Generator(device=dev).manual_seed(1)
+    kc = torch.randn((nb, bs, Hkv, D), generator=gen, device=dev).to(torch.bfloat16)
+    vc = torch.randn((nb, bs, Hkv, D), generator=gen, device=dev).to(torch.bfloat16)
+    bb = bs * Hkv * D * 2
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    lines = []
+    for n in (64, 4096):
+        perm = torch.randperm(nb, generator=torch.Generator().manual_seed(n))[:2 * n]
+        pairs = perm.view(n, 2).to(torch.int64).to(dev)
+        ms = _event_time_ms(lambda: pkv.paged_kv_copy_blocks(kc, vc, pairs), steps, warmup,
+                            flush=flush.zero_)
+        byt = 2 * 2 * n * bb                     # K and V, read and write
+        gbs = byt / ms / 1e6
+        lines.append({"metric": "paged_kv_copy_blocks (copy-on-write) HBM GB/s", "value": round(gbs, 1),
+                      "unit": "GB/s", "higher_is_better": True, "us_per_call": round(ms * 1e3, 2),
+                      "dtype": "bf16", "data": "synthetic",
+                      "config": {"workload": f"{n} random block pairs of a [{nb}, {bs}, {Hkv}, {D}] "
+                                             "bf16 pool (K and V)", "l2": "flushed before each call"},
+                      "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
+                                   "peak_source": peak_src, "unit": "GB/s",
+                                   "frac": round(gbs / peak, 4), "traffic": None,
+                                   "bytes": byt}})
+    # Swap: n blocks device -> pinned host and back, against one contiguous copy
+    # of the same bytes through the copy engine.
+    n = 2048
+    hk = torch.empty((n, bs, Hkv, D), dtype=torch.bfloat16).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    src = torch.randperm(nb, generator=torch.Generator().manual_seed(3))[:n].to(torch.int64)
+    out_pairs = torch.stack([src, torch.arange(n)], 1).to(dev)
+    in_pairs = torch.stack([torch.arange(n), src.flip(0)], 1).to(dev)
+    byt = 2 * n * bb
+    ms_out = _event_time_ms(lambda: pkv.paged_kv_swap_blocks(kc, vc, hk, hv, out_pairs), steps,
+                            warmup)
+    ms_in = _event_time_ms(lambda: pkv.paged_kv_swap_blocks(hk, hv, kc, vc, in_pairs), steps,
+                           warmup)
+    big = torch.empty(2 * n * bb, dtype=torch.uint8).pin_memory()
+    dbig = torch.empty(2 * n * bb, dtype=torch.uint8, device=dev)
+    ms_d2h = _event_time_ms(lambda: big.copy_(dbig, non_blocking=True), steps, warmup)
+    ms_h2d = _event_time_ms(lambda: dbig.copy_(big, non_blocking=True), steps, warmup)
+    for name, ms, ref in (("swap-out (device -> pinned host)", ms_out, ms_d2h),
+                          ("swap-in (pinned host -> device)", ms_in, ms_h2d)):
+        gbs, ref_gbs = byt / ms / 1e6, byt / ref / 1e6
+        lines.append({"metric": f"paged_kv_swap_blocks {name} GB/s", "value": round(gbs, 2),
+                      "unit": "GB/s", "higher_is_better": True, "ms_per_call": round(ms, 3),
+                      "dtype": "bf16", "data": "synthetic",
+                      "config": {"workload": f"{n} scattered blocks of 32 KB, K and V "
+                                             f"({byt / 2**20:.0f} MiB)"},
+                      "roofline": {"bound": "host link", "achieved": round(gbs, 2),
+                                   "peak": round(ref_gbs, 2),
+                                   "peak_source": "one contiguous pinned cudaMemcpyAsync of the "
+                                                  "same bytes, measured in this run",
+                                   "unit": "GB/s", "frac": round(gbs / ref_gbs, 4),
+                                   "traffic": None}})
+    # Host block manager: a decode-serving trace of 128 sequences.
+    S, steps_bm = 128, 2000
+    rng = np.random.default_rng(0)
+    bm = BlockManager(S * ((8192 + steps_bm) // 16 + 2), 16, prefix_caching=True)
+    system = list(rng.integers(0, 32000, size=1024))
+    t0 = time.perf_counter()
+    for s in range(S):
+        bm.allocate(s, system + list(rng.integers(0, 32000, size=int(rng.integers(16, 4096)))))
+    t1 = time.perf_counter()
+    toks = rng.integers(0, 32000, size=(steps_bm, S))
+    for k in range(steps_bm):
+        for s in range(S):
+            bm.append_slot(s, int(toks[k, s]))
+    t2 = time.perf_counter()
+    per_step_us = (t2 - t1) / steps_bm * 1e6
+    lines.append({"metric": "host block manager append_slot calls/s", "value":
+                  round(S * steps_bm / (t2 - t1), 0), "unit": "calls/s", "higher_is_better": True,
+                  "us_per_decode_step": round(per_step_us, 2),
+                  "allocate_ms_per_prompt": round((t1 - t0) / S * 1e3, 4),
+                  "config": {"workload": f"{S} sequences with a shared 1024-token prompt "
+                                         "(prefix caching on), 2000 decode steps, through the "
+                                         "Python binding"}, "data": "synthetic"})
+    return lines
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", "0"))
@@ -442,6 +552,11 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=dev)
     try:
+        if args.op == "blocks":
+            if rank == 0:
+                for line in run_block_ops(args, dev):
+                    print(json.dumps(line), flush=True)
+            return
         res = run_ours(args, rank, world, dev)
         if rank == 0:
             print(json.dumps(res), flush=True)

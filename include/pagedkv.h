@@ -58,7 +58,10 @@ typedef enum {
   PKV_ERR_UNSUPPORTED = -4, /* head_dim or block_size outside the supported set */
   PKV_ERR_WORKSPACE = -5,   /* workspace missing or smaller than required */
   PKV_ERR_CUDA = -6,        /* a CUDA runtime call or kernel launch failed */
-  PKV_ERR_ALIGN = -7        /* a pointer is not 16-byte aligned */
+  PKV_ERR_ALIGN = -7,       /* a pointer is not 16-byte aligned */
+  PKV_ERR_NO_BLOCKS = -8,   /* not enough free blocks (block manager) */
+  PKV_ERR_SEQ = -9,         /* unknown, duplicate or swapped-out sequence id */
+  PKV_ERR_MEMORY = -10      /* a pool is neither device memory nor pinned host memory */
 } pkv_status;
 
 /* Flags for paged_attention_decode. */

@@ -15,7 +15,7 @@ import os
 import torch
 
 __all__ = ["paged_kv_append", "paged_attention_decode", "paged_attention_workspace_size",
-           "paged_attention_decode_static",
+           "paged_attention_decode_static", "paged_kv_copy_blocks", "paged_kv_swap_blocks",
            "pkv_device_status", "pkv_status_string", "pkv_version", "load_library", "PagedKVError",
            "PKV_F32", "PKV_F16", "PKV_BF16", "PKV_FP8_E4M3", "PKV_DECODE_FORCE_SIMT",
            "LIB_PATH", "EXPORTED_SYMBOLS"]
@@ -27,7 +27,13 @@ PKV_DECODE_FORCE_SIMT = 1
 
 EXPORTED_SYMBOLS = ("paged_kv_append", "paged_attention_workspace_size",
                     "paged_attention_decode", "paged_attention_decode_static",
-                    "pkv_device_status", "pkv_status_string", "pkv_version")
+                    "pkv_device_status", "pkv_status_string", "pkv_version",
+                    # include/pagedkv_blocks.h
+                    "pkv_bm_create", "pkv_bm_destroy", "pkv_bm_num_free", "pkv_bm_num_free_host",
+                    "pkv_bm_can_allocate", "pkv_bm_allocate", "pkv_bm_can_append",
+                    "pkv_bm_append_slot", "pkv_bm_fork", "pkv_bm_free", "pkv_bm_swap_out",
+                    "pkv_bm_swap_in", "pkv_bm_block_tables", "pkv_bm_seq_len", "pkv_bm_refcount",
+                    "pkv_bm_check", "paged_kv_copy_blocks", "paged_kv_swap_blocks")
 
 _DTYPE_CODES = {torch.float32: PKV_F32, torch.float16: PKV_F16, torch.bfloat16: PKV_BF16,
                 torch.uint8: PKV_FP8_E4M3, torch.float8_e4m3fn: PKV_FP8_E4M3}
@@ -68,6 +74,41 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.paged_attention_decode_static.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I64, I, F,
                                                   I, I, P, P, I, I, U, P]
     lib.paged_attention_decode_static.restype = I
+    # Block manager and block copies (include/pagedkv_blocks.h).
+    lib.pkv_bm_create.argtypes = [I64, I64, I, I]
+    lib.pkv_bm_create.restype = P
+    lib.pkv_bm_destroy.argtypes = [P]
+    lib.pkv_bm_destroy.restype = None
+    for name in ("pkv_bm_num_free", "pkv_bm_num_free_host"):
+        getattr(lib, name).argtypes = [P]
+        getattr(lib, name).restype = I64
+    lib.pkv_bm_can_allocate.argtypes = [P, I64]
+    lib.pkv_bm_can_allocate.restype = I
+    lib.pkv_bm_allocate.argtypes = [P, I64, P, I64, P, P]
+    lib.pkv_bm_allocate.restype = I
+    lib.pkv_bm_can_append.argtypes = [P, I64]
+    lib.pkv_bm_can_append.restype = I
+    lib.pkv_bm_append_slot.argtypes = [P, I64, ctypes.c_int32, P, P, P]
+    lib.pkv_bm_append_slot.restype = I
+    lib.pkv_bm_fork.argtypes = [P, I64, I64]
+    lib.pkv_bm_fork.restype = I
+    lib.pkv_bm_free.argtypes = [P, I64]
+    lib.pkv_bm_free.restype = I
+    for name in ("pkv_bm_swap_out", "pkv_bm_swap_in"):
+        getattr(lib, name).argtypes = [P, P, I, P, I64, P]
+        getattr(lib, name).restype = I
+    lib.pkv_bm_block_tables.argtypes = [P, P, I, I, P, P]
+    lib.pkv_bm_block_tables.restype = I
+    lib.pkv_bm_seq_len.argtypes = [P, I64]
+    lib.pkv_bm_seq_len.restype = I64
+    lib.pkv_bm_refcount.argtypes = [P, ctypes.c_int32]
+    lib.pkv_bm_refcount.restype = I
+    lib.pkv_bm_check.argtypes = [P]
+    lib.pkv_bm_check.restype = I
+    lib.paged_kv_copy_blocks.argtypes = [P, P, P, I, I64, I64, P]
+    lib.paged_kv_copy_blocks.restype = I
+    lib.paged_kv_swap_blocks.argtypes = [P, P, P, P, P, I, I64, I64, I64, P]
+    lib.paged_kv_swap_blocks.restype = I
     _lib = lib
     return lib
 
@@ -167,3 +208,36 @@ def paged_attention_decode_static(out, query, k_cache, v_cache, block_table, seq
                                            int(max_ctas), int(flags), _stream(stream))
     if st != 0:
         raise PagedKVError("paged_attention_decode_static", st)
+
+
+def _block_bytes(pool) -> int:
+    return pool[0].numel() * pool.element_size() if pool.shape[0] else \
+        int(torch.Size(pool.shape[1:]).numel()) * pool.element_size()
+
+
+def paged_kv_copy_blocks(k_cache, v_cache, block_mapping, *, stream=None) -> None:
+    """Copy-on-write copies inside one pool: for each row (src, dst) of
+    block_mapping ([n, 2] int64, device), K[src] -> K[dst] and V[src] -> V[dst];
+    see paged_kv_copy_blocks in include/pagedkv_blocks.h."""
+    lib = load_library()
+    n = block_mapping.shape[0]
+    st = lib.paged_kv_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_mapping), n,
+                                  _block_bytes(k_cache), k_cache.shape[0], _stream(stream))
+    if st != 0:
+        raise PagedKVError("paged_kv_copy_blocks", st)
+
+
+def paged_kv_swap_blocks(src_k, src_v, dst_k, dst_v, block_mapping, *, stream=None) -> None:
+    """Block copies between two pools of the same block shape, either of which
+    may be pinned host memory (swap-out / swap-in); see paged_kv_swap_blocks in
+    include/pagedkv_blocks.h."""
+    lib = load_library()
+    bb = _block_bytes(src_k)
+    if _block_bytes(dst_k) != bb:
+        raise ValueError("source and destination pools have different block shapes")
+    n = block_mapping.shape[0]
+    st = lib.paged_kv_swap_blocks(_ptr(src_k), _ptr(src_v), _ptr(dst_k), _ptr(dst_v),
+                                  _ptr(block_mapping), n, bb, src_k.shape[0], dst_k.shape[0],
+                                  _stream(stream))
+    if st != 0:
+        raise PagedKVError("paged_kv_swap_blocks", st)

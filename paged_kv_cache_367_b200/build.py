@@ -2,8 +2,9 @@
 
     python -m paged_kv_cache_367_b200.build [--force]
 
-Each .cu under csrc/ is compiled to an object under _build/ and linked into
-paged_kv_cache_367_b200/libpagedkv.so. nvcc cross-compiles, so no GPU is needed.
+Each .cu (kernels) and .cpp (host runtime) under csrc/ is compiled by nvcc to an
+object under _build/ and linked into paged_kv_cache_367_b200/libpagedkv.so.
+nvcc cross-compiles, so no GPU is needed.
 """
 from __future__ import annotations
 
@@ -26,7 +27,7 @@ FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2",
 
 
 def sources():
-    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cu"))
+    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cpp")))
 
 
 def _deps_mtime():
@@ -36,7 +37,7 @@ def _deps_mtime():
 
 
 def _compile(src, build_dir, extra):
-    obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
+    obj = os.path.join(build_dir, os.path.splitext(os.path.basename(src))[0] + ".o")
     subprocess.check_call([NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj])
     return obj
 

@@ -1,0 +1,143 @@
+// Whole-block copies: copy-on-write inside one pool and swaps between a device
+// pool and a pinned host pool.
+//
+// "vLLM 推理引擎源码级拆解" (chenxutan.com/d/5333) §2.1: a block shared by
+// several sequences is copied before one of them writes into it (the copy list
+// comes from the block manager's append_slot); §3.2: a preempted request's
+// blocks can be swapped out to host memory and back. Both are the same
+// operation: for each (src, dst) pair, the K block and the V block of src are
+// copied byte for byte to dst. One kernel does all pairs of a call: a pinned
+// host pool is read or written directly through its device-visible address,
+// so a swap of n scattered blocks is one launch rather than 2n memcpy calls.
+#include <cuda_runtime.h>
+
+#include "pagedkv_blocks.h"
+
+namespace pkv {
+namespace {
+
+constexpr int kCopyThreads = 256;
+constexpr int kCopyVecs = 4;                                   // 16-byte vectors per thread
+constexpr int64_t kPiece = (int64_t)kCopyThreads * kCopyVecs * 16;  // bytes per work item
+
+// Work item = (pair, K or V, piece of kPiece bytes). Each thread keeps its
+// kCopyVecs loads in flight before storing.
+__global__ void __launch_bounds__(kCopyThreads)
+    block_copy_kernel(const uint8_t* __restrict__ sk, const uint8_t* __restrict__ sv,
+                      uint8_t* __restrict__ dk, uint8_t* __restrict__ dv,
+                      const int64_t* __restrict__ map, int n, int64_t block_bytes,
+                      int64_t src_blocks, int64_t dst_blocks, int64_t pieces) {
+  const int64_t items = (int64_t)n * 2 * pieces;
+  for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+    const int64_t pair = it / (2 * pieces);
+    const int64_t rem = it - pair * 2 * pieces;
+    const int tensor = (int)(rem / pieces);
+    const int64_t piece = rem - tensor * pieces;
+    const int64_t src = __ldg(map + 2 * pair), dst = __ldg(map + 2 * pair + 1);
+    if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) continue;
+    const int64_t base = piece * kPiece;
+    const int64_t len = min(kPiece, block_bytes - base);
+    const uint8_t* s = (tensor ? sv : sk) + src * block_bytes + base;
+    uint8_t* d = (tensor ? dv : dk) + dst * block_bytes + base;
+    int4 r[kCopyVecs];
+#pragma unroll
+    for (int v = 0; v < kCopyVecs; ++v) {
+      const int64_t off = (int64_t)(v * kCopyThreads + threadIdx.x) * 16;
+      if (off < len) r[v] = __ldcs(reinterpret_cast<const int4*>(s + off));
+    }
+#pragma unroll
+    for (int v = 0; v < kCopyVecs; ++v) {
+      const int64_t off = (int64_t)(v * kCopyThreads + threadIdx.x) * 16;
+      if (off < len) __stcs(reinterpret_cast<int4*>(d + off), r[v]);
+    }
+  }
+}
+
+// A pointer range the kernel may touch from the current device: device memory
+// of this device, managed memory, or pinned host memory mapped at the same
+// address (unified addressing). Both ends of the range are checked.
+int check_range(const void* p, int64_t bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
+  const unsigned char* ends[2] = {static_cast<const unsigned char*>(p),
+                                  static_cast<const unsigned char*>(p) + (bytes - 1)};
+  for (const unsigned char* q : ends) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, q) != cudaSuccess) {
+      cudaGetLastError();
+      return PKV_ERR_MEMORY;
+    }
+    switch (a.type) {
+      case cudaMemoryTypeDevice:
+        if (a.device != dev) return PKV_ERR_MEMORY;
+        break;
+      case cudaMemoryTypeManaged:
+        break;
+      case cudaMemoryTypeHost:
+        if (a.devicePointer != a.hostPointer) return PKV_ERR_MEMORY;
+        break;
+      default:
+        return PKV_ERR_MEMORY;
+    }
+  }
+  return PKV_OK;
+}
+
+int num_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  return sms;
+}
+
+int copy_pairs(const void* sk, const void* sv, void* dk, void* dv, const int64_t* map, int n,
+               int64_t block_bytes, int64_t src_blocks, int64_t dst_blocks, void* stream) {
+  if (n < 0 || block_bytes <= 0 || block_bytes % 16 != 0 || src_blocks < 0 || dst_blocks < 0)
+    return PKV_ERR_SHAPE;
+  if (n == 0) return PKV_OK;
+  if (!sk || !sv || !dk || !dv || !map) return PKV_ERR_NULL;
+  const void* ptrs[4] = {sk, sv, dk, dv};
+  for (const void* q : ptrs)
+    if (reinterpret_cast<uintptr_t>(q) & 15u) return PKV_ERR_ALIGN;
+  if (reinterpret_cast<uintptr_t>(map) & 7u) return PKV_ERR_ALIGN;
+  int st;
+  if (src_blocks > 0) {
+    if ((st = check_range(sk, src_blocks * block_bytes)) != PKV_OK) return st;
+    if ((st = check_range(sv, src_blocks * block_bytes)) != PKV_OK) return st;
+  }
+  if (dst_blocks > 0) {
+    if ((st = check_range(dk, dst_blocks * block_bytes)) != PKV_OK) return st;
+    if ((st = check_range(dv, dst_blocks * block_bytes)) != PKV_OK) return st;
+  }
+  if ((st = check_range(map, (int64_t)n * 16)) != PKV_OK) return st;
+  if (src_blocks == 0 || dst_blocks == 0) return PKV_OK;  // every pair is out of range
+  const int sms = num_sms();
+  if (sms <= 0) return PKV_ERR_CUDA;
+  const int64_t pieces = (block_bytes + kPiece - 1) / kPiece;
+  const int64_t items = (int64_t)n * 2 * pieces;
+  const int64_t cap = (int64_t)sms * (2048 / kCopyThreads);  // one full wave
+  const int grid = (int)(items < cap ? items : cap);
+  block_copy_kernel<<<grid, kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(sk), static_cast<const uint8_t*>(sv),
+      static_cast<uint8_t*>(dk), static_cast<uint8_t*>(dv), map, n, block_bytes, src_blocks,
+      dst_blocks, pieces);
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" int paged_kv_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping,
+                                    int num_pairs, int64_t block_bytes, int64_t num_blocks,
+                                    void* stream) {
+  return pkv::copy_pairs(k_cache, v_cache, k_cache, v_cache, block_mapping, num_pairs,
+                         block_bytes, num_blocks, num_blocks, stream);
+}
+
+extern "C" int paged_kv_swap_blocks(const void* src_k, const void* src_v, void* dst_k,
+                                    void* dst_v, const int64_t* block_mapping, int num_pairs,
+                                    int64_t block_bytes, int64_t src_num_blocks,
+                                    int64_t dst_num_blocks, void* stream) {
+  return pkv::copy_pairs(src_k, src_v, dst_k, dst_v, block_mapping, num_pairs, block_bytes,
+                         src_num_blocks, dst_num_blocks, stream);
+}

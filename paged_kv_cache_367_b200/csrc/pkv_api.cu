@@ -82,6 +82,9 @@ const char* pkv_status_string(int status) {
     case PKV_ERR_WORKSPACE: return "workspace missing or too small";
     case PKV_ERR_CUDA: return "CUDA runtime call or kernel launch failed";
     case PKV_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case PKV_ERR_NO_BLOCKS: return "not enough free blocks";
+    case PKV_ERR_SEQ: return "unknown, duplicate or swapped-out sequence id";
+    case PKV_ERR_MEMORY: return "pool is neither device memory nor pinned host memory";
     default: return "unknown status";
   }
 }

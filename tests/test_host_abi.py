@@ -1,4 +1,4 @@
-"""The C ABI library loads without a GPU, exports every function include/pagedkv.h
+"""The C ABI library loads without a GPU, exports every function include/*.h
 declares, and rejects bad arguments on the host (nothing is enqueued, so these
 run on a machine without a GPU)."""
 import ctypes
@@ -9,7 +9,8 @@ import pytest
 
 from conftest import ROOT
 
-HEADER = os.path.join(ROOT, "include", "pagedkv.h")
+HEADERS = [os.path.join(ROOT, "include", f) for f in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if f.endswith(".h")]
 
 OK, ENULL, ESHAPE, EDTYPE, EUNSUP, EWS, ECUDA, EALIGN = 0, -1, -2, -3, -4, -5, -6, -7
 F32, F16, BF16, FP8 = 0, 1, 2, 3
@@ -25,29 +26,39 @@ def lib():
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_0-9]+)\s*\(",
-                                 text, flags=re.M)))
+    names = set()
+    for h in HEADERS:
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_0-9]+)\s*\(",
+                                text, flags=re.M))
+    return sorted(names)
 
 
 def test_every_declared_function_is_exported(lib):
     names = declared_functions()
     assert {"paged_kv_append", "paged_attention_decode", "paged_attention_workspace_size",
-            "pkv_status_string", "pkv_version"} <= set(names)
+            "pkv_status_string", "pkv_version", "pkv_bm_create", "paged_kv_copy_blocks",
+            "paged_kv_swap_blocks"} <= set(names)
     for n in names:
         assert hasattr(lib, n), n
 
 
 def test_binding_names_match_the_header(lib):
     import paged_kv_cache_367_b200 as pkv
+    from paged_kv_cache_367_b200.blocks import BlockManager
     assert set(pkv.EXPORTED_SYMBOLS) == set(declared_functions())
+    # pkv_bm_<name> is BlockManager.<name> (create / destroy: construction / close).
+    special = {"create": "__init__", "destroy": "close"}
     for n in pkv.EXPORTED_SYMBOLS:
-        assert callable(getattr(pkv, n))
+        if n.startswith("pkv_bm_"):
+            m = n[len("pkv_bm_"):]
+            assert hasattr(BlockManager, special.get(m, m)), n
+        else:
+            assert callable(getattr(pkv, n)), n
 
 
 def test_status_strings(lib):
-    for s in (OK, ENULL, ESHAPE, EDTYPE, EUNSUP, EWS, ECUDA, EALIGN):
+    for s in (OK, ENULL, ESHAPE, EDTYPE, EUNSUP, EWS, ECUDA, EALIGN, -8, -9, -10):
         assert lib.pkv_status_string(s)
     assert lib.pkv_status_string(12345) == b"unknown status"
     assert lib.pkv_version() >= 100
@@ -128,3 +139,35 @@ def test_binding_raises_when_the_library_is_missing(tmp_path):
             pkv.load_library(str(tmp_path / "absent.so"))
     finally:
         pkv._lib = saved
+
+
+def copy(lib, **kw):
+    a = dict(k_cache=A, v_cache=A, block_mapping=A, num_pairs=4, block_bytes=4096,
+             num_blocks=100, stream=None)
+    a.update(kw)
+    return lib.paged_kv_copy_blocks(*a.values())
+
+
+def swap(lib, **kw):
+    a = dict(src_k=A, src_v=A, dst_k=A, dst_v=A, block_mapping=A, num_pairs=4, block_bytes=4096,
+             src_num_blocks=100, dst_num_blocks=10, stream=None)
+    a.update(kw)
+    return lib.paged_kv_swap_blocks(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(num_pairs=0), OK), (dict(num_pairs=0, k_cache=None), OK),
+    (dict(k_cache=None), ENULL), (dict(block_mapping=None), ENULL),
+    (dict(num_pairs=-1), ESHAPE), (dict(block_bytes=0), ESHAPE), (dict(block_bytes=4100), ESHAPE),
+    (dict(num_blocks=-1), ESHAPE), (dict(v_cache=A + 8), EALIGN), (dict(block_mapping=A + 4), EALIGN),
+])
+def test_copy_blocks_rejects_bad_arguments(lib, kw, code):
+    assert copy(lib, **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(num_pairs=0), OK), (dict(dst_k=None), ENULL), (dict(src_v=None), ENULL),
+    (dict(block_bytes=8), ESHAPE), (dict(dst_num_blocks=-2), ESHAPE), (dict(src_k=A + 1), EALIGN),
+])
+def test_swap_blocks_rejects_bad_arguments(lib, kw, code):
+    assert swap(lib, **kw) == code
