@@ -95,6 +95,19 @@ int pkv_bm_can_append(const pkv_block_manager* bm, int64_t seq_id);
 int pkv_bm_append_slot(pkv_block_manager* bm, int64_t seq_id, int32_t token_id, int64_t* slot,
                        int64_t* cow_src, int64_t* cow_dst);
 
+/* One decode step for a batch: append_slot for each of seq_ids[0..n) (distinct,
+ * resident) with token_ids[i], all or nothing.
+ *   slot_mapping  host int64[n] out: each sequence's new slot, ready for
+ *                 paged_kv_append
+ *   cow_pairs     host int64[2 * n] out: the copy-on-write (src, dst) pairs of
+ *                 this step, *num_cow of them, to run with paged_kv_copy_blocks
+ *                 before the append
+ * If the free blocks cannot cover every sequence that needs a new block or a
+ * copy, nothing changes and PKV_ERR_NO_BLOCKS is returned. Errors also
+ * PKV_ERR_SEQ (unknown, swapped-out or repeated id), PKV_ERR_NULL. */
+int pkv_bm_append_slots(pkv_block_manager* bm, const int64_t* seq_ids, const int32_t* token_ids,
+                        int n, int64_t* slot_mapping, int64_t* cow_pairs, int64_t* num_cow);
+
 /* Makes child_id a sequence that shares every block of parent_id (parallel
  * sampling, beam search: §2.1 / "pgsm.cn/news/372185" §2.2). Errors:
  * PKV_ERR_SEQ (parent unknown or swapped out, child in use). */

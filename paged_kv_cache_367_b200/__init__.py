@@ -31,7 +31,7 @@ EXPORTED_SYMBOLS = ("paged_kv_append", "paged_attention_workspace_size",
                     # include/pagedkv_blocks.h
                     "pkv_bm_create", "pkv_bm_destroy", "pkv_bm_num_free", "pkv_bm_num_free_host",
                     "pkv_bm_can_allocate", "pkv_bm_allocate", "pkv_bm_can_append",
-                    "pkv_bm_append_slot", "pkv_bm_fork", "pkv_bm_free", "pkv_bm_swap_out",
+                    "pkv_bm_append_slot", "pkv_bm_append_slots", "pkv_bm_fork", "pkv_bm_free", "pkv_bm_swap_out",
                     "pkv_bm_swap_in", "pkv_bm_block_tables", "pkv_bm_seq_len", "pkv_bm_refcount",
                     "pkv_bm_check", "paged_kv_copy_blocks", "paged_kv_swap_blocks")
 
@@ -90,6 +90,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pkv_bm_can_append.restype = I
     lib.pkv_bm_append_slot.argtypes = [P, I64, ctypes.c_int32, P, P, P]
     lib.pkv_bm_append_slot.restype = I
+    lib.pkv_bm_append_slots.argtypes = [P, P, P, I, P, P, P]
+    lib.pkv_bm_append_slots.restype = I
     lib.pkv_bm_fork.argtypes = [P, I64, I64]
     lib.pkv_bm_fork.restype = I
     lib.pkv_bm_free.argtypes = [P, I64]

@@ -74,6 +74,21 @@ class BlockManager:
             ctypes.byref(dst)))
         return slot.value, src.value, dst.value
 
+    def append_slots(self, seq_ids, token_ids) -> tuple[np.ndarray, np.ndarray]:
+        """One decode step for a batch: (slot_mapping int64 [n], copy-on-write
+        pairs int64 [m, 2] to copy before the append). All or nothing."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        tok = np.ascontiguousarray(token_ids, dtype=np.int32)
+        if len(tok) != len(ids):
+            raise ValueError("seq_ids and token_ids differ in length")
+        slots = np.empty(len(ids), dtype=np.int64)
+        cow = np.empty((max(len(ids), 1), 2), dtype=np.int64)
+        m = ctypes.c_int64(0)
+        _check("pkv_bm_append_slots", self._lib.pkv_bm_append_slots(
+            self._h, ids.ctypes.data, tok.ctypes.data, len(ids), slots.ctypes.data,
+            cow.ctypes.data, ctypes.byref(m)))
+        return slots, cow[:m.value].copy()
+
     def fork(self, parent_id: int, child_id: int) -> None:
         _check("pkv_bm_fork", self._lib.pkv_bm_fork(self._h, parent_id, child_id))
 

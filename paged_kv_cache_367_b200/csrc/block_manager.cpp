@@ -311,6 +311,41 @@ int pkv_bm_append_slot(pkv_block_manager* bm, int64_t seq_id, int32_t token_id, 
   return PKV_OK;
 }
 
+int pkv_bm_append_slots(pkv_block_manager* bm, const int64_t* seq_ids, const int32_t* token_ids,
+                        int n, int64_t* slot_mapping, int64_t* cow_pairs, int64_t* num_cow) {
+  if (!bm || !num_cow) return PKV_ERR_NULL;
+  if (n < 0) return PKV_ERR_SHAPE;
+  if (n > 0 && (!seq_ids || !token_ids || !slot_mapping || !cow_pairs)) return PKV_ERR_NULL;
+  // Check everything first: known, resident, distinct; count the blocks needed.
+  std::vector<Seq*> seqs((size_t)n);
+  std::unordered_set<int64_t> seen;
+  int64_t need = 0;
+  for (int i = 0; i < n; ++i) {
+    auto it = bm->seqs.find(seq_ids[i]);
+    if (it == bm->seqs.end() || it->second.swapped || !seen.insert(seq_ids[i]).second)
+      return PKV_ERR_SEQ;
+    Seq& sq = it->second;
+    seqs[(size_t)i] = &sq;
+    if (sq.len % bm->bs == 0 || bm->dev[sq.blocks.back()].ref > 1) ++need;
+  }
+  // A shared partial block copied by one sequence of the batch may leave the
+  // last sharer writing in place, so `need` is an upper bound.
+  if (need > bm->available()) return PKV_ERR_NO_BLOCKS;
+  int64_t ncow = 0;
+  for (int i = 0; i < n; ++i) {
+    int64_t src, dst;
+    const int st = pkv_bm_append_slot(bm, seq_ids[i], token_ids[i], slot_mapping + i, &src, &dst);
+    if (st != PKV_OK) return st;  // unreachable: checked above
+    if (src >= 0) {
+      cow_pairs[2 * ncow] = src;
+      cow_pairs[2 * ncow + 1] = dst;
+      ++ncow;
+    }
+  }
+  *num_cow = ncow;
+  return PKV_OK;
+}
+
 int pkv_bm_fork(pkv_block_manager* bm, int64_t parent_id, int64_t child_id) {
   if (!bm) return PKV_ERR_NULL;
   auto it = bm->seqs.find(parent_id);

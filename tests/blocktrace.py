@@ -120,6 +120,28 @@ class Trace:
         self.pools.write([slot], [k], [v])
         self.model.append(sid, tok, k, v)
 
+    def decode_step(self):
+        """One batched decode step: every resident sequence gets a token."""
+        res = self.resident()
+        if not res:
+            return
+        toks = [int(t) for t in self.rng.integers(0, self.vocab, size=len(res))]
+        try:
+            slots, cow = self.bm.append_slots(res, toks)
+        except Exception:
+            self.stats["no_blocks"] += 1
+            return
+        if len(cow):
+            self.stats["cow"] += len(cow)
+            self.pools.copy(cow)
+        ks, vs = [], []
+        for sid, tok in zip(res, toks):
+            k, v = self.row(self.model.tokens[sid] + [tok])
+            self.model.append(sid, tok, k, v)
+            ks.append(k)
+            vs.append(v)
+        self.pools.write(slots, ks, vs)
+
     def fork(self):
         res = self.resident()
         if not res:
@@ -170,7 +192,7 @@ class Trace:
         self.swapped -= set(int(g) for g in group)
 
     def step(self, swaps=True):
-        ops = [self.admit, self.append, self.append, self.append, self.fork, self.free]
+        ops = [self.admit, self.append, self.append, self.decode_step, self.fork, self.free]
         if swaps:
             ops += [self.swap_out, self.swap_in]
         ops[self.rng.integers(len(ops))]()

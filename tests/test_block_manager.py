@@ -219,5 +219,45 @@ def test_random_traces_preserve_every_sequence(prefix, seed):
         assert st["cached"] > 0
 
 
+def test_batched_step_equals_one_call_per_sequence():
+    rng = np.random.default_rng(3)
+    a, b = BlockManager(64, 4, prefix_caching=True), BlockManager(64, 4, prefix_caching=True)
+    for bm in (a, b):
+        bm.allocate(1, [1, 2, 3, 4, 5, 6])
+        bm.allocate(2, [1, 2, 3, 4, 5, 6])          # shares the first block
+        bm.fork(1, 3)                                # shares both blocks of 1
+        bm.allocate(4, [])
+    for _ in range(9):
+        ids = [3, 1, 4, 2]
+        toks = rng.integers(0, 9, size=4)
+        slots, cow = a.append_slots(ids, toks)
+        want = [b.append_slot(i, int(t)) for i, t in zip(ids, toks)]
+        assert list(slots) == [w[0] for w in want]
+        assert cow.tolist() == [[w[1], w[2]] for w in want if w[1] >= 0]
+    for bm in (a, b):
+        bm.check()
+    ta, _ = a.block_tables([1, 2, 3, 4], 5)
+    tb, _ = b.block_tables([1, 2, 3, 4], 5)
+    assert np.array_equal(ta, tb)
+
+
+def test_batched_step_is_all_or_nothing():
+    bm = BlockManager(3, 4)
+    bm.allocate(1, [0] * 4)                          # full: the next token needs a block
+    bm.allocate(2, [0] * 4)
+    bm.allocate(3, [0] * 2)                          # partial: writes in place
+    with pytest.raises(PagedKVError) as e:
+        bm.append_slots([1, 2, 3], [0, 0, 0])        # 2 blocks needed, 0 free
+    assert status(e) == ENO_BLOCKS
+    assert [bm.seq_len(i) for i in (1, 2, 3)] == [4, 4, 2]
+    slots, cow = bm.append_slots([3], [5])
+    assert len(cow) == 0 and bm.seq_len(3) == 3
+    for ids in ([3, 3], [9], [1, 9]):
+        with pytest.raises(PagedKVError) as e:
+            bm.append_slots(ids, [0] * len(ids))
+        assert status(e) == ESEQ
+    bm.check()
+
+
 def test_model_blocks_needed_closed_form():
     assert [M.blocks_needed(n, 16) for n in (0, 1, 16, 17, 48, 200)] == [0, 1, 1, 2, 3, 13]
