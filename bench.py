@@ -70,9 +70,10 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-graph", action="store_true", help="time eager launches")
-    ap.add_argument("--op", default="decode", choices=["decode", "blocks"],
+    ap.add_argument("--op", default="decode", choices=["decode", "blocks", "blocksize"],
                     help="blocks: time the block copies (copy-on-write, swap) and the host "
-                         "block manager instead of the decode step (one JSON line each)")
+                         "block manager; blocksize: decode time and pool fragmentation for "
+                         "block sizes 8/16/32 (one JSON line each) instead of the decode step")
     return ap.parse_args()
 
 
@@ -542,6 +543,63 @@ def run_block_ops(args, dev):
     return lines
 
 
+def run_block_sizes(args, dev):
+    """Decode time of the workload at block sizes 8, 16 and 32 (same lengths),
+    and the pool fragmentation of its lengths and of a short-request mix under
+    fixed blocks, the dynamic page-size policy and whole-length reservation."""
+    from paged_kv_cache_367_b200 import fragmentation as FR
+    peak, peak_src = measured_hbm_peak()
+    base = W.CONFIGS[args.workload]
+    lines = []
+    reps, warmup = max(args.steps // 20, 20), max(args.warmup, 3)
+    for bs in (8, 16, 32):
+        wl = W.make_workload(base.replace(block_size=bs), device=dev)
+        c = wl.cfg
+        P = c.partition_size
+        bt = torch.from_numpy(wl.block_table).to(dev)
+        sl = torch.from_numpy(wl.seq_lens).to(dev)
+        nbytes = pkv.paged_attention_workspace_size(c.num_seqs, c.num_heads, c.num_kv_heads,
+                                                    c.head_dim, wl.max_seq_len, P)
+        ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+        out = torch.empty_like(wl.query)
+        ks = vs = None
+        if c.cache_dtype == "e4m3":
+            ks = torch.tensor([wl.k_scale], device=dev)
+            vs = torch.tensor([wl.v_scale], device=dev)
+
+        def call():
+            pkv.paged_attention_decode(out, wl.query, wl.k_cache, wl.v_cache, bt, sl,
+                                       max_seq_len=wl.max_seq_len, scale=c.scale,
+                                       partition_size=P, workspace=ws, k_scale=ks, v_scale=vs)
+        ms = _event_time_ms(call, reps, warmup)
+        dec, _ = step_bytes(wl)
+        gbs = dec / ms / 1e6
+        lines.append({"metric": "paged decode attention HBM GB/s by block size", "value": round(gbs, 1),
+                      "unit": "GB/s", "higher_is_better": True, "block_size": bs,
+                      "us_per_launch": round(ms * 1e3, 2), "dtype": c.q_dtype,
+                      "data": "synthetic", "config": {"workload": WORKLOAD_TEXT.get(
+                          args.workload, args.workload).replace("block 16", f"block {bs}")},
+                      "fragmentation": round(FR.fixed_block_fragmentation(wl.seq_lens, bs), 5),
+                      "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
+                                   "peak_source": peak_src, "unit": "GB/s",
+                                   "frac": round(gbs / peak, 4), "traffic": None}})
+        del wl, out, ws
+        torch.cuda.empty_cache()
+    lens = W.draw_seq_lens(base, np.random.default_rng(base.seed))
+    short = np.random.default_rng(7).integers(16, 161, size=128)
+    for name, L in ((args.workload + " lengths", lens), ("128 short requests U[16, 160]", short)):
+        lines.append({"metric": "KV pool fragmentation (allocated - used) / allocated",
+                      "unit": "fraction", "higher_is_better": False, "lengths": name,
+                      "value": round(FR.fixed_block_fragmentation(L, 16), 5),
+                      "fixed": {str(b): round(FR.fixed_block_fragmentation(L, b), 5)
+                                for b in (8, 16, 32)},
+                      "dynamic_page_size": round(FR.dynamic_fragmentation(L), 5),
+                      "reservation_to_max_len": round(
+                          FR.reservation_fragmentation(L, int(max(L))), 5),
+                      "data": "synthetic"})
+    return lines
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", "0"))
@@ -559,9 +617,10 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=dev)
     try:
-        if args.op == "blocks":
+        if args.op in ("blocks", "blocksize"):
             if rank == 0:
-                for line in run_block_ops(args, dev):
+                fn = run_block_ops if args.op == "blocks" else run_block_sizes
+                for line in fn(args, dev):
                     print(json.dumps(line), flush=True)
             return
         res = run_ours(args, rank, world, dev)

@@ -55,6 +55,12 @@ def test_fp8_prefix_block_sizes(cuda_dev, bs):
     _check(SMALL["fp8_prefix"].replace(block_size=bs), cuda_dev)
 
 
+@pytest.mark.parametrize("bs", [8, 32])
+@pytest.mark.parametrize("flags", FLAGS)
+def test_bf16_block_sizes(cuda_dev, bs, flags):
+    _check(SMALL["gqa70b"].replace(block_size=bs), cuda_dev, flags=flags)
+
+
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 4), (24, 2), (16, 1), (32, 2)])
 @pytest.mark.parametrize("dt", ["bf16", "f16"])
 def test_group_sizes(cuda_dev, Hq, Hkv, dt):
