@@ -10,7 +10,8 @@ Pages followed (title, address, section):
     append into the last block, §2.3 PagedAttention kernel (per-token block-table
     walk, dot(q, k) * scale, softmax, write back; GQA/MQA).
   * "vLLM 深度实战" (chenxutan.com/d/3332) §1.2 Block / Block Table.
-  * "vLLM 0.5 深度拆解" (chenxutan.com/d/4924) §4.2 FP8 KV cache.
+  * "vLLM 0.5 深度拆解" (chenxutan.com/d/4924) §4.2 FP8 KV cache, §2.3 chunked
+    prefill (multi-token queries over the paged cache, causal).
 
 Storage conventions of the arrays passed in (raw element storage, C order):
   f32 -> numpy float32, f16 -> numpy float16, bf16 -> numpy uint16 bit
@@ -72,6 +73,9 @@ def _load():
         lib.orc_decode_items.restype = I
         lib.orc_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I64, D, I, I, D, D, I]
         lib.orc_decode.restype = I
+        lib.orc_prefill_items.argtypes = [P, P, I64, P, P, P, P, P, P, I, I, I, I, I, I, I64,
+                                          D, I, I, D, D, I]
+        lib.orc_prefill_items.restype = I
         _lib = lib
     return _lib
 
@@ -160,3 +164,39 @@ def decode(query, k_cache, v_cache, block_table, seq_lens, *, num_heads, num_kv_
     if used < 0:
         raise ValueError("oracle decode: num_heads must be a multiple of num_kv_heads")
     return out, used
+
+
+def prefill(query, k_cache, v_cache, block_table, seq_lens, query_start, *, num_heads,
+            num_kv_heads, head_dim, block_size, scale, q_dtype, cache_dtype, k_scale=1.0,
+            v_scale=1.0, items=None, threads=0, num_blocks=None):
+    """fp64 causal attention of multi-token queries over the paged cache.
+
+    query is [num_q_tokens, num_heads, head_dim]; rows query_start[i] ..
+    query_start[i+1]-1 are the last tokens of sequence i (whose seq_lens[i]
+    cached tokens include them), and each attends over the tokens up to its own
+    position. Returns (out, threads_used): out is [num_q_tokens, num_heads,
+    head_dim], or [n, head_dim] for `items` (an [n, 2] array of (row, query head)).
+    """
+    block_table = np.ascontiguousarray(block_table, dtype=np.int32)
+    seq_lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    query_start = np.ascontiguousarray(query_start, dtype=np.int32)
+    scale, k_scale, v_scale = (float(np.float32(x)) for x in (scale, k_scale, v_scale))
+    S, mbps = block_table.shape
+    T = int(query_start[-1])
+    nb = num_blocks if num_blocks is not None else k_cache.shape[0]
+    if items is None:
+        items = np.stack(np.meshgrid(np.arange(T), np.arange(num_heads), indexing="ij"),
+                         -1).reshape(-1, 2)
+        shape = (T, num_heads, head_dim)
+    else:
+        shape = (len(items), head_dim)
+    items = np.ascontiguousarray(items, dtype=np.int32).reshape(-1, 2)
+    out = np.empty((len(items), head_dim), dtype=np.float64)
+    used = _load().orc_prefill_items(
+        _ptr(out), _ptr(items), len(items), _ptr(query), _ptr(k_cache), _ptr(v_cache),
+        _ptr(block_table), _ptr(seq_lens), _ptr(query_start), S, num_heads, num_kv_heads,
+        head_dim, block_size, mbps, nb, float(scale), DTYPE_CODES[q_dtype],
+        DTYPE_CODES[cache_dtype], float(k_scale), float(v_scale), int(threads))
+    if used < 0:
+        raise ValueError("oracle prefill: num_heads must be a multiple of num_kv_heads")
+    return out.reshape(shape), used

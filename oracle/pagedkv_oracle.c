@@ -189,21 +189,19 @@ typedef struct {
 } orc_problem;
 
 /*
- * Attention of query head j of sequence i over that sequence's cached tokens:
- *   K[t] = cache element at (block_table[i][t / bs], t % bs, kv head, :)
+ * Attention of one query row (query element offset qoff, KV head h) over the
+ * first L cached tokens of sequence i:
+ *   K[t] = cache element at (block_table[i][t / bs], t % bs, h, :)
  *   s_t  = scale * <q, K[t]>
  *   out  = sum_t exp(s_t - max s) V[t] / sum_t exp(s_t - max s)
- * out_row receives head_dim doubles; sbuf holds seq_len doubles.
+ * out_row receives head_dim doubles (zeros if L <= 0); sbuf holds L doubles.
  */
-static void orc_decode_item(const orc_problem* p, int i, int j, double* out_row, double* sbuf) {
+static void orc_attend_row(const orc_problem* p, int64_t qoff, int i, int h, int64_t L,
+                           double* out_row, double* sbuf) {
   int D = p->head_dim;
-  int g = p->num_heads / p->num_kv_heads;
-  int h = j / g;
-  int64_t L = p->seq_lens[i];
   for (int d = 0; d < D; ++d) out_row[d] = 0.0;
   if (L <= 0) return;
   const int32_t* bt = p->block_table + (int64_t)i * p->max_blocks_per_seq;
-  int64_t qoff = ((int64_t)i * p->num_heads + j) * D;
   int is8 = p->cache_dtype == ORC_E4M3;
   double ks = is8 ? p->k_scale : 1.0, vs = is8 ? p->v_scale : 1.0;
 
@@ -229,6 +227,13 @@ static void orc_decode_item(const orc_problem* p, int i, int j, double* out_row,
       out_row[d] += w * (orc_load(p->v_cache, base + d, p->cache_dtype) * vs);
   }
   for (int d = 0; d < D; ++d) out_row[d] /= denom;
+}
+
+/* Decode: query head j of sequence i (query row i) over all L_i cached tokens. */
+static void orc_decode_item(const orc_problem* p, int i, int j, double* out_row, double* sbuf) {
+  int g = p->num_heads / p->num_kv_heads;
+  int64_t qoff = ((int64_t)i * p->num_heads + j) * p->head_dim;
+  orc_attend_row(p, qoff, i, j / g, p->seq_lens[i], out_row, sbuf);
 }
 
 /*
@@ -287,6 +292,64 @@ int orc_decode(double* out, const void* query, const void* k_cache, const void* 
 }
 
 /* ---- array helpers for the Python wrapper ----------------------------- */
+
+/* ---- multi-token queries: chunked prefill / prefix-cache continuation ---- */
+
+/*
+ * Query rows query_start[i] .. query_start[i+1]-1 belong to sequence i, whose
+ * seq_lens[i] cached tokens include them as its last q_i = query_start[i+1] -
+ * query_start[i] tokens ("vLLM 0.5 深度拆解" §2.3 chunked prefill: a long prompt
+ * is filled in chunks, each chunk's tokens attending over everything before
+ * them; "vLLM 推理引擎源码级拆解" §4.2: a request whose prefix blocks are cached
+ * computes only the rest). Row r of sequence i sits at position
+ *   pos = seq_lens[i] - q_i + (r - query_start[i])
+ * and attends causally over tokens 0..pos. items holds (row, query head)
+ * pairs; out receives num_items*head_dim doubles in item order. Returns the
+ * threads used, or -1 for a bad head ratio.
+ */
+int orc_prefill_items(double* out, const int32_t* items, int64_t num_items,
+                      const void* query, const void* k_cache, const void* v_cache,
+                      const int32_t* block_table, const int32_t* seq_lens,
+                      const int32_t* query_start, int num_seqs, int num_heads, int num_kv_heads,
+                      int head_dim, int block_size, int max_blocks_per_seq, int64_t num_blocks,
+                      double scale, int q_dtype, int cache_dtype, double k_scale,
+                      double v_scale, int num_threads) {
+  if (num_kv_heads <= 0 || num_heads % num_kv_heads) return -1;
+  orc_problem p = {query, k_cache, v_cache, block_table, seq_lens, num_heads, num_kv_heads,
+                   head_dim, block_size, max_blocks_per_seq, num_blocks, scale, k_scale,
+                   v_scale, q_dtype, cache_dtype};
+  int g = num_heads / num_kv_heads;
+  int64_t max_len = 1;
+  for (int i = 0; i < num_seqs; ++i)
+    if (seq_lens[i] > max_len) max_len = seq_lens[i];
+  int used = 1;
+#ifdef _OPENMP
+  if (num_threads <= 0) num_threads = omp_get_max_threads();
+  used = num_threads;
+#pragma omp parallel num_threads(num_threads)
+#endif
+  {
+    double* sbuf = (double*)malloc(sizeof(double) * max_len);
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+    for (int64_t n = 0; n < num_items; ++n) {
+      int r = items[2 * n], j = items[2 * n + 1];
+      int i = 0;
+      while (i < num_seqs && !(query_start[i] <= r && r < query_start[i + 1])) ++i;
+      double* row = out + n * head_dim;
+      if (i == num_seqs) {
+        for (int d = 0; d < head_dim; ++d) row[d] = 0.0;
+        continue;
+      }
+      int64_t q_i = query_start[i + 1] - query_start[i];
+      int64_t pos = (int64_t)seq_lens[i] - q_i + (r - query_start[i]);
+      orc_attend_row(&p, ((int64_t)r * num_heads + j) * head_dim, i, j / g, pos + 1, row, sbuf);
+    }
+    free(sbuf);
+  }
+  return used;
+}
 
 void orc_e4m3_encode_array(const float* x, uint8_t* out, int64_t n) {
   for (int64_t k = 0; k < n; ++k) out[k] = orc_e4m3_encode(x[k]);
