@@ -70,10 +70,11 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-graph", action="store_true", help="time eager launches")
-    ap.add_argument("--op", default="decode", choices=["decode", "blocks", "blocksize"],
+    ap.add_argument("--op", default="decode", choices=["decode", "blocks", "blocksize", "prefill"],
                     help="blocks: time the block copies (copy-on-write, swap) and the host "
                          "block manager; blocksize: decode time and pool fragmentation for "
-                         "block sizes 8/16/32 (one JSON line each) instead of the decode step")
+                         "block sizes 8/16/32; prefill: causal multi-token queries over the "
+                         "paged cache (one JSON line each) instead of the decode step")
     return ap.parse_args()
 
 
@@ -600,6 +601,67 @@ def run_block_sizes(args, dev):
     return lines
 
 
+def measured_bf16_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured burst (MEASURED_PEAKS.json bf16_tflops)"
+    except Exception:
+        return 1590.0, "fallback 1.59 PFLOP/s"
+
+
+def run_prefill(args, dev):
+    """Causal multi-token queries over the paged cache: a chunked-prefill step
+    (chunks of 1024 tokens continuing cached contexts) and full prefills, in the
+    70B-class GQA shape. TFLOP/s counts 4 * head_dim flops per (query head, row,
+    attended token): the two contractions of the causal range, nothing masked."""
+    peak, peak_src = measured_bf16_peak()
+    Hq, Hkv, D, bs = 64, 8, 128, 16
+    lines = []
+    reps, warmup = max(args.steps // 20, 20), max(args.warmup, 3)
+    for name, ctx, qlen in (("chunked prefill: 8 sequences, 1024-token chunks after 2048 "
+                             "cached tokens", [3072] * 8, [1024] * 8),
+                            ("full prefill: 4 prompts of 4096 tokens", [4096] * 4, [4096] * 4),
+                            ("full prefill: 16 prompts of 512 tokens", [512] * 16, [512] * 16)):
+        S = len(ctx)
+        nbs = [-(-L // bs) for L in ctx]
+        nb = sum(nbs)
+        g = torch.Generator(device=dev).manual_seed(5)
+        kc = torch.randn((nb, bs, Hkv, D), generator=g, device=dev).to(torch.bfloat16)
+        vc = torch.randn((nb, bs, Hkv, D), generator=g, device=dev).to(torch.bfloat16)
+        perm = torch.randperm(nb, generator=torch.Generator().manual_seed(6)).to(torch.int32)
+        bt = torch.full((S, max(nbs)), -1, dtype=torch.int32)
+        o = 0
+        for i, k in enumerate(nbs):
+            bt[i, :k] = perm[o:o + k]
+            o += k
+        qs = torch.tensor(np.concatenate([[0], np.cumsum(qlen)]), dtype=torch.int32)
+        T = int(qs[-1])
+        q = torch.randn((T, Hq, D), generator=g, device=dev).to(torch.bfloat16)
+        out = torch.empty_like(q)
+        btd, lensd, qsd = bt.to(dev), torch.tensor(ctx, dtype=torch.int32, device=dev), qs.to(dev)
+
+        def call():
+            pkv.paged_attention_prefill(out, q, kc, vc, btd, lensd, qsd, max_q_len=max(qlen),
+                                        scale=D ** -0.5)
+        ms = _event_time_ms(call, reps, warmup)
+        attended = sum(sum(L - n + r + 1 for r in range(n)) for L, n in zip(ctx, qlen))
+        flops = 4.0 * D * Hq * attended
+        tflops = flops / ms / 1e9
+        lines.append({"metric": "paged causal multi-token attention TFLOP/s", "value": round(tflops, 1),
+                      "unit": "TFLOP/s", "higher_is_better": True, "us_per_launch": round(ms * 1e3, 1),
+                      "tokens_per_s": round(T / ms * 1e3, 0), "dtype": "bf16", "data": "synthetic",
+                      "config": {"workload": name + f"; {Hq} q / {Hkv} KV heads, head_dim {D}, "
+                                                    f"block {bs}, shuffled pool"},
+                      "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak,
+                                   "peak_source": peak_src, "unit": "TFLOP/s",
+                                   "frac": round(tflops / peak, 4), "traffic": None,
+                                   "flops": flops,
+                                   "kernel": "mma.sync m16n8k16 (legacy tensor path)"}})
+        del kc, vc, q, out
+        torch.cuda.empty_cache()
+    return lines
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", "0"))
@@ -617,9 +679,10 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=dev)
     try:
-        if args.op in ("blocks", "blocksize"):
+        if args.op in ("blocks", "blocksize", "prefill"):
             if rank == 0:
-                fn = run_block_ops if args.op == "blocks" else run_block_sizes
+                fn = {"blocks": run_block_ops, "blocksize": run_block_sizes,
+                      "prefill": run_prefill}[args.op]
                 for line in fn(args, dev):
                     print(json.dumps(line), flush=True)
             return

@@ -188,6 +188,42 @@ int paged_attention_decode_static(void* out, const void* query, const void* k_ca
                                   int max_ctas, unsigned flags, void* stream);
 
 /*
+ * paged_attention_prefill — multi-token queries over the paged cache, causal.
+ *
+ * "vLLM 0.5 深度拆解" (chenxutan.com/d/4924) §2.3: a long prompt is filled in
+ * chunks, each chunk's tokens attending over everything before them and over
+ * the chunk itself; "vLLM 推理引擎源码级拆解" (chenxutan.com/d/5333) §4.2: a
+ * request whose leading blocks are cached computes only the rest. Both are:
+ *
+ *   query        [num_q_tokens, num_heads, head_dim], q_dtype (BF16/F16)
+ *   query_start  [num_seqs + 1] int32, device: rows query_start[i] ..
+ *                query_start[i+1]-1 are the last q_i tokens of sequence i
+ *   seq_lens     [num_seqs] int32, device: sequence i's cached tokens, the q_i
+ *                chunk tokens included (their K/V appended beforehand with
+ *                paged_kv_append)
+ *   k_cache,
+ *   v_cache      the pool, cache_dtype == q_dtype
+ *   out          [num_q_tokens, num_heads, head_dim], q_dtype
+ *
+ * Row r of sequence i sits at position p = seq_lens[i] - q_i + (r -
+ * query_start[i]) and gets softmax(scale * q . K[t]) over t = 0..p applied to V
+ * (GQA: query head j reads KV head j / (num_heads / num_kv_heads)); a row with
+ * p < 0 gets zeros. max_q_len must be >= every q_i: a longer chunk has only its
+ * last max_q_len rows computed. Lengths are clamped to max_blocks_per_seq *
+ * block_size and query_start to [0, num_q_tokens]. head_dim 64 or 128,
+ * block_size 8/16/32; FP8 caches are not supported here (PKV_ERR_DTYPE).
+ * Errors: PKV_ERR_SHAPE, PKV_ERR_UNSUPPORTED, PKV_ERR_DTYPE, PKV_ERR_NULL,
+ * PKV_ERR_ALIGN, PKV_ERR_CUDA.
+ */
+int paged_attention_prefill(void* out, const void* query, const void* k_cache,
+                            const void* v_cache, const int32_t* block_table,
+                            const int32_t* seq_lens, const int32_t* query_start, int num_seqs,
+                            int num_q_tokens, int max_q_len, int num_heads, int num_kv_heads,
+                            int head_dim, int block_size, int max_blocks_per_seq,
+                            int64_t num_blocks, float scale, int q_dtype, int cache_dtype,
+                            void* stream);
+
+/*
  * Health word of the device kernels. Every wait inside a kernel is bounded
  * (about one second); a wait that expires makes its CTA skip the rest of its
  * work and sets this word, so a wrong result is reported instead of a hung GPU.

@@ -16,6 +16,7 @@ import torch
 
 __all__ = ["paged_kv_append", "paged_attention_decode", "paged_attention_workspace_size",
            "paged_attention_decode_static", "paged_kv_copy_blocks", "paged_kv_swap_blocks",
+           "paged_attention_prefill",
            "pkv_device_status", "pkv_status_string", "pkv_version", "load_library", "PagedKVError",
            "PKV_F32", "PKV_F16", "PKV_BF16", "PKV_FP8_E4M3", "PKV_DECODE_FORCE_SIMT",
            "LIB_PATH", "EXPORTED_SYMBOLS"]
@@ -27,7 +28,7 @@ PKV_DECODE_FORCE_SIMT = 1
 
 EXPORTED_SYMBOLS = ("paged_kv_append", "paged_attention_workspace_size",
                     "paged_attention_decode", "paged_attention_decode_static",
-                    "pkv_device_status", "pkv_status_string", "pkv_version",
+                    "paged_attention_prefill", "pkv_device_status", "pkv_status_string", "pkv_version",
                     # include/pagedkv_blocks.h
                     "pkv_bm_create", "pkv_bm_destroy", "pkv_bm_num_free", "pkv_bm_num_free_host",
                     "pkv_bm_can_allocate", "pkv_bm_allocate", "pkv_bm_can_append",
@@ -74,6 +75,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.paged_attention_decode_static.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I64, I, F,
                                                   I, I, P, P, I, I, U, P]
     lib.paged_attention_decode_static.restype = I
+    lib.paged_attention_prefill.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I64, F,
+                                            I, I, P]
+    lib.paged_attention_prefill.restype = I
     # Block manager and block copies (include/pagedkv_blocks.h).
     lib.pkv_bm_create.argtypes = [I64, I64, I, I]
     lib.pkv_bm_create.restype = P
@@ -210,6 +214,24 @@ def paged_attention_decode_static(out, query, k_cache, v_cache, block_table, seq
                                            int(max_ctas), int(flags), _stream(stream))
     if st != 0:
         raise PagedKVError("paged_attention_decode_static", st)
+
+
+def paged_attention_prefill(out, query, k_cache, v_cache, block_table, seq_lens, query_start, *,
+                            max_q_len, scale, stream=None) -> None:
+    """Causal attention of multi-token queries (chunked prefill, the uncached
+    rest of a prefix-cache hit) over the paged cache; see
+    paged_attention_prefill in include/pagedkv.h."""
+    lib = load_library()
+    T, Hq, D = query.shape
+    nb, bs, Hkv, _ = k_cache.shape
+    S = seq_lens.shape[0]
+    st = lib.paged_attention_prefill(_ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache),
+                                     _ptr(block_table), _ptr(seq_lens), _ptr(query_start), S, T,
+                                     int(max_q_len), Hq, Hkv, D, bs, block_table.shape[1], nb,
+                                     float(scale), _dtype_code(query), _dtype_code(k_cache),
+                                     _stream(stream))
+    if st != 0:
+        raise PagedKVError("paged_attention_prefill", st)
 
 
 def _block_bytes(pool) -> int:

@@ -38,8 +38,11 @@
 #include <cudaTypedefs.h>
 
 #include "schedule.cuh"
+#include "tc_common.cuh"
 
 namespace pkv {
+
+using namespace tcx;
 
 __device__ int g_tc_timeout = 0;
 
@@ -50,7 +53,6 @@ constexpr int kConsumerWarps = 4;                    // 16 tokens of a chunk eac
 constexpr int kProducerWarp = kConsumerWarps;        // TMA issue
 constexpr int kEpilogueWarp = kConsumerWarps + 1;    // combine, store, merge
 constexpr int kThreads = (kConsumerWarps + 2) * 32;
-constexpr long long kWaitCycles = 1ll << 31;         // ~1 s at 2 GHz
 
 template <int D, int NT, int NS, int EKV>
 struct Cfg {
@@ -66,138 +68,10 @@ struct Cfg {
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA exceeds 227 KB");
 };
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait for the phase of `bar` with the given parity. Returns false if
-// the CTA is aborting or the wait expired (which starts the abort).
+// Bounded wait that reports expiry in this kernel's error word.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  if (*abort) return false;
-  const long long t0 = clock64();
-  for (int it = 1;; ++it) {
-    if (mbar_try(bar, parity)) return true;
-    if ((it & 31) == 0) {
-      if (*abort) return false;
-      if (clock64() - t0 > kWaitCycles) {
-        *abort = 1;
-        atomicExch(&g_tc_timeout, 1);
-        return false;
-      }
-    }
-  }
+  return mbar_wait_or_abort(bar, parity, abort, &g_tc_timeout);
 }
-
-__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
-                                            int c3, int c4, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
-      "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-// Two E4M3 codes (low byte first) to an f16x2 pair.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
-  uint32_t d;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"((unsigned short)(two_codes & 0xffffu)));
-  return d;
-}
-
-// bf16x2 or f16x2 bits to f16x2 bits.
-template <typename T> __device__ __forceinline__ uint32_t to_f16x2(uint32_t v);
-template <> __device__ __forceinline__ uint32_t to_f16x2<__half>(uint32_t v) { return v; }
-template <> __device__ __forceinline__ uint32_t to_f16x2<__nv_bfloat16>(uint32_t v) {
-  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v));
-  __half2 h = __floats2half2_rn(f.x, f.y);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
-__device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
-  uint32_t d;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
-  return d;
-}
-
-template <typename T> struct Mma;
-template <> struct Mma<__nv_bfloat16> {
-  static __device__ __forceinline__ void run(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                             uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-  }
-  static __device__ __forceinline__ uint32_t pack(float lo, float hi, float& rlo, float& rhi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    rlo = __low2float(v);
-    rhi = __high2float(v);
-    return *reinterpret_cast<uint32_t*>(&v);
-  }
-};
-template <> struct Mma<__half> {
-  static __device__ __forceinline__ void run(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                             uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-  }
-  static __device__ __forceinline__ uint32_t pack(float lo, float hi, float& rlo, float& rhi) {
-    __half2 v = __floats2half2_rn(lo, hi);
-    rlo = __low2float(v);
-    rhi = __high2float(v);
-    return *reinterpret_cast<uint32_t*>(&v);
-  }
-};
 
 __device__ __forceinline__ void named_sync_consumers() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
@@ -914,40 +788,6 @@ __global__ void __launch_bounds__(kThreads, MINB)
 
 // ---------------------------------------------------------------- host side ----
 
-static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
-                                         &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// 5-D view of a [num_blocks, bs, Hkv, D] pool of e-byte elements: (d_lo 128/e,
-// token bs, d_hi D*e/128, head Hkv, block num_blocks); one box is a whole
-// (block, head) tile, landing as 128-byte rows with the 128B swizzle.
-static bool encode_pool_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int e,
-                            int D, int bs, int Hkv, int64_t nb) {
-  auto enc = tensor_map_encoder();
-  if (!enc) return false;
-  const cuuint64_t row = 128 / e;  // elements per 128-byte row
-  cuuint64_t dims[5] = {row, (cuuint64_t)bs, (cuuint64_t)(D / row), (cuuint64_t)Hkv, (cuuint64_t)nb};
-  cuuint64_t strides[4] = {(cuuint64_t)Hkv * D * e, 128, (cuuint64_t)D * e,
-                           (cuuint64_t)bs * Hkv * D * e};
-  cuuint32_t box[5] = {(cuuint32_t)row, (cuuint32_t)bs, (cuuint32_t)(D / row), 1, 1};
-  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUresult r = enc(map, dt, 5, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-// Returns the timeout word of the tensor-core kernel (1 if any bounded wait
-// expired), optionally clearing it. Synchronises the device.
 int tc_timeout_flag(bool clear, int* value) {
   int v = 0;
   if (cudaMemcpyFromSymbol(&v, g_tc_timeout, sizeof(int)) != cudaSuccess) return -1;

@@ -15,6 +15,7 @@ bool tc_supported(int q_dtype, int cache_dtype, int head_dim, int group);
 cudaError_t launch_decode_tc(const DecodeParams& prm, int q_dtype, int cache_dtype,
                              int max_ctas, int num_sms, cudaStream_t stream);
 int tc_timeout_flag(bool clear, int* value);
+int pf_timeout_flag(bool clear, int* value);
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
@@ -67,9 +68,10 @@ extern "C" {
 int pkv_version(void) { return 100; }
 
 int pkv_device_status(int clear) {
-  int v = 0;
-  if (tc_timeout_flag(clear != 0, &v) != 0) return PKV_ERR_CUDA;
-  return v;
+  int v = 0, w = 0;
+  if (tc_timeout_flag(clear != 0, &v) != 0 || pf_timeout_flag(clear != 0, &w) != 0)
+    return PKV_ERR_CUDA;
+  return v | w;
 }
 
 const char* pkv_status_string(int status) {

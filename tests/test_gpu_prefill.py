@@ -1,0 +1,158 @@
+"""paged_attention_prefill (causal multi-token queries over the paged cache)
+through the C ABI against the fp64 oracle: full prefills, chunks continuing a
+cached context, GQA/MQA group sizes, head dims, block sizes, dtypes, and the
+edge cases (poisoned slots past the range, out-of-pool ids, chunks longer than
+max_q_len, chunks longer than their context)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_367_b200 as pkv
+from paged_kv_cache_367_b200 import workloads as W
+from parity import TOL
+
+pytestmark = pytest.mark.gpu
+
+TORCH = {"bf16": torch.bfloat16, "f16": torch.float16}
+
+
+def make_case(lens, qlens, Hq, Hkv, D, bs, dt, dev, seed=0, spare=5):
+    rng = np.random.default_rng(seed)
+    gen = torch.Generator().manual_seed(seed)
+    nbs = [-(-L // bs) for L in lens]
+    nb = sum(nbs) + spare
+    ids = rng.permutation(nb)
+    mbps = max(nbs + [1])
+    bt = np.full((len(lens), mbps), -1, np.int32)
+    n = 0
+    for i, k in enumerate(nbs):
+        bt[i, :k] = ids[n:n + k]
+        n += k
+    kc = torch.randn((nb, bs, Hkv, D), generator=gen).to(TORCH[dt])
+    vc = torch.randn((nb, bs, Hkv, D), generator=gen).to(TORCH[dt])
+    # Slots past every sequence's length hold NaN: they must never reach the output.
+    used = np.zeros((nb, bs), bool)
+    for i, L in enumerate(lens):
+        for t in range(L):
+            used[bt[i, t // bs], t % bs] = True
+    mask = torch.from_numpy(~used)
+    kc[mask] = float("nan")
+    vc[mask] = float("nan")
+    qs = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    q = torch.randn((int(qs[-1]), Hq, D), generator=gen).to(TORCH[dt])
+    return dict(kc=kc.to(dev), vc=vc.to(dev), bt=bt, lens=np.asarray(lens, np.int32), qs=qs,
+                q=q.to(dev), Hq=Hq, Hkv=Hkv, D=D, bs=bs, dt=dt, dev=dev)
+
+
+def run_gpu(c, max_q_len=None, bt=None, fill=float("nan")):
+    dev = c["dev"]
+    out = torch.full(tuple(c["q"].shape), fill, dtype=c["q"].dtype, device=dev)
+    bt = c["bt"] if bt is None else bt
+    mq = int(np.diff(c["qs"]).max()) if max_q_len is None else max_q_len
+    pkv.paged_attention_prefill(out, c["q"], c["kc"], c["vc"], torch.from_numpy(bt).to(dev),
+                                torch.from_numpy(c["lens"]).to(dev),
+                                torch.from_numpy(c["qs"]).to(dev), max_q_len=mq,
+                                scale=c["D"] ** -0.5)
+    torch.cuda.synchronize()
+    assert pkv.pkv_device_status() == 0
+    return out
+
+
+def run_oracle(c, bt=None):
+    bt = c["bt"] if bt is None else bt
+    want, _ = oracle.prefill(W.host(c["q"]), W.host(c["kc"]), W.host(c["vc"]), bt, c["lens"],
+                             c["qs"], num_heads=c["Hq"], num_kv_heads=c["Hkv"], head_dim=c["D"],
+                             block_size=c["bs"], scale=c["D"] ** -0.5, q_dtype=c["dt"],
+                             cache_dtype=c["dt"])
+    return want
+
+
+def check(got, want, dt, rows=None):
+    g = got.float().cpu().numpy().astype(np.float64)
+    if rows is not None:
+        g, want = g[rows], want[rows]
+    err = np.abs(g - want)
+    assert np.all(np.isfinite(g))
+    assert err.max() <= TOL[dt][0] and err.mean() <= TOL[dt][1], (err.max(), err.mean())
+
+
+CASES = {
+    "full prefills": ([1, 17, 64, 100, 300], [1, 17, 64, 100, 300]),
+    "chunks over a cached context": ([500, 130, 64, 1000], [128, 3, 64, 37]),
+    "single tokens": ([1, 50, 777], [1, 1, 1]),
+}
+
+
+@pytest.mark.parametrize("case", list(CASES))
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (32, 8), (16, 1), (12, 2), (6, 2), (64, 4)])
+def test_prefill_parity_group_sizes(cuda_dev, case, Hq, Hkv):
+    lens, qlens = CASES[case]
+    c = make_case(lens, qlens, Hq, Hkv, 128, 16, "bf16", cuda_dev, seed=Hq + Hkv)
+    check(run_gpu(c), run_oracle(c), "bf16")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("bs", [8, 16, 32])
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+def test_prefill_parity_dims_blocks_dtypes(cuda_dev, D, bs, dt):
+    c = make_case([400, 90, 33], [200, 90, 5], 16, 4, D, bs, dt, cuda_dev, seed=D + bs)
+    check(run_gpu(c), run_oracle(c), dt)
+
+
+def test_prefill_long_chunk_many_tiles(cuda_dev):
+    c = make_case([3000, 2100], [1024, 2100], 32, 8, 128, 16, "bf16", cuda_dev, seed=9)
+    got = run_gpu(c)
+    # Sampled rows (the oracle is slow at this size): every 37th row and the last ones.
+    T = int(c["qs"][-1])
+    rows = np.unique(np.concatenate([np.arange(0, T, 37), np.arange(T - 5, T)]))
+    items = np.stack(np.meshgrid(rows, np.arange(32), indexing="ij"), -1).reshape(-1, 2)
+    want, _ = oracle.prefill(W.host(c["q"]), W.host(c["kc"]), W.host(c["vc"]), c["bt"],
+                             c["lens"], c["qs"], num_heads=32, num_kv_heads=8, head_dim=128,
+                             block_size=16, scale=128 ** -0.5, q_dtype="bf16",
+                             cache_dtype="bf16", items=items)
+    g = got.float().cpu().numpy()[items[:, 0], items[:, 1]].astype(np.float64)
+    err = np.abs(g - want)
+    assert err.max() <= TOL["bf16"][0] and err.mean() <= TOL["bf16"][1]
+
+
+def test_single_token_rows_match_decode(cuda_dev):
+    c = make_case([1, 50, 777, 64], [1, 1, 1, 1], 32, 8, 128, 16, "bf16", cuda_dev, seed=4)
+    got = run_gpu(c)
+    out = torch.empty_like(c["q"])
+    S = 4
+    ws = torch.empty(pkv.paged_attention_workspace_size(S, 32, 8, 128, 777, 0) + 1,
+                     dtype=torch.uint8, device=cuda_dev)
+    pkv.paged_attention_decode(out, c["q"], c["kc"], c["vc"], torch.from_numpy(c["bt"]).to(cuda_dev),
+                               torch.from_numpy(c["lens"]).to(cuda_dev), max_seq_len=777,
+                               scale=128 ** -0.5, workspace=ws)
+    torch.cuda.synchronize()
+    assert (got.float() - out.float()).abs().max().item() <= 2 * TOL["bf16"][0]
+
+
+def test_chunk_longer_than_max_q_len_computes_its_last_rows(cuda_dev):
+    c = make_case([200, 100], [150, 100], 8, 2, 64, 16, "bf16", cuda_dev, seed=12)
+    got = run_gpu(c, max_q_len=64, fill=0.0)
+    want = run_oracle(c)
+    rows = np.r_[150 - 64:150, 250 - 64:250]
+    check(got, want, "bf16", rows=rows)
+    skipped = np.r_[0:150 - 64, 150:250 - 64]
+    assert torch.all(got[torch.from_numpy(skipped).to(cuda_dev)] == 0)
+
+
+def test_chunk_longer_than_its_context_gives_zero_rows(cuda_dev):
+    # 10 query tokens over a 6-token context: the first 4 sit before position 0.
+    c = make_case([6, 40], [10, 8], 8, 8, 64, 8, "bf16", cuda_dev, seed=2)
+    got = run_gpu(c)
+    want = run_oracle(c)
+    assert np.all(want[:4] == 0)
+    check(got, want, "bf16")
+
+
+def test_block_ids_outside_the_pool_read_as_zeros(cuda_dev):
+    c = make_case([70, 33], [20, 33], 16, 4, 128, 16, "bf16", cuda_dev, seed=6)
+    bt = c["bt"].copy()
+    nb = c["kc"].shape[0]
+    bt[0, 1] = nb + 7
+    bt[1, 0] = -3
+    check(run_gpu(c, bt=bt), run_oracle(c, bt=bt), "bf16")

@@ -171,3 +171,26 @@ def test_copy_blocks_rejects_bad_arguments(lib, kw, code):
 ])
 def test_swap_blocks_rejects_bad_arguments(lib, kw, code):
     assert swap(lib, **kw) == code
+
+
+def prefill(lib, **kw):
+    a = dict(out=A, query=A, k_cache=A, v_cache=A, block_table=A, seq_lens=A, query_start=A,
+             num_seqs=2, num_q_tokens=10, max_q_len=8, num_heads=8, num_kv_heads=2, head_dim=128,
+             block_size=16, max_blocks_per_seq=8, num_blocks=100, scale=0.1, q_dtype=BF16,
+             cache_dtype=BF16, stream=None)
+    a.update(kw)
+    return lib.paged_attention_prefill(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(num_seqs=0), OK), (dict(num_q_tokens=0), OK), (dict(max_q_len=0), OK),
+    (dict(out=None), ENULL), (dict(query_start=None), ENULL), (dict(block_table=None), ENULL),
+    (dict(num_heads=6, num_kv_heads=4), ESHAPE), (dict(num_seqs=-1), ESHAPE),
+    (dict(num_blocks=0), ESHAPE), (dict(max_blocks_per_seq=0), ESHAPE),
+    (dict(scale=float("nan")), ESHAPE), (dict(num_seqs=70000), ESHAPE),
+    (dict(head_dim=96), EUNSUP), (dict(block_size=4), EUNSUP),
+    (dict(cache_dtype=FP8), EDTYPE), (dict(q_dtype=F32, cache_dtype=F32), EDTYPE),
+    (dict(query=A + 8), EALIGN), (dict(query_start=A + 2), EALIGN),
+])
+def test_prefill_rejects_bad_arguments(lib, kw, code):
+    assert prefill(lib, **kw) == code
