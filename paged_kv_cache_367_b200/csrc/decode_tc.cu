@@ -34,6 +34,7 @@
 //    error word, skips the rest of its work and still waits, bounded, for its
 //    own copies in flight before it exits.
 #include <cuda.h>
+#include <atomic>
 #include <type_traits>
 #include <cudaTypedefs.h>
 
@@ -812,7 +813,12 @@ static cudaError_t launch_tc_t(const DecodeParams& prm, const CUtensorMap& mk,
                                cudaStream_t stream) {
   using C = tc::Cfg<D, NT, NS, F8 ? 1 : 2>;
   auto kernel = tc::decode_tc_kernel<T, D, NT, NS, MINB, F8>;
-  static int occ = 0;
+  // The shared-memory opt-in is a per-device setting: done, and the residency
+  // queried, once per device.
+  static std::atomic<int> occ_of[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  int occ = occ_of[dev].load(std::memory_order_relaxed);
   if (occ == 0) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmem);
@@ -821,6 +827,7 @@ static cudaError_t launch_tc_t(const DecodeParams& prm, const CUtensorMap& mk,
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, tc::kThreads, C::kSmem);
     if (e != cudaSuccess) return e;
     occ = n > 0 ? n : 1;
+    occ_of[dev].store(occ, std::memory_order_relaxed);
   }
   int grid = occ * num_sms;
   if (grid > kMaxRanges) grid = kMaxRanges;

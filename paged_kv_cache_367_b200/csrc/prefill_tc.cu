@@ -30,6 +30,8 @@
 //    zeroed in V, so stale or poisoned memory never reaches the output.
 //  * Every mbarrier wait is bounded; expiry sets an error word, the CTA stops
 //    and still waits, bounded, for its own copies in flight.
+#include <atomic>
+
 #include "common.cuh"
 #include "tc_common.cuh"
 
@@ -326,9 +328,15 @@ cudaError_t launch_t(const PrefillParams& p, const CUtensorMap& mk, const CUtens
   constexpr int NS = D == 128 ? 2 : 4;
   using C = Cfg<D, NS>;
   auto kernel = prefill_tc_kernel<T, D, NS>;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::kSmem);
-  if (e != cudaSuccess) return e;
+  static std::atomic<int> opted_in[64];  // the shared-memory opt-in, once per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!opted_in[dev].load(std::memory_order_relaxed)) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (e != cudaSuccess) return e;
+    opted_in[dev].store(1, std::memory_order_relaxed);
+  }
   const int g = p.num_heads / p.num_kv_heads;
   const int64_t tiles = ((int64_t)max_q_len * g + kRows - 1) / kRows;
   dim3 grid((unsigned)tiles, (unsigned)num_seqs, (unsigned)p.num_kv_heads);
