@@ -67,6 +67,19 @@ typedef enum {
 /* Flags for paged_attention_decode. */
 #define PKV_DECODE_FORCE_SIMT 1u  /* use the CUDA-core kernel even where the
                                      tensor-core kernel applies */
+/* The workspace's split counters are zero on entry, as every decode call
+ * leaves them (or as the caller zeroed them): the call skips the memset that
+ * zeroes them. Do not set it on a fresh workspace, on one used for anything
+ * else since, or after pkv_device_status reported an expired wait. */
+#define PKV_DECODE_ZEROED_WORKSPACE 2u
+/* Start the tensor-core kernel while the previous kernel in the stream is still
+ * running (programmatic dependent launch); it sets up its schedule and reads
+ * the block table, and waits for that kernel to finish only before its first
+ * read of the caches. Allowed only when the previous kernel writes nothing the
+ * call reads except the K/V caches (e.g. paged_kv_append of this step's
+ * tokens) and does not touch `out` or the workspace. Without a preceding
+ * kernel, or on the CUDA-core path, it changes nothing. */
+#define PKV_DECODE_EARLY_START 4u
 
 /*
  * paged_kv_append — write new tokens' K/V into their slots ("reshape and cache").

@@ -19,12 +19,15 @@ __all__ = ["paged_kv_append", "paged_attention_decode", "paged_attention_workspa
            "paged_attention_prefill",
            "pkv_device_status", "pkv_status_string", "pkv_version", "load_library", "PagedKVError",
            "PKV_F32", "PKV_F16", "PKV_BF16", "PKV_FP8_E4M3", "PKV_DECODE_FORCE_SIMT",
+           "PKV_DECODE_ZEROED_WORKSPACE", "PKV_DECODE_EARLY_START",
            "LIB_PATH", "EXPORTED_SYMBOLS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedkv.so")
 
 PKV_F32, PKV_F16, PKV_BF16, PKV_FP8_E4M3 = 0, 1, 2, 3
 PKV_DECODE_FORCE_SIMT = 1
+PKV_DECODE_ZEROED_WORKSPACE = 2
+PKV_DECODE_EARLY_START = 4
 
 EXPORTED_SYMBOLS = ("paged_kv_append", "paged_attention_workspace_size",
                     "paged_attention_decode", "paged_attention_decode_static",

@@ -50,6 +50,10 @@ __global__ void __launch_bounds__(256) append_kernel(
     void* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping, int num_tokens,
     int num_kv_heads, int head_dim, int64_t num_slots, const float* __restrict__ k_scale,
     const float* __restrict__ v_scale) {
+  // A kernel launched after this one with programmatic stream serialization
+  // (the decode's early start) may begin now; it waits for this grid to finish
+  // before it reads the caches.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int vec_per_row = head_dim / 8;
   const int64_t row = (int64_t)num_kv_heads * head_dim;
   const int64_t total = (int64_t)num_tokens * num_kv_heads * vec_per_row;

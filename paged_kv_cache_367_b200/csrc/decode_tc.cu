@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
     // tile copies. A final descriptor marks the end.
     uint32_t kc = 0;  // chunk counter: stage kc % NS, phase (kc / NS) & 1
     uint32_t armed = 0, last_parity = 0;
-    bool ok = true;
+    bool ok = true, waited = false;
     const T* qbase = static_cast<const T*>(prm.query);
     int64_t r = blockIdx.x;
     int ci = sched->d_i;            // forward cursor for dynamic ranges
@@ -369,6 +369,12 @@ __global__ void __launch_bounds__(kThreads, MINB)
                         qbytes, full + stage);
           }
           __syncwarp();
+          if (!waited) {
+            // Launched early (programmatic dependent launch): the previous
+            // kernel may still be writing the caches. A no-op otherwise.
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            waited = true;
+          }
           const int b = lane - (rel - batch);
           if (ok && b >= 0 && b < nblk) {
             tma_load_5d(st + b * tile, &tmap_k, 0, 0, 0, seg.head, cur, full + stage);
@@ -810,7 +816,7 @@ bool tc_supported(int q_dtype, int cache_dtype, int head_dim, int group) {
 template <typename T, int D, int NT, int NS, int MINB, bool F8>
 static cudaError_t launch_tc_t(const DecodeParams& prm, const CUtensorMap& mk,
                                const CUtensorMap& mv, int max_ctas, int num_sms,
-                               cudaStream_t stream) {
+                               bool early_start, cudaStream_t stream) {
   using C = tc::Cfg<D, NT, NS, F8 ? 1 : 2>;
   auto kernel = tc::decode_tc_kernel<T, D, NT, NS, MINB, F8>;
   // The shared-memory opt-in is a per-device setting: done, and the residency
@@ -842,6 +848,19 @@ static cudaError_t launch_tc_t(const DecodeParams& prm, const CUtensorMap& mk,
                      ? (kDynRanges < kMaxRanges - grid ? kDynRanges : kMaxRanges - grid)
                      : 0;
   p.static_share = 870;
+  if (early_start) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(tc::kThreads);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, p, mk, mv);
+  }
   kernel<<<grid, tc::kThreads, C::kSmem, stream>>>(p, mk, mv);
   return cudaGetLastError();
 }
@@ -849,19 +868,19 @@ static cudaError_t launch_tc_t(const DecodeParams& prm, const CUtensorMap& mk,
 template <typename T, int D, bool F8>
 static cudaError_t launch_tc_d(const DecodeParams& prm, const CUtensorMap& mk,
                                const CUtensorMap& mv, int max_ctas, int num_sms,
-                               cudaStream_t stream) {
+                               bool early_start, cudaStream_t stream) {
   // Two CTAs per SM (two producers keep more copies in flight than one) where
   // shared memory allows; head_dim 128 with more than 8 heads per group runs one.
   const int g = prm.num_heads / prm.num_kv_heads;
   // E4M3 stages are half the size: four of them per CTA.
   constexpr int kNS = F8 ? 4 : (D == 128 ? 2 : 4);
-  if (g <= 8) return launch_tc_t<T, D, 1, kNS, 2, F8>(prm, mk, mv, max_ctas, num_sms, stream);
-  if (D == 64 || F8) return launch_tc_t<T, D, 2, 4, 2, F8>(prm, mk, mv, max_ctas, num_sms, stream);
-  return launch_tc_t<T, D, 2, 4, 1, F8>(prm, mk, mv, max_ctas, num_sms, stream);
+  if (g <= 8) return launch_tc_t<T, D, 1, kNS, 2, F8>(prm, mk, mv, max_ctas, num_sms, early_start, stream);
+  if (D == 64 || F8) return launch_tc_t<T, D, 2, 4, 2, F8>(prm, mk, mv, max_ctas, num_sms, early_start, stream);
+  return launch_tc_t<T, D, 2, 4, 1, F8>(prm, mk, mv, max_ctas, num_sms, early_start, stream);
 }
 
 cudaError_t launch_decode_tc(const DecodeParams& prm, int q_dtype, int cache_dtype, int max_ctas,
-                             int num_sms, cudaStream_t stream) {
+                             int num_sms, bool early_start, cudaStream_t stream) {
   const bool f8 = cache_dtype == PKV_FP8_E4M3;
   const CUtensorMapDataType dt = f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                  : q_dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -875,16 +894,16 @@ cudaError_t launch_decode_tc(const DecodeParams& prm, int q_dtype, int cache_dty
     return cudaErrorInvalidValue;
   if (f8) {
     return q_dtype == PKV_BF16
-               ? launch_tc_d<__nv_bfloat16, 128, true>(prm, mk, mv, max_ctas, num_sms, stream)
-               : launch_tc_d<__half, 128, true>(prm, mk, mv, max_ctas, num_sms, stream);
+               ? launch_tc_d<__nv_bfloat16, 128, true>(prm, mk, mv, max_ctas, num_sms, early_start, stream)
+               : launch_tc_d<__half, 128, true>(prm, mk, mv, max_ctas, num_sms, early_start, stream);
   }
   if (q_dtype == PKV_BF16) {
     return prm.head_dim == 128
-               ? launch_tc_d<__nv_bfloat16, 128, false>(prm, mk, mv, max_ctas, num_sms, stream)
-               : launch_tc_d<__nv_bfloat16, 64, false>(prm, mk, mv, max_ctas, num_sms, stream);
+               ? launch_tc_d<__nv_bfloat16, 128, false>(prm, mk, mv, max_ctas, num_sms, early_start, stream)
+               : launch_tc_d<__nv_bfloat16, 64, false>(prm, mk, mv, max_ctas, num_sms, early_start, stream);
   }
-  return prm.head_dim == 128 ? launch_tc_d<__half, 128, false>(prm, mk, mv, max_ctas, num_sms, stream)
-                             : launch_tc_d<__half, 64, false>(prm, mk, mv, max_ctas, num_sms, stream);
+  return prm.head_dim == 128 ? launch_tc_d<__half, 128, false>(prm, mk, mv, max_ctas, num_sms, early_start, stream)
+                             : launch_tc_d<__half, 64, false>(prm, mk, mv, max_ctas, num_sms, early_start, stream);
 }
 
 }  // namespace pkv

@@ -13,7 +13,7 @@ cudaError_t launch_decode_simt(const DecodeParams& prm, int q_dtype, int cache_d
                                int max_ctas, int num_sms, cudaStream_t stream);
 bool tc_supported(int q_dtype, int cache_dtype, int head_dim, int group);
 cudaError_t launch_decode_tc(const DecodeParams& prm, int q_dtype, int cache_dtype,
-                             int max_ctas, int num_sms, cudaStream_t stream);
+                             int max_ctas, int num_sms, bool early_start, cudaStream_t stream);
 int tc_timeout_flag(bool clear, int* value);
 int pf_timeout_flag(bool clear, int* value);
 
@@ -134,7 +134,8 @@ int paged_attention_decode(void* out, const void* query, const void* k_cache,
                            void* stream) {
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 ||
       max_blocks_per_seq <= 0 || num_blocks <= 0 || max_seq_len < 0 || partition_size < 0 ||
-      max_ctas < 0 || !isfinite(scale))
+      max_ctas < 0 || !isfinite(scale) ||
+      (flags & ~(PKV_DECODE_FORCE_SIMT | PKV_DECODE_ZEROED_WORKSPACE | PKV_DECODE_EARLY_START)))
     return PKV_ERR_SHAPE;
   if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
   if (block_size != 8 && block_size != 16 && block_size != 32) return PKV_ERR_UNSUPPORTED;
@@ -189,15 +190,16 @@ int paged_attention_decode(void* out, const void* query, const void* k_cache,
   cudaStream_t st = (cudaStream_t)stream;
   const int group = num_heads / num_kv_heads;
   cudaError_t e;
-  if (ws.total > 0) {
+  if (ws.total > 0 && !(flags & PKV_DECODE_ZEROED_WORKSPACE)) {
     // Per-unit counters of finished split tokens and the dynamic-range counter
-    // start at zero every call.
+    // start at zero (each call also leaves them at zero).
     e = cudaMemsetAsync(prm.ws_done, 0, sizeof(int32_t) * ((size_t)num_seqs * num_kv_heads + 1),
                         st);
     if (e != cudaSuccess) return PKV_ERR_CUDA;
   }
   if (!(flags & PKV_DECODE_FORCE_SIMT) && tc_supported(q_dtype, cache_dtype, head_dim, group))
-    e = launch_decode_tc(prm, q_dtype, cache_dtype, max_ctas, sms, st);
+    e = launch_decode_tc(prm, q_dtype, cache_dtype, max_ctas, sms,
+                         (flags & PKV_DECODE_EARLY_START) != 0, st);
   else
     e = launch_decode_simt(prm, q_dtype, cache_dtype, max_ctas, sms, st);
   if (e != cudaSuccess) return PKV_ERR_CUDA;

@@ -491,7 +491,11 @@ __device__ __forceinline__ bool complete_piece(const DecodeParams& prm, const Se
                : "=r"(before)
                : "l"(prm.ws_done + u), "r"(s.t1 - s.t0)
                : "memory");
-  return before + (s.t1 - s.t0) == s.len;
+  const bool last = before + (s.t1 - s.t0) == s.len;
+  // Every piece is in and no other CTA touches this counter again in this
+  // call: leave it at zero for the next call on the same workspace.
+  if (last) prm.ws_done[u] = 0;
+  return last;
 }
 
 // Called by `nthreads` threads (index tid) of one CTA after they wrote the

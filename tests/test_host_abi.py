@@ -194,3 +194,8 @@ def prefill(lib, **kw):
 ])
 def test_prefill_rejects_bad_arguments(lib, kw, code):
     assert prefill(lib, **kw) == code
+
+
+def test_decode_rejects_unknown_flags(lib):
+    assert decode(lib, flags=8) == ESHAPE
+    assert decode(lib, flags=1 << 31) == ESHAPE
