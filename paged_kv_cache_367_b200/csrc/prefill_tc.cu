@@ -218,12 +218,14 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
     {
+      // k-steps outermost: the eight n-tiles are eight independent accumulation
+      // chains, so consecutive MMAs do not wait on each other.
       const int mi = lane >> 3, rr = lane & 7;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int t = 16 * q + rr + 8 * (mi >> 1);
+      for (int ks = 0; ks < KS; ++ks) {
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
+        for (int q = 0; q < 4; ++q) {
+          const int t = 16 * q + rr + 8 * (mi >> 1);
           uint32_t b[4];
           ldsm_x4(b, kst + kv_offset<D>(t, 2 * ks + (mi & 1), bs));
           Mma<T>::run(s[2 * q], qa[ks], b[0], b[1]);
