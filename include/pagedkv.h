@@ -237,11 +237,14 @@ int paged_attention_prefill(void* out, const void* query, const void* k_cache,
                             void* stream);
 
 /*
- * Health word of the device kernels. Every wait inside a kernel is bounded
- * (about one second); a wait that expires makes its CTA skip the rest of its
- * work and sets this word, so a wrong result is reported instead of a hung GPU.
- * Returns 0 (no expiry since the last clear), 1 (a wait expired), or
- * PKV_ERR_CUDA. Synchronises the current device; clear != 0 resets the word.
+ * Health word of the device kernels, a bitmask since the last clear:
+ *   1  a bounded wait inside a kernel expired (every wait is bounded, about one
+ *      second; the CTA skips the rest of its work, so a wrong result is
+ *      reported instead of a hung GPU);
+ *   2  a kernel read a block-table entry outside [0, num_blocks) (a corrupt
+ *      table; those rows read as zeros).
+ * Returns 0 when healthy, the bitmask, or PKV_ERR_CUDA. Synchronises the
+ * current device; clear != 0 resets the word.
  */
 int pkv_device_status(int clear);
 

@@ -142,6 +142,14 @@ int64_t pkv_bm_seq_len(const pkv_block_manager* bm, int64_t seq_id);
 /* Reference count of a device block (0 for free or cached-unheld), or
  * PKV_ERR_SHAPE for an id out of range. */
 int pkv_bm_refcount(const pkv_block_manager* bm, int32_t block);
+/* Pool usage, the ledger's metrics (the pages' KV-pool usage gauge, p4 §6.6):
+ * out (host int64[6]) receives num_blocks, blocks held by resident sequences,
+ * cached blocks no sequence holds, free blocks, tokens of resident sequences
+ * (each sequence counted), and the slots of held blocks that hold a token
+ * (a shared block counted once, at its fullest). Fragmentation of the held
+ * blocks is 1 - used slots / (held * block_size). */
+int pkv_bm_usage(const pkv_block_manager* bm, int64_t* out);
+
 /* Full consistency check of the ledger: every reference count equals the
  * number of table entries that point at the block, and every block is exactly
  * one of held, free, or cached-unheld. PKV_OK or PKV_ERR_SHAPE. */

@@ -37,7 +37,7 @@ EXPORTED_SYMBOLS = ("paged_kv_append", "paged_attention_workspace_size",
                     "pkv_bm_can_allocate", "pkv_bm_allocate", "pkv_bm_can_append",
                     "pkv_bm_append_slot", "pkv_bm_append_slots", "pkv_bm_fork", "pkv_bm_free", "pkv_bm_swap_out",
                     "pkv_bm_swap_in", "pkv_bm_block_tables", "pkv_bm_seq_len", "pkv_bm_refcount",
-                    "pkv_bm_check", "paged_kv_copy_blocks", "paged_kv_swap_blocks")
+                    "pkv_bm_usage", "pkv_bm_check", "paged_kv_copy_blocks", "paged_kv_swap_blocks")
 
 _DTYPE_CODES = {torch.float32: PKV_F32, torch.float16: PKV_F16, torch.bfloat16: PKV_BF16,
                 torch.uint8: PKV_FP8_E4M3, torch.float8_e4m3fn: PKV_FP8_E4M3}
@@ -112,6 +112,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pkv_bm_seq_len.restype = I64
     lib.pkv_bm_refcount.argtypes = [P, ctypes.c_int32]
     lib.pkv_bm_refcount.restype = I
+    lib.pkv_bm_usage.argtypes = [P, P]
+    lib.pkv_bm_usage.restype = I
     lib.pkv_bm_check.argtypes = [P]
     lib.pkv_bm_check.restype = I
     lib.paged_kv_copy_blocks.argtypes = [P, P, P, I, I64, I64, P]

@@ -130,5 +130,15 @@ class BlockManager:
     def refcount(self, block: int) -> int:
         return self._lib.pkv_bm_refcount(self._h, block)
 
+    def usage(self) -> dict:
+        """Pool usage: blocks held / cached-unheld / free, resident tokens, used
+        slots of held blocks, and the held blocks' fragmentation."""
+        out = np.zeros(6, dtype=np.int64)
+        _check("pkv_bm_usage", self._lib.pkv_bm_usage(self._h, out.ctypes.data))
+        nb, held, cached, free, tokens, used = (int(x) for x in out)
+        return {"num_blocks": nb, "held": held, "cached_unheld": cached, "free": free,
+                "usage": held / nb if nb else 0.0, "tokens": tokens, "used_slots": used,
+                "fragmentation": 1.0 - used / (held * self.block_size) if held else 0.0}
+
     def check(self) -> None:
         _check("pkv_bm_check", self._lib.pkv_bm_check(self._h))

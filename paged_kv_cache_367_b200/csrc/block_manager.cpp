@@ -490,6 +490,31 @@ int pkv_bm_refcount(const pkv_block_manager* bm, int32_t block) {
   return bm->dev[block].ref;
 }
 
+int pkv_bm_usage(const pkv_block_manager* bm, int64_t* out) {
+  if (!bm || !out) return PKV_ERR_NULL;
+  std::unordered_map<int32_t, int64_t> fill;  // held block -> fullest use
+  int64_t tokens = 0;
+  for (const auto& kv : bm->seqs) {
+    const Seq& s = kv.second;
+    if (s.swapped) continue;
+    tokens += s.len;
+    for (size_t j = 0; j < s.blocks.size(); ++j) {
+      const int64_t f = std::min<int64_t>(bm->bs, s.len - (int64_t)j * bm->bs);
+      int64_t& cur = fill[s.blocks[j]];
+      cur = std::max(cur, f);
+    }
+  }
+  int64_t used = 0;
+  for (const auto& kv : fill) used += kv.second;
+  out[0] = (int64_t)bm->dev.size();
+  out[1] = (int64_t)fill.size();
+  out[2] = (int64_t)bm->lru.size();
+  out[3] = (int64_t)bm->free_dev.size();
+  out[4] = tokens;
+  out[5] = used;
+  return PKV_OK;
+}
+
 int pkv_bm_check(const pkv_block_manager* bm) {
   if (!bm) return PKV_ERR_NULL;
   const size_t nb = bm->dev.size(), nh = bm->host_ref.size();

@@ -19,6 +19,8 @@
 
 namespace pkv {
 
+__device__ int g_simt_status = 0;  // bit 1: a block id outside the pool was read
+
 constexpr int kSimtThreads = 128;
 constexpr int kSimtHeads = 8;    // query heads per pass
 
@@ -90,6 +92,7 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(const DecodeP
           act[u] = t < seg.t1;
           int64_t phys = -1;
           if (act[u]) phys = __ldg(bt + t / bs);
+          if (act[u] && (phys < 0 || phys >= prm.num_blocks)) atomicOr(&g_simt_status, 2);
           if (act[u] && phys >= 0 && phys < prm.num_blocks) {
             const int64_t off = ((phys * bs + t % bs) * row_stride) + (int64_t)h * D + l16 * DPL;
             load_row<KT, DPL>(kc + off, kv[u]);
@@ -221,6 +224,17 @@ cudaError_t launch_decode_simt(const DecodeParams& prm_in, int q_dtype, int cach
     default:
       return cudaErrorInvalidValue;
   }
+}
+
+int simt_status_flag(bool clear, int* value) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_simt_status, sizeof(int)) != cudaSuccess) return -1;
+  if (clear && v) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_simt_status, &zero, sizeof(int)) != cudaSuccess) return -1;
+  }
+  *value = v;
+  return 0;
 }
 
 }  // namespace pkv

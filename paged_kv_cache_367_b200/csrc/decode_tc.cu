@@ -45,7 +45,7 @@ namespace pkv {
 
 using namespace tcx;
 
-__device__ int g_tc_timeout = 0;
+__device__ int g_tc_timeout = 0;  // bit 0: a wait expired; bit 1: a block id outside the pool
 
 namespace tc {
 
@@ -377,6 +377,9 @@ __global__ void __launch_bounds__(kThreads, MINB)
           }
           const int b = lane - (rel - batch);
           if (ok && b >= 0 && b < nblk) {
+            // An id outside the pool reads as zeros (the copy's bounds fill);
+            // it is also reported in the status word (bit 1).
+            if ((unsigned)cur >= (unsigned)prm.num_blocks) atomicOr(&g_tc_timeout, 2);
             tma_load_5d(st + b * tile, &tmap_k, 0, 0, 0, seg.head, cur, full + stage);
             tma_load_5d(st + C::kKV + b * tile, &tmap_v, 0, 0, 0, seg.head, cur, full + stage);
           }

@@ -37,7 +37,7 @@
 
 namespace pkv {
 
-__device__ int g_pf_timeout = 0;
+__device__ int g_pf_timeout = 0;  // bit 0: a wait expired; bit 1: a block id outside the pool
 
 namespace pf {
 
@@ -56,6 +56,7 @@ struct PrefillParams {
   const int32_t* query_start;
   int num_heads, num_kv_heads, block_size, max_blocks_per_seq;
   int num_q_tokens, max_q_len;
+  int num_blocks;
   float score_scale;  // softmax scale * log2(e)
 };
 
@@ -145,6 +146,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (lane == 0) mbar_expect_tx(full + stage, (uint32_t)(2 * nblk * tile));
       __syncwarp();
       if (lane < nblk) {
+        if ((unsigned)blk >= (unsigned)p.num_blocks) atomicOr(&g_pf_timeout, 2);  // reads as zeros
         tma_load_5d(st + lane * tile, &tmap_k, 0, 0, 0, h, blk, full + stage);
         tma_load_5d(st + C::kKV + lane * tile, &tmap_v, 0, 0, 0, h, blk, full + stage);
       }
@@ -405,6 +407,7 @@ extern "C" int paged_attention_prefill(void* out, const void* query, const void*
   p.max_blocks_per_seq = max_blocks_per_seq;
   p.num_q_tokens = num_q_tokens;
   p.max_q_len = max_q_len;
+  p.num_blocks = (int)num_blocks;
   p.score_scale = scale * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;

@@ -259,5 +259,24 @@ def test_batched_step_is_all_or_nothing():
     bm.check()
 
 
+def test_usage_metrics():
+    from paged_kv_cache_367_b200 import fragmentation as FR
+    bm = BlockManager(32, 4, prefix_caching=True)
+    lens = [7, 4, 10]
+    for i, L in enumerate(lens):
+        bm.allocate(i, list(range(100 * i, 100 * i + L)))  # nothing shared
+    u = bm.usage()
+    assert (u["num_blocks"], u["held"], u["cached_unheld"], u["free"]) == (32, 6, 0, 26)
+    assert u["tokens"] == 21 and u["used_slots"] == 21
+    assert u["fragmentation"] == pytest.approx(FR.fixed_block_fragmentation(lens, 4))
+    bm.fork(0, 9)                                     # shares seq 0's two blocks
+    u = bm.usage()
+    assert u["held"] == 6 and u["tokens"] == 28 and u["used_slots"] == 21
+    bm.free(1)                                        # its full block stays cached
+    u = bm.usage()
+    assert (u["held"], u["cached_unheld"], u["free"]) == (5, 1, 26)
+    bm.check()
+
+
 def test_model_blocks_needed_closed_form():
     assert [M.blocks_needed(n, 16) for n in (0, 1, 16, 17, 48, 200)] == [0, 1, 1, 2, 3, 13]

@@ -172,6 +172,8 @@ def test_seq_lens_are_clamped_to_the_table(cuda_dev):
     clamped = np.clip(big, 0, wl.max_blocks_per_seq * cfg.block_size).astype(np.int32)
     want = oracle_decode(wl, kc, vc, seq_lens=clamped)
     assert_close(to_f64(out), want, cfg)
+    # The clamped length reaches the table's unused (-1) entries: reported.
+    assert pkv.pkv_device_status(clear=True) == 2
 
 
 def test_block_ids_outside_the_pool_read_as_zeros(cuda_dev):
@@ -187,6 +189,7 @@ def test_block_ids_outside_the_pool_read_as_zeros(cuda_dev):
         out = gpu_step(wl, cuda_dev, append=False, block_table=bt, flags=flags)
         want = oracle_decode(wl, kc, vc, block_table=bt)
         assert_close(to_f64(out), want, cfg)
+        assert pkv.pkv_device_status(clear=True) == 2  # the corrupt entries are reported
 
 
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (32, 8), (64, 8), (16, 1)])
