@@ -81,7 +81,8 @@ def parse_args():
     return ap.parse_args()
 
 
-DECODE_SOURCES = ("common.cuh", "schedule.cuh", "decode_tc.cu", "decode_simt.cu", "pkv_api.cu")
+DECODE_SOURCES = ("common.cuh", "schedule.cuh", "tc_common.cuh", "decode_tc.cu", "decode_simt.cu",
+                  "pkv_api.cu")
 
 
 def source_sha() -> str:
@@ -656,23 +657,27 @@ def run_prefill(args, dev):
         out = torch.empty_like(q)
         btd, lensd, qsd = bt.to(dev), torch.tensor(ctx, dtype=torch.int32, device=dev), qs.to(dev)
 
-        def call():
-            pkv.paged_attention_prefill(out, q, kc, vc, btd, lensd, qsd, max_q_len=max(qlen),
-                                        scale=D ** -0.5)
-        ms = _event_time_ms(call, reps, warmup)
         attended = sum(sum(L - n + r + 1 for r in range(n)) for L, n in zip(ctx, qlen))
         flops = 4.0 * D * Hq * attended
-        tflops = flops / ms / 1e9
-        lines.append({"metric": "paged causal multi-token attention TFLOP/s", "value": round(tflops, 1),
-                      "unit": "TFLOP/s", "higher_is_better": True, "us_per_launch": round(ms * 1e3, 1),
-                      "tokens_per_s": round(T / ms * 1e3, 0), "dtype": "bf16", "data": "synthetic",
-                      "config": {"workload": name + f"; {Hq} q / {Hkv} KV heads, head_dim {D}, "
-                                                    f"block {bs}, shuffled pool"},
-                      "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak,
-                                   "peak_source": peak_src, "unit": "TFLOP/s",
-                                   "frac": round(tflops / peak, 4), "traffic": None,
-                                   "flops": flops,
-                                   "kernel": "mma.sync m16n8k16 (legacy tensor path)"}})
+        for flags, kname in ((0, "tcgen05.mma, accumulators in tensor memory"),
+                             (pkv.PKV_PREFILL_MMA_SYNC, "mma.sync m16n8k16 (legacy tensor path)")):
+            def call():
+                pkv.paged_attention_prefill(out, q, kc, vc, btd, lensd, qsd, max_q_len=max(qlen),
+                                            scale=D ** -0.5, flags=flags)
+            ms = _event_time_ms(call, reps, warmup)
+            assert pkv.pkv_device_status(clear=True) == 0, "device wait expired"
+            tflops = flops / ms / 1e9
+            lines.append({"metric": "paged causal multi-token attention TFLOP/s",
+                          "value": round(tflops, 1), "unit": "TFLOP/s", "higher_is_better": True,
+                          "us_per_launch": round(ms * 1e3, 1),
+                          "tokens_per_s": round(T / ms * 1e3, 0), "dtype": "bf16",
+                          "data": "synthetic",
+                          "config": {"workload": name + f"; {Hq} q / {Hkv} KV heads, head_dim {D}, "
+                                                        f"block {bs}, shuffled pool"},
+                          "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak,
+                                       "peak_source": peak_src, "unit": "TFLOP/s",
+                                       "frac": round(tflops / peak, 4), "traffic": None,
+                                       "flops": flops, "kernel": kname}})
         del kc, vc, q, out
         torch.cuda.empty_cache()
     return lines

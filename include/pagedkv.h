@@ -224,17 +224,21 @@ int paged_attention_decode_static(void* out, const void* query, const void* k_ca
  * p < 0 gets zeros. max_q_len must be >= every q_i: a longer chunk has only its
  * last max_q_len rows computed. Lengths are clamped to max_blocks_per_seq *
  * block_size and query_start to [0, num_q_tokens]. head_dim 64 or 128,
- * block_size 8/16/32; FP8 caches are not supported here (PKV_ERR_DTYPE).
+ * block_size 8/16/32; FP8 caches are not supported here (PKV_ERR_DTYPE). The
+ * default kernel runs on the tcgen05 tensor cores with tensor-memory
+ * accumulators (128 query rows per CTA); flags PKV_PREFILL_MMA_SYNC selects
+ * the mma.sync kernel (64 rows per CTA) instead; other flag bits are an error.
  * Errors: PKV_ERR_SHAPE, PKV_ERR_UNSUPPORTED, PKV_ERR_DTYPE, PKV_ERR_NULL,
  * PKV_ERR_ALIGN, PKV_ERR_CUDA.
  */
+#define PKV_PREFILL_MMA_SYNC 1u  /* use the mma.sync kernel instead of the tcgen05 one */
 int paged_attention_prefill(void* out, const void* query, const void* k_cache,
                             const void* v_cache, const int32_t* block_table,
                             const int32_t* seq_lens, const int32_t* query_start, int num_seqs,
                             int num_q_tokens, int max_q_len, int num_heads, int num_kv_heads,
                             int head_dim, int block_size, int max_blocks_per_seq,
                             int64_t num_blocks, float scale, int q_dtype, int cache_dtype,
-                            void* stream);
+                            unsigned flags, void* stream);
 
 /*
  * Health word of the device kernels, a bitmask since the last clear:

@@ -19,7 +19,7 @@ __all__ = ["paged_kv_append", "paged_attention_decode", "paged_attention_workspa
            "paged_attention_prefill",
            "pkv_device_status", "pkv_status_string", "pkv_version", "load_library", "PagedKVError",
            "PKV_F32", "PKV_F16", "PKV_BF16", "PKV_FP8_E4M3", "PKV_DECODE_FORCE_SIMT",
-           "PKV_DECODE_ZEROED_WORKSPACE", "PKV_DECODE_EARLY_START",
+           "PKV_DECODE_ZEROED_WORKSPACE", "PKV_DECODE_EARLY_START", "PKV_PREFILL_MMA_SYNC",
            "LIB_PATH", "EXPORTED_SYMBOLS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedkv.so")
@@ -28,6 +28,7 @@ PKV_F32, PKV_F16, PKV_BF16, PKV_FP8_E4M3 = 0, 1, 2, 3
 PKV_DECODE_FORCE_SIMT = 1
 PKV_DECODE_ZEROED_WORKSPACE = 2
 PKV_DECODE_EARLY_START = 4
+PKV_PREFILL_MMA_SYNC = 1
 
 EXPORTED_SYMBOLS = ("paged_kv_append", "paged_attention_workspace_size",
                     "paged_attention_decode", "paged_attention_decode_static",
@@ -79,7 +80,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                                   I, I, P, P, I, I, U, P]
     lib.paged_attention_decode_static.restype = I
     lib.paged_attention_prefill.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I64, F,
-                                            I, I, P]
+                                            I, I, U, P]
     lib.paged_attention_prefill.restype = I
     # Block manager and block copies (include/pagedkv_blocks.h).
     lib.pkv_bm_create.argtypes = [I64, I64, I, I]
@@ -222,7 +223,7 @@ def paged_attention_decode_static(out, query, k_cache, v_cache, block_table, seq
 
 
 def paged_attention_prefill(out, query, k_cache, v_cache, block_table, seq_lens, query_start, *,
-                            max_q_len, scale, stream=None) -> None:
+                            max_q_len, scale, flags=0, stream=None) -> None:
     """Causal attention of multi-token queries (chunked prefill, the uncached
     rest of a prefix-cache hit) over the paged cache; see
     paged_attention_prefill in include/pagedkv.h."""
@@ -234,7 +235,7 @@ def paged_attention_prefill(out, query, k_cache, v_cache, block_table, seq_lens,
                                      _ptr(block_table), _ptr(seq_lens), _ptr(query_start), S, T,
                                      int(max_q_len), Hq, Hkv, D, bs, block_table.shape[1], nb,
                                      float(scale), _dtype_code(query), _dtype_code(k_cache),
-                                     _stream(stream))
+                                     int(flags), _stream(stream))
     if st != 0:
         raise PagedKVError("paged_attention_prefill", st)
 

@@ -17,6 +17,7 @@ cudaError_t launch_decode_tc(const DecodeParams& prm, int q_dtype, int cache_dty
 int tc_timeout_flag(bool clear, int* value);
 int pf_timeout_flag(bool clear, int* value);
 int simt_status_flag(bool clear, int* value);
+int pf5_status_flag(bool clear, int* value);
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
@@ -69,11 +70,11 @@ extern "C" {
 int pkv_version(void) { return 100; }
 
 int pkv_device_status(int clear) {
-  int v = 0, w = 0, x = 0;
+  int v = 0, w = 0, x = 0, y = 0;
   if (tc_timeout_flag(clear != 0, &v) != 0 || pf_timeout_flag(clear != 0, &w) != 0 ||
-      simt_status_flag(clear != 0, &x) != 0)
+      simt_status_flag(clear != 0, &x) != 0 || pf5_status_flag(clear != 0, &y) != 0)
     return PKV_ERR_CUDA;
-  return v | w | x;
+  return v | w | x | y;
 }
 
 const char* pkv_status_string(int status) {

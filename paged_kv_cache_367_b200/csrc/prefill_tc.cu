@@ -33,6 +33,7 @@
 #include <atomic>
 
 #include "common.cuh"
+#include "prefill.cuh"
 #include "tc_common.cuh"
 
 namespace pkv {
@@ -47,18 +48,6 @@ constexpr int kChunk = 64;          // K/V tokens per stage
 constexpr int kRows = 64;           // query rows per CTA
 constexpr int kConsumerWarps = 4;   // 16 rows each
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-
-struct PrefillParams {
-  void* out;
-  const void* query;
-  const int32_t* block_table;
-  const int32_t* seq_lens;
-  const int32_t* query_start;
-  int num_heads, num_kv_heads, block_size, max_blocks_per_seq;
-  int num_q_tokens, max_q_len;
-  int num_blocks;
-  float score_scale;  // softmax scale * log2(e)
-};
 
 template <int D, int NS>
 struct Cfg {
@@ -369,12 +358,13 @@ extern "C" int paged_attention_prefill(void* out, const void* query, const void*
                                        int num_seqs, int num_q_tokens, int max_q_len,
                                        int num_heads, int num_kv_heads, int head_dim,
                                        int block_size, int max_blocks_per_seq, int64_t num_blocks,
-                                       float scale, int q_dtype, int cache_dtype, void* stream) {
+                                       float scale, int q_dtype, int cache_dtype, unsigned flags,
+                                       void* stream) {
   using namespace pkv;
   if (num_seqs < 0 || num_q_tokens < 0 || max_q_len < 0 || num_kv_heads <= 0 ||
       num_heads <= 0 || num_heads % num_kv_heads != 0 || num_blocks <= 0 ||
       num_blocks > INT32_MAX || max_blocks_per_seq <= 0 || num_seqs > 65535 ||
-      num_kv_heads > 65535 || !(scale == scale))
+      num_kv_heads > 65535 || !(scale == scale) || (flags & ~PKV_PREFILL_MMA_SYNC))
     return PKV_ERR_SHAPE;
   if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
   if (block_size != 8 && block_size != 16 && block_size != 32) return PKV_ERR_UNSUPPORTED;
@@ -391,9 +381,12 @@ extern "C" int paged_attention_prefill(void* out, const void* query, const void*
   if (tiles > INT32_MAX) return PKV_ERR_SHAPE;
   const CUtensorMapDataType dt =
       q_dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const bool tc5 = !(flags & PKV_PREFILL_MMA_SYNC) && pf::prefill_tc5_supported(head_dim);
   CUtensorMap mk, mv;
-  if (!tcx::encode_pool_map(&mk, k_cache, dt, 2, head_dim, block_size, num_kv_heads, num_blocks) ||
-      !tcx::encode_pool_map(&mv, v_cache, dt, 2, head_dim, block_size, num_kv_heads, num_blocks))
+  if (!tcx::encode_pool_map(&mk, k_cache, dt, 2, head_dim, block_size, num_kv_heads, num_blocks,
+                            tc5) ||
+      !tcx::encode_pool_map(&mv, v_cache, dt, 2, head_dim, block_size, num_kv_heads, num_blocks,
+                            tc5))
     return PKV_ERR_CUDA;
   pf::PrefillParams p;
   p.out = out;
@@ -411,7 +404,9 @@ extern "C" int paged_attention_prefill(void* out, const void* query, const void*
   p.score_scale = scale * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (q_dtype == PKV_BF16)
+  if (tc5)
+    e = pf::launch_prefill_tc5(p, mk, mv, head_dim, q_dtype == PKV_BF16, num_seqs, st);
+  else if (q_dtype == PKV_BF16)
     e = head_dim == 128 ? pf::launch_t<__nv_bfloat16, 128>(p, mk, mv, max_q_len, num_seqs, st)
                         : pf::launch_t<__nv_bfloat16, 64>(p, mk, mv, max_q_len, num_seqs, st);
   else

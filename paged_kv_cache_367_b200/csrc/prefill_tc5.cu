@@ -1,0 +1,489 @@
+// Multi-token paged attention with a causal mask on the 5th-generation tensor
+// cores (tcgen05, accumulators in tensor memory), sm_100a.
+//
+// Same operation as prefill_tc.cu ("vLLM 0.5 深度拆解" §2.3 chunked prefill,
+// "vLLM 推理引擎源码级拆解" §4.2 prefix-cache continuation, the §2.3 block-table
+// walk): row r of a chunk of q_i query tokens sits at position seq_lens[i] - q_i
+// + r and attends over tokens 0..pos of its sequence.
+//
+// How:
+//  * A CTA owns 128 query rows — (token, query head of the group) pairs of one
+//    (sequence, KV head) — which is the M of one tcgen05.mma. Six warps: four
+//    softmax warps (warp w owns tensor-memory lanes 32w..32w+31, one row per
+//    thread), a TMA producer warp and an MMA warp (one thread issues every MMA).
+//  * The producer streams the causal range in 64-token chunks through a
+//    three-stage ring. Each (block, KV head) tile is copied as one TMA box per
+//    64-element piece of head_dim, so in shared memory a chunk's K (and V) is,
+//    per piece, 64 token rows of 128 bytes in the 128B swizzle: K is a K-major
+//    operand and V an MN-major operand of the tensor core as it lands.
+//  * S = Q K^T (M 128, N 64, K 16 per instruction) goes to one of two tensor-
+//    memory buffers, so the next chunk's S overlaps this chunk's softmax. The
+//    softmax threads load their row of S, apply the causal mask and the scale,
+//    and keep a running maximum that is only raised (and O rescaled in tensor
+//    memory) when a chunk's maximum exceeds it by more than 2^8, so rescaling is
+//    rare and P = 2^(s - m) stays below 256. P goes to shared memory in the
+//    operand layout, and O += P V (M 128, N head_dim) accumulates in tensor
+//    memory. At the end each thread reads its row of O, divides by its sum and
+//    stores it.
+//  * Slots past the causal range are masked in S and zeroed in V before the
+//    last PV, so stale or poisoned memory never reaches the output.
+//  * Every wait is bounded; on expiry the CTA records it, stops, waits (bounded)
+//    for its own copies and MMAs in flight, and frees its tensor memory.
+#include <atomic>
+#include <type_traits>
+
+#include "common.cuh"
+#include "prefill.cuh"
+#include "tc_common.cuh"
+
+namespace pkv {
+
+__device__ int g_pf5_status = 0;  // bit 0: a wait expired; bit 1: a block id outside the pool
+
+namespace pf {
+namespace {
+
+using namespace tcx;
+
+constexpr int kChunk = 64;      // K/V tokens per stage = N of S
+constexpr int kRows = 128;      // query rows per CTA = M of every MMA
+constexpr int kSoftWarps = 4;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kThreads = 6 * 32;
+constexpr int kNS = 3;          // K/V stages
+constexpr uint32_t kTmemCols = 256;  // S buffers at columns 0 and 64, O at 128..128+D
+
+template <int D>
+struct Cfg5 {
+  static constexpr int kPlanes = D / 64;          // 128-byte pieces of head_dim
+  static constexpr int kPlaneKV = kChunk * 128;   // one piece of a K (or V) chunk
+  static constexpr int kKV = kPlanes * kPlaneKV;
+  static constexpr int kStage = 2 * kKV;
+  static constexpr int kPlaneQ = kRows * 128;
+  static constexpr int kQ = kPlanes * kPlaneQ;
+  static constexpr int kP = kRows * 128;          // one P buffer: 128 rows x 64 tokens
+  static constexpr int kBars = 2 * kNS + 8;       // full, empty, s_full[2], p_full[2], o_done[2], q_full, drain
+  static constexpr int kSmem = 1024 + kNS * kStage + kQ + 2 * kP + kBars * 8 + 16;
+  static_assert(kSmem <= 227 * 1024, "shared memory per CTA exceeds 227 KB");
+};
+
+__device__ __forceinline__ bool wait5(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return mbar_wait_or_abort(bar, parity, abort, &g_pf5_status);
+}
+
+// Shared-memory matrix descriptor: 128B swizzle, 8-row groups 1024 bytes apart,
+// `lbo` between 64-element pieces (MN-major operands).
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)(1024u >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16 with an fp32 accumulator: A and B
+// bf16 (1) or f16 (0), B K-major (0) or MN-major (1), shape M x N.
+template <typename T>
+__host__ __device__ constexpr uint32_t idesc(int M, int N, bool b_mn_major) {
+  return (1u << 4) | ((std::is_same<T, __nv_bfloat16>::value ? 1u : 0u) << 7) |
+         ((std::is_same<T, __nv_bfloat16>::value ? 1u : 0u) << 10) |
+         ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id,
+                                     uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(id), "r"(accumulate)
+      : "memory");
+}
+
+// Arrives on `bar` once every MMA this thread issued so far has completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Byte offset of 16-byte chunk j of row r in a 128B-swizzled region of 128-byte rows.
+__device__ __forceinline__ uint32_t sw(int r, int j) {
+  return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4));
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_tc5_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_k,
+                       const __grid_constant__ CUtensorMap tmap_v) {
+  using C = Cfg5<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* ring = smem;                          // kNS stages: K pieces, then V pieces
+  uint8_t* qs = ring + kNS * C::kStage;          // Q pieces
+  uint8_t* ps = qs + C::kQ;                      // two P buffers
+  uint64_t* full = reinterpret_cast<uint64_t*>(ps + 2 * C::kP);
+  uint64_t* empty = full + kNS;
+  uint64_t* s_full = empty + kNS;    // [2] S of a chunk is in tensor memory
+  uint64_t* p_full = s_full + 2;     // [2] P of a chunk is in shared memory
+  uint64_t* o_done = p_full + 2;     // [2] the PV of a chunk has completed
+  uint64_t* q_full = o_done + 2;     // Q is staged
+  uint64_t* drain = q_full + 1;      // the MMA warp's last MMAs have completed
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
+
+  const int Hq = p.num_heads, g = Hq / p.num_kv_heads, bs = p.block_size;
+  const int seq = blockIdx.y, h = blockIdx.z;
+  const int q1 = min(max(__ldg(p.query_start + seq + 1), 0), p.num_q_tokens);
+  const int q0 = max(min(max(__ldg(p.query_start + seq), 0), q1), q1 - p.max_q_len);
+  const int qn = q1 - q0, rows = qn * g;
+  const int L = min(__ldg(p.seq_lens + seq), p.max_blocks_per_seq * bs);
+  const int row0 = (int)(gridDim.x - 1 - blockIdx.x) * kRows;  // longest causal ranges first
+  if (qn <= 0 || row0 >= rows || L <= 0) return;
+  const int base_pos = L - qn;
+  const int last_row = min(rows, row0 + kRows) - 1;
+  const int kv_end = min(L, base_pos + last_row / g + 1);
+  if (kv_end <= 0) return;
+  const int nchunks = (kv_end + kChunk - 1) / kChunk;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kNS; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(s_full + b, 1);
+      mbar_init(p_full + b, kSoftWarps * 32);
+      mbar_init(o_done + b, 1);
+    }
+    mbar_init(q_full, kSoftWarps * 32);
+    mbar_init(drain, 1);
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tslot)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer ----
+    const int32_t* bt = p.block_table + (int64_t)seq * p.max_blocks_per_seq;
+    const int piece = bs * 128;  // bytes of one (block, piece of head_dim) box
+    uint32_t armed = 0, last_parity = 0;
+    bool ok = true;
+    for (int c = 0; c < nchunks && ok; ++c) {
+      const int stage = c % kNS;
+      const uint32_t phase = (uint32_t)(c / kNS) & 1u;
+      const int c0 = c * kChunk;
+      const int nblk = (min(kChunk, kv_end - c0) + bs - 1) / bs;
+      const int blk = lane < nblk ? __ldg(bt + c0 / bs + lane) : 0;
+      if (lane == 0) ok = wait5(empty + stage, phase ^ 1u, abort);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      uint8_t* st = ring + stage * C::kStage;
+      if (lane == 0) mbar_expect_tx(full + stage, (uint32_t)(2 * C::kPlanes * nblk * piece));
+      __syncwarp();
+      if (lane < nblk) {
+        if ((unsigned)blk >= (unsigned)p.num_blocks) atomicOr(&g_pf5_status, 2);  // reads as zeros
+#pragma unroll
+        for (int pc = 0; pc < C::kPlanes; ++pc) {
+          tma_load_5d(st + pc * C::kPlaneKV + lane * piece, &tmap_k, 0, 0, pc, h, blk, full + stage);
+          tma_load_5d(st + C::kKV + pc * C::kPlaneKV + lane * piece, &tmap_v, 0, 0, pc, h, blk,
+                      full + stage);
+        }
+      }
+      armed |= 1u << stage;
+      last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+    }
+    if (!ok && lane == 0) {  // wait, bounded, for this CTA's copies in flight
+      for (int s = 0; s < kNS; ++s) {
+        if (!(armed >> s & 1u)) continue;
+        const long long t0 = clock64();
+        while (!mbar_try(full + s, (last_parity >> s) & 1u))
+          if (clock64() - t0 > kWaitCycles) break;
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ----------------------------------------------------------------- MMA ----
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc<T>(kRows, kChunk, false);
+      constexpr uint32_t idO = idesc<T>(kRows, D, true);
+      const uint32_t q_addr = smem_u32(qs), p_addr = smem_u32(ps), r_addr = smem_u32(ring);
+      bool ok = wait5(q_full, 0, abort);
+      tc_fence_after();
+      // O += P V for chunk c (its P in buffer c & 1, its V in stage c % kNS).
+      auto issue_pv = [&](int c) -> bool {
+        if (!wait5(p_full + (c & 1), (uint32_t)(c >> 1) & 1u, abort)) return false;
+        tc_fence_after();
+        const uint32_t v = r_addr + (c % kNS) * C::kStage + C::kKV;
+        const uint32_t pa = p_addr + (c & 1) * C::kP;
+#pragma unroll
+        for (int s = 0; s < kChunk / 16; ++s)
+          umma(tmem + 128, sdesc(pa + s * 32, 16), sdesc(v + s * 16 * 128, C::kPlaneKV), idO,
+               (c > 0 || s > 0) ? 1u : 0u);
+        umma_commit(o_done + (c & 1));
+        umma_commit(empty + c % kNS);
+        return true;
+      };
+      for (int c = 0; c < nchunks && ok; ++c) {
+        const int stage = c % kNS;
+        ok = wait5(full + stage, (uint32_t)(c / kNS) & 1u, abort);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t k = r_addr + stage * C::kStage;
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s) {
+          const int pc = s / 4, off = (s % 4) * 32;
+          umma(tmem + 64 * (c & 1), sdesc(q_addr + pc * C::kPlaneQ + off, 16),
+               sdesc(k + pc * C::kPlaneKV + off, 16), idS, s > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full + (c & 1));
+        if (c > 0) ok = issue_pv(c - 1);
+      }
+      if (ok) issue_pv(nchunks - 1);
+      // Whatever happened, wait (bounded) until every MMA issued has completed.
+      umma_commit(drain);
+      const long long t0 = clock64();
+      while (!mbar_try(drain, 0))
+        if (clock64() - t0 > kWaitCycles) break;
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------- softmax ----
+    const int r = 32 * warp + lane;       // this thread's tensor-memory lane and tile row
+    const int R = row0 + r;
+    const bool valid = R < rows;
+    const int tok = valid ? R / g : 0, j = valid ? R - tok * g : 0;
+    const int pos = valid ? base_pos + tok : -1;
+    const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
+    // Stage this row of Q (zeros past the chunk) in the operand layout.
+    {
+      const uint4* src = reinterpret_cast<const uint4*>(
+          static_cast<const T*>(p.query) + ((int64_t)(q0 + tok) * Hq + h * g + j) * D);
+#pragma unroll
+      for (int u = 0; u < D / 8; ++u) {
+        const uint4 v = valid ? __ldg(src + u) : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(qs + (u >> 3) * C::kPlaneQ + sw(r, u & 7)) = v;
+      }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_arrive(q_full);
+    const float sscale = p.score_scale;
+    float m_use = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int c = 0; c < nchunks; ++c) {
+      ok = wait5(s_full + (c & 1), (uint32_t)(c >> 1) & 1u, abort);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[64];
+      {
+        float a[32];
+        tmem_ld32(trow + 64 * (c & 1), a);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[i] = a[i];
+        tmem_ld32(trow + 64 * (c & 1) + 32, a);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[32 + i] = a[i];
+      }
+      const int c0 = c * kChunk;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        s[i] = c0 + i <= pos ? s[i] * sscale : -INFINITY;
+        mx = fmaxf(mx, s[i]);
+      }
+      // Raise the running maximum only when this chunk exceeds it by 2^8.
+      const bool raise = mx > m_use + 8.f;
+      const bool rescale = raise && m_use != -INFINITY;
+      if (__any_sync(0xffffffffu, rescale)) {
+        if (c > 0) {  // the last PV must have landed in O
+          ok = wait5(o_done + ((c - 1) & 1), (uint32_t)((c - 1) >> 1) & 1u, abort);
+          if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        const float alpha = rescale ? fast_exp2(m_use - mx) : 1.f;
+#pragma unroll
+        for (int q = 0; q < D / 32; ++q) {
+          float o[32];
+          tmem_ld32(trow + 128 + 32 * q, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(trow + 128 + 32 * q, o);
+        }
+        l *= alpha;
+      }
+      if (raise) m_use = mx;
+      const float msub = m_use == -INFINITY ? 0.f : m_use;
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        float lo, hi;
+        pk[i] = Mma<T>::pack(fast_exp2(s[2 * i] - msub), fast_exp2(s[2 * i + 1] - msub), lo, hi);
+        l += lo + hi;
+      }
+      if (c >= 2) {  // the PV that read this P buffer (chunk c - 2) has completed
+        ok = wait5(o_done + (c & 1), (uint32_t)((c - 2) >> 1) & 1u, abort);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+      }
+      if (c == nchunks - 1 && c0 + kChunk > kv_end) {
+        // Zero V rows past the range (stale or poisoned) before the last PV.
+        uint8_t* v = ring + (c % kNS) * C::kStage + C::kKV;
+        const int t0 = kv_end - c0, per_row = 8 * C::kPlanes;
+        for (int e = r; e < (kChunk - t0) * per_row; e += kSoftWarps * 32) {
+          const int t = t0 + e / per_row, u = e % per_row;
+          *reinterpret_cast<uint4*>(v + (u >> 3) * C::kPlaneKV + t * 128 + (u & 7) * 16) =
+              make_uint4(0, 0, 0, 0);
+        }
+      }
+      uint8_t* prow = ps + (c & 1) * C::kP;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        *reinterpret_cast<uint4*>(prow + sw(r, u)) =
+            make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive(p_full + (c & 1));
+    }
+    if (ok) {
+      ok = wait5(o_done + ((nchunks - 1) & 1), (uint32_t)((nchunks - 1) >> 1) & 1u, abort);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      T* dst = static_cast<T*>(p.out) + ((int64_t)(q0 + tok) * Hq + h * g + j) * D;
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) {
+        float o[32];
+        tmem_ld32(trow + 128 + 32 * q, o);
+        if (valid) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 w;
+            float a, b;
+            w.x = Mma<T>::pack(o[8 * u + 0] * inv, o[8 * u + 1] * inv, a, b);
+            w.y = Mma<T>::pack(o[8 * u + 2] * inv, o[8 * u + 3] * inv, a, b);
+            w.z = Mma<T>::pack(o[8 * u + 4] * inv, o[8 * u + 5] * inv, a, b);
+            w.w = Mma<T>::pack(o[8 * u + 6] * inv, o[8 * u + 7] * inv, a, b);
+            *reinterpret_cast<uint4*>(dst + 32 * q + 8 * u) = w;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols));
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch5(const PrefillParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
+                    int num_seqs, cudaStream_t stream) {
+  using C = Cfg5<D>;
+  auto kernel = prefill_tc5_kernel<T, D>;
+  static std::atomic<int> opted_in[64];  // the shared-memory opt-in, once per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!opted_in[dev].load(std::memory_order_relaxed)) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (e != cudaSuccess) return e;
+    opted_in[dev].store(1, std::memory_order_relaxed);
+  }
+  const int g = p.num_heads / p.num_kv_heads;
+  const int64_t tiles = ((int64_t)p.max_q_len * g + kRows - 1) / kRows;
+  dim3 grid((unsigned)tiles, (unsigned)num_seqs, (unsigned)p.num_kv_heads);
+  kernel<<<grid, kThreads, C::kSmem, stream>>>(p, mk, mv);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool prefill_tc5_supported(int head_dim) { return head_dim == 64 || head_dim == 128; }
+
+cudaError_t launch_prefill_tc5(const PrefillParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
+                               int head_dim, bool bf16, int num_seqs, cudaStream_t stream) {
+  if (bf16)
+    return head_dim == 128 ? launch5<__nv_bfloat16, 128>(p, mk, mv, num_seqs, stream)
+                           : launch5<__nv_bfloat16, 64>(p, mk, mv, num_seqs, stream);
+  return head_dim == 128 ? launch5<__half, 128>(p, mk, mv, num_seqs, stream)
+                         : launch5<__half, 64>(p, mk, mv, num_seqs, stream);
+}
+
+}  // namespace pf
+
+int pf5_status_flag(bool clear, int* value) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_pf5_status, sizeof(int)) != cudaSuccess) return -1;
+  if (clear && v) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_pf5_status, &zero, sizeof(int)) != cudaSuccess) return -1;
+  }
+  *value = v;
+  return 0;
+}
+
+}  // namespace pkv

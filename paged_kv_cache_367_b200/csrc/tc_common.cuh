@@ -170,24 +170,23 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // 5-D view of a [num_blocks, bs, Hkv, D] pool of e-byte elements: (d_lo 128/e,
 // token bs, d_hi D*e/128, head Hkv, block num_blocks); one box is a whole
 // (block, head) tile, landing as 128-byte rows with the 128B swizzle.
+// per_plane: the box covers one 128-byte piece of head_dim (d_hi extent 1)
+// instead of all of them, for copies that place each piece in its own region.
 inline bool encode_pool_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int e,
-                            int D, int bs, int Hkv, int64_t nb) {
+                            int D, int bs, int Hkv, int64_t nb, bool per_plane = false) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   const cuuint64_t row = 128 / e;  // elements per 128-byte row
   cuuint64_t dims[5] = {row, (cuuint64_t)bs, (cuuint64_t)(D / row), (cuuint64_t)Hkv, (cuuint64_t)nb};
   cuuint64_t strides[4] = {(cuuint64_t)Hkv * D * e, 128, (cuuint64_t)D * e,
                            (cuuint64_t)bs * Hkv * D * e};
-  cuuint32_t box[5] = {(cuuint32_t)row, (cuuint32_t)bs, (cuuint32_t)(D / row), 1, 1};
+  cuuint32_t box[5] = {(cuuint32_t)row, (cuuint32_t)bs, per_plane ? 1u : (cuuint32_t)(D / row), 1, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = enc(map, dt, 5, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
-
-// Returns the timeout word of the tensor-core kernel (1 if any bounded wait
-// expired), optionally clearing it. Synchronises the device.
 
 }  // namespace tcx
 }  // namespace pkv

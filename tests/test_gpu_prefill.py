@@ -45,7 +45,7 @@ def make_case(lens, qlens, Hq, Hkv, D, bs, dt, dev, seed=0, spare=5):
                 q=q.to(dev), Hq=Hq, Hkv=Hkv, D=D, bs=bs, dt=dt, dev=dev)
 
 
-def run_gpu(c, max_q_len=None, bt=None, fill=float("nan"), status=0):
+def run_gpu(c, max_q_len=None, bt=None, fill=float("nan"), status=0, flags=0):
     dev = c["dev"]
     out = torch.full(tuple(c["q"].shape), fill, dtype=c["q"].dtype, device=dev)
     bt = c["bt"] if bt is None else bt
@@ -53,7 +53,7 @@ def run_gpu(c, max_q_len=None, bt=None, fill=float("nan"), status=0):
     pkv.paged_attention_prefill(out, c["q"], c["kc"], c["vc"], torch.from_numpy(bt).to(dev),
                                 torch.from_numpy(c["lens"]).to(dev),
                                 torch.from_numpy(c["qs"]).to(dev), max_q_len=mq,
-                                scale=c["D"] ** -0.5)
+                                scale=c["D"] ** -0.5, flags=flags)
     torch.cuda.synchronize()
     assert pkv.pkv_device_status(clear=True) == status
     return out
@@ -84,25 +84,54 @@ CASES = {
 }
 
 
+KERNELS = [0, pkv.PKV_PREFILL_MMA_SYNC]  # tcgen05 (default), mma.sync
+
+
 @pytest.mark.parametrize("case", list(CASES))
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (32, 8), (16, 1), (12, 2), (6, 2), (64, 4)])
-def test_prefill_parity_group_sizes(cuda_dev, case, Hq, Hkv):
+@pytest.mark.parametrize("flags", KERNELS)
+def test_prefill_parity_group_sizes(cuda_dev, case, Hq, Hkv, flags):
     lens, qlens = CASES[case]
     c = make_case(lens, qlens, Hq, Hkv, 128, 16, "bf16", cuda_dev, seed=Hq + Hkv)
-    check(run_gpu(c), run_oracle(c), "bf16")
+    check(run_gpu(c, flags=flags), run_oracle(c), "bf16")
 
 
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("bs", [8, 16, 32])
 @pytest.mark.parametrize("dt", ["bf16", "f16"])
-def test_prefill_parity_dims_blocks_dtypes(cuda_dev, D, bs, dt):
+@pytest.mark.parametrize("flags", KERNELS)
+def test_prefill_parity_dims_blocks_dtypes(cuda_dev, D, bs, dt, flags):
     c = make_case([400, 90, 33], [200, 90, 5], 16, 4, D, bs, dt, cuda_dev, seed=D + bs)
-    check(run_gpu(c), run_oracle(c), dt)
+    check(run_gpu(c, flags=flags), run_oracle(c), dt)
 
 
-def test_prefill_long_chunk_many_tiles(cuda_dev):
+def test_prefill_large_score_range_forces_rescaling(cuda_dev):
+    # Keys aligned with the queries and growing along the sequence give scores
+    # whose running maximum rises by more than 2^8 several times (the tcgen05
+    # kernel then rescales O in tensor memory). Both kernels must meet the
+    # tolerance and agree with each other to within the rounding of P.
+    c = make_case([700, 300], [700, 40], 8, 2, 128, 16, "bf16", cuda_dev, seed=31)
+    L = 700
+    ramp = torch.linspace(0.2, 3.0, L).to(torch.bfloat16)
+    q = c["q"].float()
+    kc, bt = c["kc"].float(), c["bt"]
+    for t in range(L):  # sequence 0: key t = the mean of its position's query group, scaled
+        kc[bt[0, t // 16], t % 16] = q[t].view(2, 4, 128).mean(1) * ramp[t]
+    c["kc"] = kc.to(torch.bfloat16)
+    want = run_oracle(c)
+    tc5 = run_gpu(c)
+    mma = run_gpu(c, flags=pkv.PKV_PREFILL_MMA_SYNC)
+    check(tc5, want, "bf16")
+    check(mma, want, "bf16")
+    # (outputs are rounded to bf16 once: allow a unit or two in the last place)
+    a, b = tc5.float(), mma.float()
+    assert torch.all((a - b).abs() <= 2 ** -7 * b.abs() + 2e-3)
+
+
+@pytest.mark.parametrize("flags", KERNELS)
+def test_prefill_long_chunk_many_tiles(cuda_dev, flags):
     c = make_case([3000, 2100], [1024, 2100], 32, 8, 128, 16, "bf16", cuda_dev, seed=9)
-    got = run_gpu(c)
+    got = run_gpu(c, flags=flags)
     # Sampled rows (the oracle is slow at this size): every 37th row and the last ones.
     T = int(c["qs"][-1])
     rows = np.unique(np.concatenate([np.arange(0, T, 37), np.arange(T - 5, T)]))
@@ -140,19 +169,21 @@ def test_chunk_longer_than_max_q_len_computes_its_last_rows(cuda_dev):
     assert torch.all(got[torch.from_numpy(skipped).to(cuda_dev)] == 0)
 
 
-def test_chunk_longer_than_its_context_gives_zero_rows(cuda_dev):
+@pytest.mark.parametrize("flags", KERNELS)
+def test_chunk_longer_than_its_context_gives_zero_rows(cuda_dev, flags):
     # 10 query tokens over a 6-token context: the first 4 sit before position 0.
     c = make_case([6, 40], [10, 8], 8, 8, 64, 8, "bf16", cuda_dev, seed=2)
-    got = run_gpu(c)
+    got = run_gpu(c, flags=flags)
     want = run_oracle(c)
     assert np.all(want[:4] == 0)
     check(got, want, "bf16")
 
 
-def test_block_ids_outside_the_pool_read_as_zeros(cuda_dev):
+@pytest.mark.parametrize("flags", KERNELS)
+def test_block_ids_outside_the_pool_read_as_zeros(cuda_dev, flags):
     c = make_case([70, 33], [20, 33], 16, 4, 128, 16, "bf16", cuda_dev, seed=6)
     bt = c["bt"].copy()
     nb = c["kc"].shape[0]
     bt[0, 1] = nb + 7
     bt[1, 0] = -3
-    check(run_gpu(c, bt=bt, status=2), run_oracle(c, bt=bt), "bf16")  # reported, read as zeros
+    check(run_gpu(c, bt=bt, status=2, flags=flags), run_oracle(c, bt=bt), "bf16")  # reported
