@@ -18,8 +18,8 @@
 //    operand and V an MN-major operand of the tensor core as it lands.
 //  * S = Q K^T (M 128, N 64, K 16 per instruction) goes to one of two tensor-
 //    memory buffers, so the next chunk's S overlaps this chunk's softmax. The
-//    softmax threads load their row of S, apply the causal mask and the scale,
-//    and keep a running maximum that is only raised (and O rescaled in tensor
+//    softmax threads load their row of S, apply the causal mask (only in chunks
+//    that reach past a row's position) and the scale, and keep a running maximum that is only raised (and O rescaled in tensor
 //    memory) when a chunk's maximum exceeds it by more than 2^8, so rescaling is
 //    rare and P = 2^(s - m) stays below 256. P goes to shared memory in the
 //    operand layout, and O += P V (M 128, N head_dim) accumulates in tensor
@@ -339,12 +339,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 32; ++i) s[32 + i] = a[i];
       }
       const int c0 = c * kChunk;
+      // Raw scores; the causal mask only where the chunk reaches past a row's
+      // position. The scale is applied with the exponent (it is positive, so the
+      // maximum of the raw scores gives the maximum of the scaled ones).
       float mx = -INFINITY;
+      if (__any_sync(0xffffffffu, c0 + kChunk - 1 > pos)) {
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        s[i] = c0 + i <= pos ? s[i] * sscale : -INFINITY;
-        mx = fmaxf(mx, s[i]);
+        for (int i = 0; i < 64; ++i) {
+          s[i] = c0 + i <= pos ? s[i] : -INFINITY;
+          mx = fmaxf(mx, s[i]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) mx = fmaxf(mx, s[i]);
       }
+      mx *= sscale;
       // Raise the running maximum only when this chunk exceeds it by 2^8.
       const bool raise = mx > m_use + 8.f;
       const bool rescale = raise && m_use != -INFINITY;
@@ -373,8 +382,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        float lo, hi;
-        pk[i] = Mma<T>::pack(fast_exp2(s[2 * i] - msub), fast_exp2(s[2 * i + 1] - msub), lo, hi);
+        const float p0 = fast_exp2(fmaf(s[2 * i], sscale, -msub));
+        const float p1 = fast_exp2(fmaf(s[2 * i + 1], sscale, -msub));
+        float lo, hi;  // the rounded values enter the sum, as the MMA sees them
+        pk[i] = Mma<T>::pack(p0, p1, lo, hi);
         l += lo + hi;
       }
       if (c >= 2) {  // the PV that read this P buffer (chunk c - 2) has completed
