@@ -22,9 +22,11 @@
 //    that reach past a row's position) and the scale, and keep a running maximum that is only raised (and O rescaled in tensor
 //    memory) when a chunk's maximum exceeds it by more than 2^8, so rescaling is
 //    rare and P = 2^(s - m) stays below 256. P goes to shared memory in the
-//    operand layout, and O += P V (M 128, N head_dim) accumulates in tensor
-//    memory. At the end each thread reads its row of O, divides by its sum and
-//    stores it.
+//    operand layout, and O += P [V | 1] (M 128, N head_dim + 16) accumulates
+//    in tensor memory: the extra operand piece holds a column of ones, so the
+//    row sums of the rounded P come out of the tensor core beside O, rescaled
+//    with it. At the end each thread reads its row of O and its sum, divides
+//    and stores it.
 //  * Slots past the causal range are masked in S and zeroed in V before the
 //    last PV, so stale or poisoned memory never reaches the output.
 //  * Every wait is bounded; on expiry the CTA records it, stops, waits (bounded)
@@ -52,14 +54,17 @@ constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kThreads = 6 * 32;
 constexpr int kNS = 3;          // K/V stages
-constexpr uint32_t kTmemCols = 256;  // S buffers at columns 0 and 64, O at 128..128+D
+constexpr uint32_t kTmemCols = 512;  // S buffers at columns 0 and 64; O at 128..128+D, and
+                                     // the row sums at column 128+D (the ones column of V)
 
 template <int D>
 struct Cfg5 {
   static constexpr int kPlanes = D / 64;          // 128-byte pieces of head_dim
   static constexpr int kPlaneKV = kChunk * 128;   // one piece of a K (or V) chunk
   static constexpr int kKV = kPlanes * kPlaneKV;
-  static constexpr int kStage = 2 * kKV;
+  // K pieces, V pieces, then one more V piece whose first column is 1 and the
+  // rest 0: O += P [V | 1] yields the row sums of P in the column after O.
+  static constexpr int kStage = 2 * kKV + kPlaneKV;
   static constexpr int kPlaneQ = kRows * 128;
   static constexpr int kQ = kPlanes * kPlaneQ;
   static constexpr int kP = kRows * 128;          // one P buffer: 128 rows x 64 tokens
@@ -257,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ----------------------------------------------------------------- MMA ----
     if (lane == 0) {
       constexpr uint32_t idS = idesc<T>(kRows, kChunk, false);
-      constexpr uint32_t idO = idesc<T>(kRows, D, true);
+      constexpr uint32_t idO = idesc<T>(kRows, D + 16, true);  // O and the row sums
       const uint32_t q_addr = smem_u32(qs), p_addr = smem_u32(ps), r_addr = smem_u32(ring);
       bool ok = wait5(q_full, 0, abort);
       tc_fence_after();
@@ -316,10 +321,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<uint4*>(qs + (u >> 3) * C::kPlaneQ + sw(r, u & 7)) = v;
       }
     }
+    // The ones piece of every stage (written once; the copies never touch it).
+    for (int e = r; e < kNS * kChunk * 8; e += kSoftWarps * 32) {
+      const int st = e / (kChunk * 8), t = (e / 8) % kChunk, u = e % 8;
+      const uint16_t one = std::is_same<T, __nv_bfloat16>::value ? 0x3F80u : 0x3C00u;
+      const uint32_t w0 = (u == (t & 7)) ? (uint32_t)one : 0u;  // element 0 of the row
+      *reinterpret_cast<uint4*>(ring + st * C::kStage + 2 * C::kKV + t * 128 + u * 16) =
+          make_uint4(w0, 0u, 0u, 0u);
+    }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     mbar_arrive(q_full);
     const float sscale = p.score_scale;
-    float m_use = -INFINITY, l = 0.f;
+    float m_use = -INFINITY;
     bool ok = true;
     for (int c = 0; c < nchunks; ++c) {
       ok = wait5(s_full + (c & 1), (uint32_t)(c >> 1) & 1u, abort);
@@ -368,14 +381,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float alpha = rescale ? fast_exp2(m_use - mx) : 1.f;
 #pragma unroll
-        for (int q = 0; q < D / 32; ++q) {
+        for (int q = 0; q <= D / 32; ++q) {  // O and, in the last group, the row sums
           float o[32];
           tmem_ld32(trow + 128 + 32 * q, o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] *= alpha;
           tmem_st32(trow + 128 + 32 * q, o);
         }
-        l *= alpha;
       }
       if (raise) m_use = mx;
       const float msub = m_use == -INFINITY ? 0.f : m_use;
@@ -384,9 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < 32; ++i) {
         const float p0 = fast_exp2(fmaf(s[2 * i], sscale, -msub));
         const float p1 = fast_exp2(fmaf(s[2 * i + 1], sscale, -msub));
-        float lo, hi;  // the rounded values enter the sum, as the MMA sees them
+        float lo, hi;  // (the row sums come from the tensor core, of the rounded P)
         pk[i] = Mma<T>::pack(p0, p1, lo, hi);
-        l += lo + hi;
       }
       if (c >= 2) {  // the PV that read this P buffer (chunk c - 2) has completed
         ok = wait5(o_done + (c & 1), (uint32_t)((c - 2) >> 1) & 1u, abort);
@@ -420,7 +431,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) {
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      float ls[32];
+      tmem_ld32(trow + 128 + D, ls);  // column 128 + D: the row sum of P
+      const float inv = ls[0] > 0.f ? 1.f / ls[0] : 0.f;
       T* dst = static_cast<T*>(p.out) + ((int64_t)(q0 + tok) * Hq + h * g + j) * D;
 #pragma unroll
       for (int q = 0; q < D / 32; ++q) {
