@@ -394,8 +394,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float p0 = fast_exp2(fmaf(s[2 * i], sscale, -msub));
-        const float p1 = fast_exp2(fmaf(s[2 * i + 1], sscale, -msub));
+        float x0, x1;  // s * scale - m for a pair, as one packed f32x2 FMA
+        {
+          uint64_t xy, sc, mm, rr;
+          asm("mov.b64 %0, {%1, %2};" : "=l"(xy) : "f"(s[2 * i]), "f"(s[2 * i + 1]));
+          asm("mov.b64 %0, {%1, %1};" : "=l"(sc) : "f"(sscale));
+          asm("mov.b64 %0, {%1, %1};" : "=l"(mm) : "f"(-msub));
+          asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rr) : "l"(xy), "l"(sc), "l"(mm));
+          asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(rr));
+        }
+        const float p0 = fast_exp2(x0);
+        const float p1 = fast_exp2(x1);
         float lo, hi;  // (the row sums come from the tensor core, of the rounded P)
         pk[i] = Mma<T>::pack(p0, p1, lo, hi);
       }
