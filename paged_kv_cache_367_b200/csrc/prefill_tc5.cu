@@ -7,26 +7,30 @@
 // + r and attends over tokens 0..pos of its sequence.
 //
 // How:
-//  * A CTA owns 128 query rows — (token, query head of the group) pairs of one
-//    (sequence, KV head) — which is the M of one tcgen05.mma. Six warps: four
-//    softmax warps (warp w owns tensor-memory lanes 32w..32w+31, one row per
-//    thread), a TMA producer warp and an MMA warp (one thread issues every MMA).
+//  * A CTA owns 256 query rows — (token, query head of the group) pairs of one
+//    (sequence, KV head) — as two tiles of 128, each the M of one tcgen05.mma.
+//    Ten warps: eight softmax warps (warp w serves tile w / 4 and owns tensor-
+//    memory lanes 32 (w % 4) .. +31, one row per thread), a TMA producer warp
+//    and an MMA warp (one thread issues every MMA).
 //  * The producer streams the causal range in 64-token chunks through a
-//    three-stage ring. Each (block, KV head) tile is copied as one TMA box per
-//    64-element piece of head_dim, so in shared memory a chunk's K (and V) is,
-//    per piece, 64 token rows of 128 bytes in the 128B swizzle: K is a K-major
-//    operand and V an MN-major operand of the tensor core as it lands.
-//  * S = Q K^T (M 128, N 64, K 16 per instruction) goes to one of two tensor-
-//    memory buffers, so the next chunk's S overlaps this chunk's softmax. The
-//    softmax threads load their row of S, apply the causal mask (only in chunks
-//    that reach past a row's position) and the scale, and keep a running maximum that is only raised (and O rescaled in tensor
-//    memory) when a chunk's maximum exceeds it by more than 2^8, so rescaling is
-//    rare and P = 2^(s - m) stays below 256. P goes to shared memory in the
-//    operand layout, and O += P [V | 1] (M 128, N head_dim + 16) accumulates
-//    in tensor memory: the extra operand piece holds a column of ones, so the
-//    row sums of the rounded P come out of the tensor core beside O, rescaled
-//    with it. At the end each thread reads its row of O and its sum, divides
-//    and stores it.
+//    three-stage ring shared by both tiles. Each (block, KV head) tile is
+//    copied as one TMA box per 64-element piece of head_dim, so in shared
+//    memory a chunk's K (and V) is, per piece, 64 token rows of 128 bytes in
+//    the 128B swizzle: K is a K-major operand and V an MN-major operand of the
+//    tensor core as it lands.
+//  * S = Q K^T of a tile (M 128, N 64, K 16 per instruction) lands in the
+//    tile's S columns of tensor memory; the MMA warp issues the next chunk's S
+//    as soon as the softmax threads have read this one, so it overlaps their
+//    softmax. They apply the causal mask (only in chunks that reach past a
+//    row's position) and the scale, and keep a running maximum that is only
+//    raised (and O rescaled in tensor memory) when a chunk's maximum exceeds it
+//    by more than 2^8, so rescaling is rare and P = 2^(s - m) stays below 256.
+//  * P goes back to tensor memory as 16-bit pairs, and O += P [V | 1] (A from
+//    tensor memory, M 128, N head_dim + 16) accumulates in the tile's O
+//    columns: the extra operand piece holds a column of ones, so the row sums
+//    of the rounded P come out of the tensor core beside O, rescaled with it.
+//    At the end each thread reads its row of O and its sum, divides and
+//    stores it.
 //  * Slots past the causal range are masked in S and zeroed in V before the
 //    last PV, so stale or poisoned memory never reaches the output.
 //  * Every wait is bounded; on expiry the CTA records it, stops, waits (bounded)
@@ -48,14 +52,34 @@ namespace {
 using namespace tcx;
 
 constexpr int kChunk = 64;      // K/V tokens per stage = N of S
-constexpr int kRows = 128;      // query rows per CTA = M of every MMA
-constexpr int kSoftWarps = 4;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kThreads = 6 * 32;
+constexpr int kRows = 128;      // query rows per tile = M of every MMA
+constexpr int kTiles = 2;       // tiles per CTA, sharing each K/V chunk
+constexpr int kCtaRows = kTiles * kRows;
+constexpr int kSoftWarps = 4 * kTiles;
+constexpr int kProducerWarp = kSoftWarps;
+constexpr int kMmaWarp = kSoftWarps + 1;
+constexpr int kThreads = (kSoftWarps + 2) * 32;
 constexpr int kNS = 3;          // K/V stages
-constexpr uint32_t kTmemCols = 512;  // S buffers at columns 0 and 64; O at 128..128+D, and
-                                     // the row sums at column 128+D (the ones column of V)
+constexpr uint32_t kTmemCols = 512;
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Maximum of 64 values as a tree of three-input maxima (depth 4, 32 ops)
+// instead of a chain of 63 dependent two-input ones.
+__device__ __forceinline__ float max64(const float (&s)[64]) {
+  float t[22], u[8];
+#pragma unroll
+  for (int i = 0; i < 21; ++i) t[i] = max3f(s[3 * i], s[3 * i + 1], s[3 * i + 2]);
+  t[21] = s[63];
+#pragma unroll
+  for (int i = 0; i < 7; ++i) u[i] = max3f(t[3 * i], t[3 * i + 1], t[3 * i + 2]);
+  u[7] = t[21];
+  return max3f(max3f(u[0], u[1], u[2]), max3f(u[3], u[4], u[5]), fmaxf(u[6], u[7]));
+}
 
 template <int D>
 struct Cfg5 {
@@ -66,10 +90,14 @@ struct Cfg5 {
   // rest 0: O += P [V | 1] yields the row sums of P in the column after O.
   static constexpr int kStage = 2 * kKV + kPlaneKV;
   static constexpr int kPlaneQ = kRows * 128;
-  static constexpr int kQ = kPlanes * kPlaneQ;
-  static constexpr int kP = kRows * 128;          // one P buffer: 128 rows x 64 tokens
-  static constexpr int kBars = 2 * kNS + 8;       // full, empty, s_full[2], p_full[2], o_done[2], q_full, drain
-  static constexpr int kSmem = 1024 + kNS * kStage + kQ + 2 * kP + kBars * 8 + 16;
+  static constexpr int kQ = kPlanes * kPlaneQ;    // Q of one tile
+  // Tensor-memory columns: S of tile t at 64 t, P of tile t (bf16 pairs, 32
+  // columns) at 128 + 32 t, O of tile t at 192 + t (D + 32): D columns of O,
+  // the row sum, and padding to a whole group of 32.
+  static constexpr uint32_t kColP = 128, kColO = 192, kOCols = D + 32;
+  static_assert(kColO + kTiles * kOCols <= kTmemCols, "tensor memory per CTA");
+  static constexpr int kBars = 2 * kNS + 4 * kTiles + 2;  // full, empty, s_full, s_free, p_full, o_done, q_full, drain
+  static constexpr int kSmem = 1024 + kNS * kStage + kTiles * kQ + kBars * 8 + 16;
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA exceeds 227 KB");
 };
 
@@ -85,7 +113,7 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo) {
 }
 
 // Instruction descriptor of kind::f16 with an fp32 accumulator: A and B
-// bf16 (1) or f16 (0), B K-major (0) or MN-major (1), shape M x N.
+// bf16 (1) or f16 (0), A K-major, B K-major (0) or MN-major (1), shape M x N.
 template <typename T>
 __host__ __device__ constexpr uint32_t idesc(int M, int N, bool b_mn_major) {
   return (1u << 4) | ((std::is_same<T, __nv_bfloat16>::value ? 1u : 0u) << 7) |
@@ -93,12 +121,24 @@ __host__ __device__ constexpr uint32_t idesc(int M, int N, bool b_mn_major) {
          ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// D (tensor memory) [+]= A (shared memory) x B (shared memory).
 __device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id,
                                      uint32_t accumulate) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(id), "r"(accumulate)
+      : "memory");
+}
+
+// D (tensor memory) [+]= A (tensor memory: row i in lane i, K packed two
+// elements per column) x B (shared memory).
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t id,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(id), "r"(accumulate)
       : "memory");
 }
 
@@ -116,40 +156,56 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+#define PKV_TMEM_REGS32(r)                                                                   \
+  "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),     \
+      "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), \
+      "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),          \
+      "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),          \
+      "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+#define PKV_TMEM_LD32 \
+  "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14," \
+  "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+
 // 32 consecutive fp32 columns of this thread's tensor-memory lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
+  asm volatile(PKV_TMEM_LD32 : PKV_TMEM_REGS32(r) : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+// 64 consecutive fp32 columns: two loads in flight, one wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t a[32], b[32];
+  asm volatile(PKV_TMEM_LD32 : PKV_TMEM_REGS32(a) : "r"(taddr));
+  asm volatile(PKV_TMEM_LD32 : PKV_TMEM_REGS32(b) : "r"(taddr + 32));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    v[i] = __uint_as_float(a[i]);
+    v[32 + i] = __uint_as_float(b[i]);
+  }
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
       "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
-      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
-      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
-      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
-      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
-      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  uint32_t u[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(v[i]);
+  tmem_st32(taddr, u);
 }
 
 // Byte offset of 16-byte chunk j of row r in a 128B-swizzled region of 128-byte rows.
@@ -165,16 +221,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* ring = smem;                          // kNS stages: K pieces, then V pieces
-  uint8_t* qs = ring + kNS * C::kStage;          // Q pieces
-  uint8_t* ps = qs + C::kQ;                      // two P buffers
-  uint64_t* full = reinterpret_cast<uint64_t*>(ps + 2 * C::kP);
+  uint8_t* ring = smem;                          // kNS stages: K pieces, V pieces, ones piece
+  uint8_t* qs = ring + kNS * C::kStage;          // Q pieces of tile 0, then of tile 1
+  uint64_t* full = reinterpret_cast<uint64_t*>(qs + kTiles * C::kQ);
   uint64_t* empty = full + kNS;
-  uint64_t* s_full = empty + kNS;    // [2] S of a chunk is in tensor memory
-  uint64_t* p_full = s_full + 2;     // [2] P of a chunk is in shared memory
-  uint64_t* o_done = p_full + 2;     // [2] the PV of a chunk has completed
-  uint64_t* q_full = o_done + 2;     // Q is staged
-  uint64_t* drain = q_full + 1;      // the MMA warp's last MMAs have completed
+  uint64_t* s_full = empty + kNS;       // [tile] S of the tile's chunk is in tensor memory
+  uint64_t* s_free = s_full + kTiles;   // [tile] the tile's softmax warps have read S
+  uint64_t* p_full = s_free + kTiles;   // [tile] P of the tile's chunk is in tensor memory
+  uint64_t* o_done = p_full + kTiles;   // [tile] the tile's PV of the chunk has completed
+  uint64_t* q_full = o_done + kTiles;   // Q is staged
+  uint64_t* drain = q_full + 1;         // the MMA warp's last MMAs have completed
   uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
 
@@ -184,13 +240,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int q0 = max(min(max(__ldg(p.query_start + seq), 0), q1), q1 - p.max_q_len);
   const int qn = q1 - q0, rows = qn * g;
   const int L = min(__ldg(p.seq_lens + seq), p.max_blocks_per_seq * bs);
-  const int row0 = (int)(gridDim.x - 1 - blockIdx.x) * kRows;  // longest causal ranges first
+  const int row0 = (int)(gridDim.x - 1 - blockIdx.x) * kCtaRows;  // longest causal ranges first
   if (qn <= 0 || row0 >= rows || L <= 0) return;
   const int base_pos = L - qn;
-  const int last_row = min(rows, row0 + kRows) - 1;
+  const int last_row = min(rows, row0 + kCtaRows) - 1;
   const int kv_end = min(L, base_pos + last_row / g + 1);
   if (kv_end <= 0) return;
   const int nchunks = (kv_end + kChunk - 1) / kChunk;
+  const int ntiles = rows - row0 > kRows ? 2 : 1;  // the second tile only if it has rows
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -198,10 +255,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(s_full + b, 1);
-      mbar_init(p_full + b, kSoftWarps * 32);
-      mbar_init(o_done + b, 1);
+    for (int t = 0; t < kTiles; ++t) {
+      mbar_init(s_full + t, 1);
+      mbar_init(s_free + t, kRows);
+      mbar_init(p_full + t, kRows);
+      mbar_init(o_done + t, 1);
     }
     mbar_init(q_full, kSoftWarps * 32);
     mbar_init(drain, 1);
@@ -260,42 +318,52 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------------- MMA ----
+    // S = Q K^T of each tile for chunk c + 1 as soon as the tile's softmax has
+    // read S of chunk c, so it overlaps that softmax; then O += P [V | 1] of
+    // each tile for chunk c once its P is in tensor memory, which also frees
+    // the chunk's stage.
     if (lane == 0) {
       constexpr uint32_t idS = idesc<T>(kRows, kChunk, false);
       constexpr uint32_t idO = idesc<T>(kRows, D + 16, true);  // O and the row sums
-      const uint32_t q_addr = smem_u32(qs), p_addr = smem_u32(ps), r_addr = smem_u32(ring);
+      const uint32_t q_addr = smem_u32(qs), r_addr = smem_u32(ring);
       bool ok = wait5(q_full, 0, abort);
       tc_fence_after();
-      // O += P V for chunk c (its P in buffer c & 1, its V in stage c % kNS).
-      auto issue_pv = [&](int c) -> bool {
-        if (!wait5(p_full + (c & 1), (uint32_t)(c >> 1) & 1u, abort)) return false;
-        tc_fence_after();
-        const uint32_t v = r_addr + (c % kNS) * C::kStage + C::kKV;
-        const uint32_t pa = p_addr + (c & 1) * C::kP;
+      auto issue_qk = [&](int c) -> bool {
+        const int stage = c % kNS;
+        if (!wait5(full + stage, (uint32_t)(c / kNS) & 1u, abort)) return false;
+        const uint32_t k = r_addr + stage * C::kStage;
+        for (int t = 0; t < ntiles; ++t) {
+          if (c > 0 && !wait5(s_free + t, (uint32_t)(c - 1) & 1u, abort)) return false;
+          tc_fence_after();
 #pragma unroll
-        for (int s = 0; s < kChunk / 16; ++s)
-          umma(tmem + 128, sdesc(pa + s * 32, 16), sdesc(v + s * 16 * 128, C::kPlaneKV), idO,
-               (c > 0 || s > 0) ? 1u : 0u);
-        umma_commit(o_done + (c & 1));
+          for (int s = 0; s < D / 16; ++s) {
+            const int pc = s / 4, off = (s % 4) * 32;
+            umma(tmem + 64 * t, sdesc(q_addr + t * C::kQ + pc * C::kPlaneQ + off, 16),
+                 sdesc(k + pc * C::kPlaneKV + off, 16), idS, s > 0 ? 1u : 0u);
+          }
+          umma_commit(s_full + t);
+        }
+        return true;
+      };
+      auto issue_pv = [&](int c) -> bool {
+        const uint32_t v = r_addr + (c % kNS) * C::kStage + C::kKV;
+        for (int t = 0; t < ntiles; ++t) {
+          if (!wait5(p_full + t, (uint32_t)c & 1u, abort)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int s = 0; s < kChunk / 16; ++s)
+            umma_ts(tmem + C::kColO + t * C::kOCols, tmem + C::kColP + 32 * t + 8 * s,
+                    sdesc(v + s * 16 * 128, C::kPlaneKV), idO, (c > 0 || s > 0) ? 1u : 0u);
+          umma_commit(o_done + t);
+        }
         umma_commit(empty + c % kNS);
         return true;
       };
+      if (ok) ok = issue_qk(0);
       for (int c = 0; c < nchunks && ok; ++c) {
-        const int stage = c % kNS;
-        ok = wait5(full + stage, (uint32_t)(c / kNS) & 1u, abort);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t k = r_addr + stage * C::kStage;
-#pragma unroll
-        for (int s = 0; s < D / 16; ++s) {
-          const int pc = s / 4, off = (s % 4) * 32;
-          umma(tmem + 64 * (c & 1), sdesc(q_addr + pc * C::kPlaneQ + off, 16),
-               sdesc(k + pc * C::kPlaneKV + off, 16), idS, s > 0 ? 1u : 0u);
-        }
-        umma_commit(s_full + (c & 1));
-        if (c > 0) ok = issue_pv(c - 1);
+        if (c + 1 < nchunks) ok = issue_qk(c + 1);
+        if (ok) ok = issue_pv(c);
       }
-      if (ok) issue_pv(nchunks - 1);
       // Whatever happened, wait (bounded) until every MMA issued has completed.
       umma_commit(drain);
       const long long t0 = clock64();
@@ -305,88 +373,81 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------- softmax ----
-    const int r = 32 * warp + lane;       // this thread's tensor-memory lane and tile row
-    const int R = row0 + r;
+    const int t = warp / 4;                 // this warp's tile
+    const int r = 32 * (warp % 4) + lane;   // this thread's tensor-memory lane and row of the tile
+    const int R = row0 + kRows * t + r;
     const bool valid = R < rows;
     const int tok = valid ? R / g : 0, j = valid ? R - tok * g : 0;
     const int pos = valid ? base_pos + tok : -1;
-    const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
+    const uint32_t trow = tmem + ((uint32_t)(32 * (warp % 4)) << 16);
+    const uint32_t tS = trow + 64 * t, tP = trow + C::kColP + 32 * t,
+                   tO = trow + C::kColO + t * C::kOCols;
     // Stage this row of Q (zeros past the chunk) in the operand layout.
     {
+      uint8_t* qt = qs + t * C::kQ;
       const uint4* src = reinterpret_cast<const uint4*>(
           static_cast<const T*>(p.query) + ((int64_t)(q0 + tok) * Hq + h * g + j) * D);
 #pragma unroll
       for (int u = 0; u < D / 8; ++u) {
         const uint4 v = valid ? __ldg(src + u) : make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(qs + (u >> 3) * C::kPlaneQ + sw(r, u & 7)) = v;
+        *reinterpret_cast<uint4*>(qt + (u >> 3) * C::kPlaneQ + sw(r, u & 7)) = v;
       }
     }
     // The ones piece of every stage (written once; the copies never touch it).
-    for (int e = r; e < kNS * kChunk * 8; e += kSoftWarps * 32) {
-      const int st = e / (kChunk * 8), t = (e / 8) % kChunk, u = e % 8;
+    for (int e = threadIdx.x; e < kNS * kChunk * 8; e += kSoftWarps * 32) {
+      const int st = e / (kChunk * 8), tk = (e / 8) % kChunk, u = e % 8;
       const uint16_t one = std::is_same<T, __nv_bfloat16>::value ? 0x3F80u : 0x3C00u;
-      const uint32_t w0 = (u == (t & 7)) ? (uint32_t)one : 0u;  // element 0 of the row
-      *reinterpret_cast<uint4*>(ring + st * C::kStage + 2 * C::kKV + t * 128 + u * 16) =
+      const uint32_t w0 = (u == (tk & 7)) ? (uint32_t)one : 0u;  // element 0 of the row
+      *reinterpret_cast<uint4*>(ring + st * C::kStage + 2 * C::kKV + tk * 128 + u * 16) =
           make_uint4(w0, 0u, 0u, 0u);
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     mbar_arrive(q_full);
     const float sscale = p.score_scale;
     float m_use = -INFINITY;
-    bool ok = true;
-    for (int c = 0; c < nchunks; ++c) {
-      ok = wait5(s_full + (c & 1), (uint32_t)(c >> 1) & 1u, abort);
+    bool ok = t < ntiles;
+    for (int c = 0; c < nchunks && ok; ++c) {
+      ok = wait5(s_full + t, (uint32_t)c & 1u, abort);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
       float s[64];
-      {
-        float a[32];
-        tmem_ld32(trow + 64 * (c & 1), a);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[i] = a[i];
-        tmem_ld32(trow + 64 * (c & 1) + 32, a);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[32 + i] = a[i];
-      }
+      tmem_ld64(tS, s);
+      tc_fence_before();
+      mbar_arrive(s_free + t);  // the next S of this tile may overwrite it
       const int c0 = c * kChunk;
       // Raw scores; the causal mask only where the chunk reaches past a row's
       // position. The scale is applied with the exponent (it is positive, so the
       // maximum of the raw scores gives the maximum of the scaled ones).
-      float mx = -INFINITY;
       if (__any_sync(0xffffffffu, c0 + kChunk - 1 > pos)) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          s[i] = c0 + i <= pos ? s[i] : -INFINITY;
-          mx = fmaxf(mx, s[i]);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) mx = fmaxf(mx, s[i]);
+        for (int i = 0; i < 64; ++i) s[i] = c0 + i <= pos ? s[i] : -INFINITY;
       }
-      mx *= sscale;
+      const float mx = max64(s) * sscale;
       // Raise the running maximum only when this chunk exceeds it by 2^8.
       const bool raise = mx > m_use + 8.f;
       const bool rescale = raise && m_use != -INFINITY;
+      bool pv_waited = false;
       if (__any_sync(0xffffffffu, rescale)) {
         if (c > 0) {  // the last PV must have landed in O
-          ok = wait5(o_done + ((c - 1) & 1), (uint32_t)((c - 1) >> 1) & 1u, abort);
+          ok = wait5(o_done + t, (uint32_t)(c - 1) & 1u, abort);
           if (!__all_sync(0xffffffffu, ok)) {
             ok = false;
             break;
           }
           tc_fence_after();
+          pv_waited = true;
         }
         const float alpha = rescale ? fast_exp2(m_use - mx) : 1.f;
 #pragma unroll
         for (int q = 0; q <= D / 32; ++q) {  // O and, in the last group, the row sums
           float o[32];
-          tmem_ld32(trow + 128 + 32 * q, o);
+          tmem_ld32(tO + 32 * q, o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(trow + 128 + 32 * q, o);
+          tmem_st32(tO + 32 * q, o);
         }
       }
       if (raise) m_use = mx;
@@ -408,46 +469,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         float lo, hi;  // (the row sums come from the tensor core, of the rounded P)
         pk[i] = Mma<T>::pack(p0, p1, lo, hi);
       }
-      if (c >= 2) {  // the PV that read this P buffer (chunk c - 2) has completed
-        ok = wait5(o_done + (c & 1), (uint32_t)((c - 2) >> 1) & 1u, abort);
+      if (c > 0 && !pv_waited) {  // the PV that read P of the previous chunk has completed
+        ok = wait5(o_done + t, (uint32_t)(c - 1) & 1u, abort);
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
         }
+        tc_fence_after();
       }
-      if (c == nchunks - 1 && c0 + kChunk > kv_end) {
-        // Zero V rows past the range (stale or poisoned) before the last PV.
+      if (t == 0 && c == nchunks - 1 && c0 + kChunk > kv_end) {
+        // Zero V rows past the range (stale or poisoned) before the last PVs
+        // (tile 0's goes first, so tile 1's comes after these stores too).
         uint8_t* v = ring + (c % kNS) * C::kStage + C::kKV;
         const int t0 = kv_end - c0, per_row = 8 * C::kPlanes;
-        for (int e = r; e < (kChunk - t0) * per_row; e += kSoftWarps * 32) {
-          const int t = t0 + e / per_row, u = e % per_row;
-          *reinterpret_cast<uint4*>(v + (u >> 3) * C::kPlaneKV + t * 128 + (u & 7) * 16) =
+        for (int e = r; e < (kChunk - t0) * per_row; e += kRows) {
+          const int tk = t0 + e / per_row, u = e % per_row;
+          *reinterpret_cast<uint4*>(v + (u >> 3) * C::kPlaneKV + tk * 128 + (u & 7) * 16) =
               make_uint4(0, 0, 0, 0);
         }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
-      uint8_t* prow = ps + (c & 1) * C::kP;
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        *reinterpret_cast<uint4*>(prow + sw(r, u)) =
-            make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tmem_st32(tP, pk);
       tc_fence_before();
-      mbar_arrive(p_full + (c & 1));
+      mbar_arrive(p_full + t);
     }
     if (ok) {
-      ok = wait5(o_done + ((nchunks - 1) & 1), (uint32_t)((nchunks - 1) >> 1) & 1u, abort);
+      ok = wait5(o_done + t, (uint32_t)(nchunks - 1) & 1u, abort);
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
       tc_fence_after();
       float ls[32];
-      tmem_ld32(trow + 128 + D, ls);  // column 128 + D: the row sum of P
+      tmem_ld32(tO + D, ls);  // column D of the tile's O: the row sum of P
       const float inv = ls[0] > 0.f ? 1.f / ls[0] : 0.f;
       T* dst = static_cast<T*>(p.out) + ((int64_t)(q0 + tok) * Hq + h * g + j) * D;
 #pragma unroll
       for (int q = 0; q < D / 32; ++q) {
         float o[32];
-        tmem_ld32(trow + 128 + 32 * q, o);
+        tmem_ld32(tO + 32 * q, o);
         if (valid) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
@@ -487,7 +546,7 @@ cudaError_t launch5(const PrefillParams& p, const CUtensorMap& mk, const CUtenso
     opted_in[dev].store(1, std::memory_order_relaxed);
   }
   const int g = p.num_heads / p.num_kv_heads;
-  const int64_t tiles = ((int64_t)p.max_q_len * g + kRows - 1) / kRows;
+  const int64_t tiles = ((int64_t)p.max_q_len * g + kCtaRows - 1) / kCtaRows;
   dim3 grid((unsigned)tiles, (unsigned)num_seqs, (unsigned)p.num_kv_heads);
   kernel<<<grid, kThreads, C::kSmem, stream>>>(p, mk, mv);
   return cudaGetLastError();
