@@ -11,6 +11,7 @@ from __future__ import annotations
 import concurrent.futures
 import os
 import subprocess
+import tempfile
 import sys
 
 PKG = os.path.dirname(os.path.abspath(__file__))
@@ -48,11 +49,17 @@ def build(force: bool = False, extra_flags=(), out: str = LIB) -> str:
     if not force and not extra_flags and os.path.exists(out) and \
             os.path.getmtime(out) >= _deps_mtime():
         return out
-    build_dir = BUILD if not extra_flags else os.path.join(BUILD, "variant_%d" % os.getpid())
-    os.makedirs(build_dir, exist_ok=True)
+    if extra_flags:  # a variant: objects in a scratch folder, removed afterwards
+        with tempfile.TemporaryDirectory(prefix="pkv_variant_") as d:
+            return _build_into(d, list(extra_flags), out)
+    os.makedirs(BUILD, exist_ok=True)
+    return _build_into(BUILD, [], out)
+
+
+def _build_into(build_dir: str, extra, out: str) -> str:
     srcs = sources()
     with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, build_dir, list(extra_flags)), srcs))
+        objs = list(ex.map(lambda s: _compile(s, build_dir, extra), srcs))
     tmp = out + f".tmp{os.getpid()}"
     subprocess.check_call([NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static"])
     os.replace(tmp, out)
