@@ -11,7 +11,8 @@
 //    (sequence, KV head) — as two tiles of 128, each the M of one tcgen05.mma.
 //    Ten warps: eight softmax warps (warp w serves tile w / 4 and owns tensor-
 //    memory lanes 32 (w % 4) .. +31, one row per thread), a TMA producer warp
-//    and an MMA warp (one thread issues every MMA).
+//    and an MMA warp (the whole warp runs the issue loop on warp-uniform
+//    operands; one elected thread issues every MMA and commit).
 //  * The producer streams the causal range in 64-token chunks through a
 //    three-stage ring shared by both tiles. Each (block, KV head) tile is
 //    copied as one TMA box per 64-element piece of head_dim, so in shared
@@ -147,6 +148,15 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_u32(bar))
                : "memory");
+}
+
+// True in exactly one thread of the (converged) warp.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(pred));
+  return pred != 0;
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -321,50 +331,63 @@ __global__ void __launch_bounds__(kThreads, 1)
     // S = Q K^T of each tile for chunk c + 1 as soon as the tile's softmax has
     // read S of chunk c, so it overlaps that softmax; then O += P [V | 1] of
     // each tile for chunk c once its P is in tensor memory, which also frees
-    // the chunk's stage.
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc<T>(kRows, kChunk, false);
-      constexpr uint32_t idO = idesc<T>(kRows, D + 16, true);  // O and the row sums
-      const uint32_t q_addr = smem_u32(qs), r_addr = smem_u32(ring);
-      bool ok = wait5(q_full, 0, abort);
-      tc_fence_after();
-      auto issue_qk = [&](int c) -> bool {
-        const int stage = c % kNS;
-        if (!wait5(full + stage, (uint32_t)(c / kNS) & 1u, abort)) return false;
-        const uint32_t k = r_addr + stage * C::kStage;
-        for (int t = 0; t < ntiles; ++t) {
-          if (c > 0 && !wait5(s_free + t, (uint32_t)(c - 1) & 1u, abort)) return false;
-          tc_fence_after();
+    // the chunk's stage. The whole warp runs the loop and computes every
+    // operand (warp-uniform values); one elected thread issues each group of
+    // MMAs and the commit that tracks them.
+    constexpr uint32_t idS = idesc<T>(kRows, kChunk, false);
+    constexpr uint32_t idO = idesc<T>(kRows, D + 16, true);  // O and the row sums
+    const uint32_t q_addr = smem_u32(qs), r_addr = smem_u32(ring);
+    const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+    const bool leader = elect_one();  // the same thread issues every MMA and commit
+    auto wait_warp = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, wait5(bar, parity, abort));
+    };
+    bool ok = wait_warp(q_full, 0);
+    tc_fence_after();
+    auto issue_qk = [&](int c) -> bool {
+      const int stage = c % kNS;
+      if (!wait_warp(full + stage, (uint32_t)(c / kNS) & 1u)) return false;
+      const uint32_t k = r_addr + stage * C::kStage;
+      for (int t = 0; t < ntiles; ++t) {
+        if (c > 0 && !wait_warp(s_free + t, (uint32_t)(c - 1) & 1u)) return false;
+        tc_fence_after();
+        if (leader) {
 #pragma unroll
           for (int s = 0; s < D / 16; ++s) {
             const int pc = s / 4, off = (s % 4) * 32;
-            umma(tmem + 64 * t, sdesc(q_addr + t * C::kQ + pc * C::kPlaneQ + off, 16),
+            umma(tm + 64 * t, sdesc(q_addr + t * C::kQ + pc * C::kPlaneQ + off, 16),
                  sdesc(k + pc * C::kPlaneKV + off, 16), idS, s > 0 ? 1u : 0u);
           }
           umma_commit(s_full + t);
         }
-        return true;
-      };
-      auto issue_pv = [&](int c) -> bool {
-        const uint32_t v = r_addr + (c % kNS) * C::kStage + C::kKV;
-        for (int t = 0; t < ntiles; ++t) {
-          if (!wait5(p_full + t, (uint32_t)c & 1u, abort)) return false;
-          tc_fence_after();
+        __syncwarp();
+      }
+      return true;
+    };
+    auto issue_pv = [&](int c) -> bool {
+      const uint32_t v = r_addr + (c % kNS) * C::kStage + C::kKV;
+      for (int t = 0; t < ntiles; ++t) {
+        if (!wait_warp(p_full + t, (uint32_t)c & 1u)) return false;
+        tc_fence_after();
+        if (leader) {
 #pragma unroll
           for (int s = 0; s < kChunk / 16; ++s)
-            umma_ts(tmem + C::kColO + t * C::kOCols, tmem + C::kColP + 32 * t + 8 * s,
+            umma_ts(tm + C::kColO + t * C::kOCols, tm + C::kColP + 32 * t + 8 * s,
                     sdesc(v + s * 16 * 128, C::kPlaneKV), idO, (c > 0 || s > 0) ? 1u : 0u);
           umma_commit(o_done + t);
+          if (t == ntiles - 1) umma_commit(empty + c % kNS);
         }
-        umma_commit(empty + c % kNS);
-        return true;
-      };
-      if (ok) ok = issue_qk(0);
-      for (int c = 0; c < nchunks && ok; ++c) {
-        if (c + 1 < nchunks) ok = issue_qk(c + 1);
-        if (ok) ok = issue_pv(c);
+        __syncwarp();
       }
-      // Whatever happened, wait (bounded) until every MMA issued has completed.
+      return true;
+    };
+    if (ok) ok = issue_qk(0);
+    for (int c = 0; c < nchunks && ok; ++c) {
+      if (c + 1 < nchunks) ok = issue_qk(c + 1);
+      if (ok) ok = issue_pv(c);
+    }
+    // Whatever happened, wait (bounded) until every MMA issued has completed.
+    if (leader) {
       umma_commit(drain);
       const long long t0 = clock64();
       while (!mbar_try(drain, 0))
