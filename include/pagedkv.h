@@ -226,7 +226,7 @@ int paged_attention_decode_static(void* out, const void* query, const void* k_ca
  * block_size and query_start to [0, num_q_tokens]. head_dim 64 or 128,
  * block_size 8/16/32; FP8 caches are not supported here (PKV_ERR_DTYPE). The
  * default kernel runs on the tcgen05 tensor cores with tensor-memory
- * accumulators (128 query rows per CTA); flags PKV_PREFILL_MMA_SYNC selects
+ * accumulators (256 query rows per CTA in two tiles); flags PKV_PREFILL_MMA_SYNC selects
  * the mma.sync kernel (64 rows per CTA) instead; other flag bits are an error.
  * Errors: PKV_ERR_SHAPE, PKV_ERR_UNSUPPORTED, PKV_ERR_DTYPE, PKV_ERR_NULL,
  * PKV_ERR_ALIGN, PKV_ERR_CUDA.
