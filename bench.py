@@ -85,13 +85,24 @@ DECODE_SOURCES = ("common.cuh", "schedule.cuh", "tc_common.cuh", "decode_tc.cu",
                   "pkv_api.cu")
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without its comments and with white space collapsed, so that
+    an edit of a comment or of the layout does not count as a kernel change."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def source_sha() -> str:
-    """Hash of the sources the decode kernels and their launch are built from."""
+    """Hash of the code (comments aside) the decode kernels and their launch are
+    built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_367_b200", "csrc")
-    for name in DECODE_SOURCES:
-        h.update(open(os.path.join(csrc, name), "rb").read())
-    h.update(open(os.path.join(ROOT, "include", "pagedkv.h"), "rb").read())
+    paths = [os.path.join(csrc, name) for name in DECODE_SOURCES]
+    paths.append(os.path.join(ROOT, "include", "pagedkv.h"))
+    for path in paths:
+        with open(path, encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:12]
 
 

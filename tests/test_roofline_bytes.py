@@ -34,3 +34,25 @@ def test_shared_prefix_counts_prefix_once():
 
 def test_append_bytes():
     assert roofline.append_bytes(64, 40, 128, 2, 2) == 2 * 64 * 40 * 128 * 4 + 8 * 64
+
+
+def test_profiled_traffic_ignores_comment_edits_but_not_code_edits(tmp_path, monkeypatch):
+    # The DRAM bytes of a committed ncu summary stay valid across a comment edit
+    # of the decode sources and are dropped (null) once the code changes.
+    import shutil
+    import bench
+    root = tmp_path / "repo"
+    shutil.copytree(bench.ROOT + "/paged_kv_cache_367_b200/csrc", root / "paged_kv_cache_367_b200/csrc")
+    shutil.copytree(bench.ROOT + "/include", root / "include")
+    (root / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    sha = bench.source_sha()
+    (root / "profiles/ncu_decode_w.md").write_text(
+        f"source_sha: {sha}\ntraffic_bytes_per_launch: 1234\n")
+    assert bench.profiled_traffic("w") == 1234.0
+    src = root / "paged_kv_cache_367_b200/csrc/decode_tc.cu"
+    text = src.read_text()
+    src.write_text("// a new comment line\n" + text.replace("\n", "  \n", 3) + "/* and a block */\n")
+    assert bench.source_sha() == sha and bench.profiled_traffic("w") == 1234.0
+    src.write_text(text + "\nstatic int pkv_extra_symbol = 1;\n")
+    assert bench.source_sha() != sha and bench.profiled_traffic("w") is None
