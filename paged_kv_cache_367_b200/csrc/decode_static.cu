@@ -17,7 +17,8 @@
 // cudaGetSymbolAddress while that device is current and keeps it; make that
 // first call before any stream capture. All calls share the array and it keeps
 // the contents of the last call: the counters that must start at zero are
-// cleared by every call (a memset on the caller's stream), and two calls whose
+// cleared by every call (a memset on the caller's stream, whatever the flags
+// say), and two calls whose
 // work overlaps on the GPU (different streams, or different host threads) race
 // on the array and must be serialised by the caller.
 #include <mutex>
@@ -65,6 +66,11 @@ extern "C" int paged_attention_decode_static(
     const int st = static_scratch_address(&scratch);
     if (st != PKV_OK) return st;
   }
+  // The shared array may hold another call's data where this call keeps its
+  // counters (their place depends on the group size and head_dim), so the
+  // counters are always cleared: a caller's PKV_DECODE_ZEROED_WORKSPACE is
+  // ignored here.
+  flags &= ~PKV_DECODE_ZEROED_WORKSPACE;
   return paged_attention_decode(out, query, k_cache, v_cache, block_table, seq_lens, num_seqs,
                                 num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
                                 num_blocks, max_seq_len, scale, q_dtype, cache_dtype, k_scale,

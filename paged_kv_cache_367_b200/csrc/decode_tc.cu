@@ -379,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
           if (ok && b >= 0 && b < nblk) {
             // An id outside the pool reads as zeros (the copy's bounds fill);
             // it is also reported in the status word (bit 1).
-            if ((unsigned)cur >= (unsigned)prm.num_blocks) atomicOr(&g_tc_timeout, 2);
+            if (cur < 0 || (int64_t)cur >= prm.num_blocks) atomicOr(&g_tc_timeout, 2);
             tma_load_5d(st + b * tile, &tmap_k, 0, 0, 0, seg.head, cur, full + stage);
             tma_load_5d(st + C::kKV + b * tile, &tmap_v, 0, 0, 0, seg.head, cur, full + stage);
           }
@@ -408,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, MINB)
         const long long t0 = clock64();
         while (!mbar_try(full + s, (last_parity >> s) & 1u)) {
           if (clock64() - t0 > kWaitCycles) {
-            atomicExch(&g_tc_timeout, 1);
+            atomicOr(&g_tc_timeout, 1);
             break;
           }
         }
@@ -794,9 +794,29 @@ __global__ void __launch_bounds__(kThreads, MINB)
   }
 }
 
+// The status word's self-test: one thread notes an out-of-pool block id (bit
+// 1) as the producer does, then waits on an mbarrier that nothing completes,
+// with a short limit, through the kernels' own bounded wait. The wait must
+// expire, add bit 0 without erasing bit 1, and return.
+__global__ void status_selftest_kernel(long long limit_cycles, int note_out_of_pool) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  abort_flag = 0;
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  if (note_out_of_pool) atomicOr(&g_tc_timeout, 2);
+  mbar_wait_or_abort(&bar, 0, &abort_flag, &g_tc_timeout, limit_cycles);
+}
+
 }  // namespace tc
 
 // ---------------------------------------------------------------- host side ----
+
+int launch_status_selftest(long long limit_cycles, int note_out_of_pool, cudaStream_t stream) {
+  tc::status_selftest_kernel<<<1, 32, 0, stream>>>(limit_cycles, note_out_of_pool);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
 
 int tc_timeout_flag(bool clear, int* value) {
   int v = 0;

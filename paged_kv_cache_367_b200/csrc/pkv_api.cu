@@ -18,6 +18,7 @@ int tc_timeout_flag(bool clear, int* value);
 int pf_timeout_flag(bool clear, int* value);
 int simt_status_flag(bool clear, int* value);
 int pf5_status_flag(bool clear, int* value);
+int launch_status_selftest(long long limit_cycles, int note_out_of_pool, cudaStream_t stream);
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
@@ -75,6 +76,13 @@ int pkv_device_status(int clear) {
       simt_status_flag(clear != 0, &x) != 0 || pf5_status_flag(clear != 0, &y) != 0)
     return PKV_ERR_CUDA;
   return v | w | x | y;
+}
+
+int pkv_selftest_expired_wait(int64_t limit_cycles, int note_out_of_pool, void* stream) {
+  if (limit_cycles < 0 || limit_cycles > (int64_t(1) << 31)) return PKV_ERR_SHAPE;
+  return launch_status_selftest(limit_cycles, note_out_of_pool, (cudaStream_t)stream) == 0
+             ? PKV_OK
+             : PKV_ERR_CUDA;
 }
 
 const char* pkv_status_string(int status) {

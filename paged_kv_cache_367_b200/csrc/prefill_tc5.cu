@@ -307,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_expect_tx(full + stage, (uint32_t)(2 * C::kPlanes * nblk * piece));
       __syncwarp();
       if (lane < nblk) {
-        if ((unsigned)blk >= (unsigned)p.num_blocks) atomicOr(&g_pf5_status, 2);  // reads as zeros
+        if (blk < 0 || blk >= p.num_blocks) atomicOr(&g_pf5_status, 2);  // reads as zeros
 #pragma unroll
         for (int pc = 0; pc < C::kPlanes; ++pc) {
           tma_load_5d(st + pc * C::kPlaneKV + lane * piece, &tmap_k, 0, 0, pc, h, blk, full + stage);

@@ -49,16 +49,17 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
 // the CTA is aborting or the wait expired, which starts the abort and sets the
 // device error word *timeout.
 __device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity,
-                                                   volatile int* abort, int* timeout) {
+                                                   volatile int* abort, int* timeout,
+                                                   long long limit = kWaitCycles) {
   if (*abort) return false;
   const long long t0 = clock64();
   for (int it = 1;; ++it) {
     if (mbar_try(bar, parity)) return true;
     if ((it & 31) == 0) {
       if (*abort) return false;
-      if (clock64() - t0 > kWaitCycles) {
+      if (clock64() - t0 > limit) {
         *abort = 1;
-        atomicExch(timeout, 1);
+        atomicOr(timeout, 1);
         return false;
       }
     }
@@ -167,23 +168,28 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 5-D view of a [num_blocks, bs, Hkv, D] pool of e-byte elements: (d_lo 128/e,
-// token bs, d_hi D*e/128, head Hkv, block num_blocks); one box is a whole
-// (block, head) tile, landing as 128-byte rows with the 128B swizzle.
-// per_plane: the box covers one 128-byte piece of head_dim (d_hi extent 1)
-// instead of all of them, for copies that place each piece in its own region.
+// 5-D view of a [num_blocks, bs, Hkv, D] pool of e-byte elements: (d_lo, token
+// bs, d_hi, head Hkv, block num_blocks), d_lo spanning a row piece of
+// min(D * e, 128) bytes; one box is a whole (block, head) tile, landing as
+// 128-byte rows with the 128B swizzle (64-byte rows with the 64B swizzle when a
+// token's whole row is 64 bytes, as for E4M3 at head_dim 64).
+// per_plane: the box covers one piece of head_dim (d_hi extent 1) instead of
+// all of them, for copies that place each piece in its own region.
 inline bool encode_pool_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int e,
                             int D, int bs, int Hkv, int64_t nb, bool per_plane = false) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
-  const cuuint64_t row = 128 / e;  // elements per 128-byte row
+  const int row_bytes = D * e >= 128 ? 128 : D * e;
+  if (row_bytes != 128 && row_bytes != 64) return false;
+  const cuuint64_t row = (cuuint64_t)(row_bytes / e);  // elements per row piece
   cuuint64_t dims[5] = {row, (cuuint64_t)bs, (cuuint64_t)(D / row), (cuuint64_t)Hkv, (cuuint64_t)nb};
-  cuuint64_t strides[4] = {(cuuint64_t)Hkv * D * e, 128, (cuuint64_t)D * e,
+  cuuint64_t strides[4] = {(cuuint64_t)Hkv * D * e, (cuuint64_t)row_bytes, (cuuint64_t)D * e,
                            (cuuint64_t)bs * Hkv * D * e};
   cuuint32_t box[5] = {(cuuint32_t)row, (cuuint32_t)bs, per_plane ? 1u : (cuuint32_t)(D / row), 1, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = enc(map, dt, 5, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
