@@ -188,8 +188,10 @@ int paged_attention_decode(void* out, const void* query, const void* k_cache,
  * Its first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make it before any stream
  * capture. Every call shares the array, and each call clears what must start at
- * zero; calls whose work overlaps on the GPU (several streams or host threads)
- * race on the array and must be serialised by the caller.
+ * zero (a memset on `stream`; PKV_DECODE_ZEROED_WORKSPACE in `flags` is ignored,
+ * since the array may hold another call's data); calls whose work overlaps on
+ * the GPU (several streams or host threads) race on the array and must be
+ * serialised by the caller.
  */
 int paged_attention_decode_static(void* out, const void* query, const void* k_cache,
                                   const void* v_cache, const int32_t* block_table,
@@ -215,7 +217,10 @@ int paged_attention_decode_static(void* out, const void* query, const void* k_ca
  *                chunk tokens included (their K/V appended beforehand with
  *                paged_kv_append)
  *   k_cache,
- *   v_cache      the pool, cache_dtype == q_dtype
+ *   v_cache      the pool, cache_dtype = q_dtype or PKV_FP8_E4M3
+ *   k_scale,
+ *   v_scale      device fp32 scalars, read only for an FP8 cache (K = code *
+ *                k_scale, V = code * v_scale, as in paged_attention_decode)
  *   out          [num_q_tokens, num_heads, head_dim], q_dtype
  *
  * Row r of sequence i sits at position p = seq_lens[i] - q_i + (r -
@@ -224,10 +229,13 @@ int paged_attention_decode_static(void* out, const void* query, const void* k_ca
  * p < 0 gets zeros. max_q_len must be >= every q_i: a longer chunk has only its
  * last max_q_len rows computed. Lengths are clamped to max_blocks_per_seq *
  * block_size and query_start to [0, num_q_tokens]. head_dim 64 or 128,
- * block_size 8/16/32; FP8 caches are not supported here (PKV_ERR_DTYPE). The
- * default kernel runs on the tcgen05 tensor cores with tensor-memory
- * accumulators (256 query rows per CTA in two tiles); flags PKV_PREFILL_MMA_SYNC selects
- * the mma.sync kernel (64 rows per CTA) instead; other flag bits are an error.
+ * block_size 8/16/32. With a 16-bit cache the default kernel runs on the
+ * tcgen05 tensor cores with tensor-memory accumulators (256 query rows per CTA
+ * in two tiles); flags PKV_PREFILL_MMA_SYNC selects the mma.sync kernel (64
+ * rows per CTA) instead; other flag bits are an error. An FP8-E4M3 cache runs on
+ * the mma.sync kernel: codes widened exactly to f16 in registers, the query
+ * rounded to f16, k_scale folded into the score scale and v_scale into the
+ * output.
  * Errors: PKV_ERR_SHAPE, PKV_ERR_UNSUPPORTED, PKV_ERR_DTYPE, PKV_ERR_NULL,
  * PKV_ERR_ALIGN, PKV_ERR_CUDA.
  */
@@ -238,7 +246,8 @@ int paged_attention_prefill(void* out, const void* query, const void* k_cache,
                             int num_q_tokens, int max_q_len, int num_heads, int num_kv_heads,
                             int head_dim, int block_size, int max_blocks_per_seq,
                             int64_t num_blocks, float scale, int q_dtype, int cache_dtype,
-                            unsigned flags, void* stream);
+                            const float* k_scale, const float* v_scale, unsigned flags,
+                            void* stream);
 
 /*
  * Health word of the device kernels, a bitmask since the last clear:
@@ -251,6 +260,19 @@ int paged_attention_prefill(void* out, const void* query, const void* k_cache,
  * current device; clear != 0 resets the word.
  */
 int pkv_device_status(int clear);
+
+/*
+ * Self-test of the health word above, with no fault: enqueues one tiny kernel
+ * on `stream` that, if note_out_of_pool != 0, records an out-of-pool block id
+ * (value 2) as the kernels do, then waits, through the same bounded wait the
+ * kernels use, on a barrier nothing completes, for at most limit_cycles SM
+ * clock cycles (0 .. 2^31, about one second at 2 GHz). The wait expires and
+ * records value 1 without clearing value 2; the kernel returns and the context
+ * stays usable. pkv_device_status() then reads 1 | (note_out_of_pool ? 2 : 0),
+ * plus whatever was set before. Errors: PKV_ERR_SHAPE (limit out of range),
+ * PKV_ERR_CUDA.
+ */
+int pkv_selftest_expired_wait(int64_t limit_cycles, int note_out_of_pool, void* stream);
 
 /* Static, NUL-terminated description of a pkv_status value. */
 const char* pkv_status_string(int status);

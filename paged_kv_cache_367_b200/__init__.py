@@ -17,7 +17,8 @@ import torch
 __all__ = ["paged_kv_append", "paged_attention_decode", "paged_attention_workspace_size",
            "paged_attention_decode_static", "paged_kv_copy_blocks", "paged_kv_swap_blocks",
            "paged_attention_prefill",
-           "pkv_device_status", "pkv_status_string", "pkv_version", "load_library", "PagedKVError",
+           "pkv_device_status", "pkv_selftest_expired_wait", "pkv_status_string", "pkv_version",
+           "load_library", "PagedKVError",
            "PKV_F32", "PKV_F16", "PKV_BF16", "PKV_FP8_E4M3", "PKV_DECODE_FORCE_SIMT",
            "PKV_DECODE_ZEROED_WORKSPACE", "PKV_DECODE_EARLY_START", "PKV_PREFILL_MMA_SYNC",
            "LIB_PATH", "EXPORTED_SYMBOLS"]
@@ -32,7 +33,8 @@ PKV_PREFILL_MMA_SYNC = 1
 
 EXPORTED_SYMBOLS = ("paged_kv_append", "paged_attention_workspace_size",
                     "paged_attention_decode", "paged_attention_decode_static",
-                    "paged_attention_prefill", "pkv_device_status", "pkv_status_string", "pkv_version",
+                    "paged_attention_prefill", "pkv_device_status", "pkv_selftest_expired_wait",
+                    "pkv_status_string", "pkv_version",
                     # include/pagedkv_blocks.h
                     "pkv_bm_create", "pkv_bm_destroy", "pkv_bm_num_free", "pkv_bm_num_free_host",
                     "pkv_bm_can_allocate", "pkv_bm_allocate", "pkv_bm_can_append",
@@ -76,11 +78,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.pkv_version.restype = I
     lib.pkv_device_status.argtypes = [I]
     lib.pkv_device_status.restype = I
+    lib.pkv_selftest_expired_wait.argtypes = [I64, I, P]
+    lib.pkv_selftest_expired_wait.restype = I
     lib.paged_attention_decode_static.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I64, I, F,
                                                   I, I, P, P, I, I, U, P]
     lib.paged_attention_decode_static.restype = I
     lib.paged_attention_prefill.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I64, F,
-                                            I, I, U, P]
+                                            I, I, P, P, U, P]
     lib.paged_attention_prefill.restype = I
     # Block manager and block copies (include/pagedkv_blocks.h).
     lib.pkv_bm_create.argtypes = [I64, I64, I, I]
@@ -134,8 +138,18 @@ def pkv_version() -> int:
 
 
 def pkv_device_status(clear: bool = False) -> int:
-    """0: no bounded wait inside a kernel has expired (since the last clear)."""
+    """Health word since the last clear: 0 healthy; | 1 a bounded wait inside a
+    kernel expired; | 2 a block-table entry outside the pool was read."""
     return load_library().pkv_device_status(1 if clear else 0)
+
+
+def pkv_selftest_expired_wait(limit_cycles: int = 1 << 20, note_out_of_pool: bool = True) -> None:
+    """Enqueue the health word's fault-free self-test (a bounded wait on a barrier
+    nothing completes) on the current stream."""
+    st = load_library().pkv_selftest_expired_wait(int(limit_cycles), 1 if note_out_of_pool else 0,
+                                                  _stream(None))
+    if st != 0:
+        raise PagedKVError("pkv_selftest_expired_wait", st)
 
 
 def _ptr(t):
@@ -223,7 +237,8 @@ def paged_attention_decode_static(out, query, k_cache, v_cache, block_table, seq
 
 
 def paged_attention_prefill(out, query, k_cache, v_cache, block_table, seq_lens, query_start, *,
-                            max_q_len, scale, flags=0, stream=None) -> None:
+                            max_q_len, scale, k_scale=None, v_scale=None, flags=0,
+                            stream=None) -> None:
     """Causal attention of multi-token queries (chunked prefill, the uncached
     rest of a prefix-cache hit) over the paged cache; see
     paged_attention_prefill in include/pagedkv.h."""
@@ -235,7 +250,7 @@ def paged_attention_prefill(out, query, k_cache, v_cache, block_table, seq_lens,
                                      _ptr(block_table), _ptr(seq_lens), _ptr(query_start), S, T,
                                      int(max_q_len), Hq, Hkv, D, bs, block_table.shape[1], nb,
                                      float(scale), _dtype_code(query), _dtype_code(k_cache),
-                                     int(flags), _stream(stream))
+                                     _ptr(k_scale), _ptr(v_scale), int(flags), _stream(stream))
     if st != 0:
         raise PagedKVError("paged_attention_prefill", st)
 

@@ -19,6 +19,8 @@ struct PrefillParams {
   int num_q_tokens, max_q_len;
   int num_blocks;
   float score_scale;  // softmax scale * log2(e)
+  const float* k_scale;  // device scalars of an E4M3 cache (unused otherwise)
+  const float* v_scale;
 };
 
 // Launch of the tcgen05 kernel (prefill_tc5.cu); mk / mv are per-plane pool maps.

@@ -28,9 +28,20 @@
 //    fragments, P re-packed in registers as the A operand of O += P V (V by
 //    ldmatrix.trans). Slots past the causal range are masked in the scores and
 //    zeroed in V, so stale or poisoned memory never reaches the output.
+//  * FP8-E4M3 caches ("vLLM 0.5 深度拆解" §4.2): the tiles land as codes and are
+//    widened in registers, exactly, to f16 pairs (cvt.rn.f16x2.e4m3x2) right
+//    after ldmatrix; the products run in f16 (the query rounded to f16 once, P
+//    in f16), k_scale is folded into the score scale and v_scale into the final
+//    division. A K row then gives each lane four consecutive dimensions of a
+//    16-dimension step, so the query fragments take the contraction index in
+//    the same permuted order; a transposed V load gives each lane two
+//    dimensions of two tokens, split by one byte permute into an even- and an
+//    odd-dimension operand, so each thread's output columns come out as four
+//    consecutive dimensions.
 //  * Every mbarrier wait is bounded; expiry sets an error word, the CTA stops
 //    and still waits, bounded, for its own copies in flight.
 #include <atomic>
+#include <type_traits>
 
 #include "common.cuh"
 #include "prefill.cuh"
@@ -49,9 +60,11 @@ constexpr int kRows = 64;           // query rows per CTA
 constexpr int kConsumerWarps = 4;   // 16 rows each
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 
-template <int D, int NS>
+template <int D, int NS, int EKV>
 struct Cfg {
-  static constexpr int kKV = kChunk * D * 2;                  // bytes of K (or V) per stage
+  static constexpr int kRowB = D * EKV;                       // bytes of one token's K (or V) row
+  static constexpr int kPieceB = kRowB >= 128 ? 128 : kRowB;  // swizzled row piece (128B or 64B)
+  static constexpr int kKV = kChunk * kRowB;                  // bytes of K (or V) per stage
   static constexpr int kStage = 2 * kKV;
   static constexpr int kQRow = D * 2 + 16;                    // padded Q staging row
   static constexpr int kQ = kConsumerWarps * 16 * kQRow;
@@ -63,20 +76,26 @@ __device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity, volatile in
   return mbar_wait_or_abort(bar, parity, abort, &g_pf_timeout);
 }
 
-// Shared-memory byte offset of 16-byte unit u (elements 8u..8u+7) of token t
-// in a stage's K (or V) half: t / bs selects the block tile, whose rows are
-// 128-byte pieces of head_dim (D / 64 of them per token) with the 128B swizzle.
-template <int D>
+// Shared-memory byte offset of 16-byte unit u of token t in a stage's K (or V)
+// half: t / bs selects the block tile, whose rows are PB-byte pieces of the
+// token's RB-byte row (RB / PB pieces, bs * PB bytes apart) in the PB-byte
+// swizzle (128B: unit j of row r at j ^ (r % 8); 64B: at j ^ (r / 2 % 4)).
+template <int RB, int PB>
 __device__ __forceinline__ uint32_t kv_offset(int t, int u, int bs) {
-  const int tt = t % bs, dh = u >> 3, uu = u & 7;
-  return (uint32_t)((t / bs) * (bs * D * 2) + dh * (bs * 128) + tt * 128 + ((uu ^ (tt & 7)) << 4));
+  constexpr int kUnits = PB / 16;
+  const int tt = t % bs, dh = u / kUnits, uu = u % kUnits;
+  const int x = PB == 128 ? (tt & 7) : ((tt >> 1) & 3);
+  return (uint32_t)((t / bs) * (bs * RB) + dh * (bs * PB) + tt * PB + ((uu ^ x) << 4));
 }
 
-template <typename T, int D, int NS>
+// T: query/output type (bf16 or f16). F8: the cache holds E4M3 codes.
+template <typename T, int D, int NS, bool F8>
 __global__ void __launch_bounds__(kThreads, 2)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_v) {
-  using C = Cfg<D, NS>;
+  constexpr int EKV = F8 ? 1 : 2;
+  using C = Cfg<D, NS, EKV>;
+  using M = typename std::conditional<F8, __half, T>::type;  // MMA operand type
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -103,7 +122,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int kv_end = min(L, base_pos + last_row / g + 1);  // causal range of the tile
   if (kv_end <= 0) return;
   const int nchunks = (kv_end + kChunk - 1) / kChunk;
-  const int tile = bs * D * 2;
+  const int tile = bs * C::kRowB;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -135,7 +154,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (lane == 0) mbar_expect_tx(full + stage, (uint32_t)(2 * nblk * tile));
       __syncwarp();
       if (lane < nblk) {
-        if ((unsigned)blk >= (unsigned)p.num_blocks) atomicOr(&g_pf_timeout, 2);  // reads as zeros
+        if (blk < 0 || blk >= p.num_blocks) atomicOr(&g_pf_timeout, 2);  // reads as zeros
         tma_load_5d(st + lane * tile, &tmap_k, 0, 0, 0, h, blk, full + stage);
         tma_load_5d(st + C::kKV + lane * tile, &tmap_v, 0, 0, 0, h, blk, full + stage);
       }
@@ -181,7 +200,21 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncwarp();
   constexpr int KS = D / 16;  // k-steps over head_dim
   uint32_t qa[KS][4];
-  {
+  if constexpr (F8) {
+    // Contraction index permuted as the E4M3 K fragments hold it: logical
+    // (2cq, 2cq+1) <- dims 4cq, 4cq+1 and (2cq+8, +9) <- dims 4cq+2, +3 of
+    // each 16-dimension step; the query rounded to f16.
+    const uint32_t* r0 = reinterpret_cast<const uint32_t*>(qs + g0 * C::kQRow);
+    const uint32_t* r1 = reinterpret_cast<const uint32_t*>(qs + (g0 + 8) * C::kQRow);
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const int e0 = (16 * ks + 4 * cq) / 2;
+      qa[ks][0] = to_f16x2<T>(r0[e0]);
+      qa[ks][1] = to_f16x2<T>(r1[e0]);
+      qa[ks][2] = to_f16x2<T>(r0[e0 + 1]);
+      qa[ks][3] = to_f16x2<T>(r1[e0 + 1]);
+    }
+  } else {
     const int rr = (lane & 7) + 8 * ((lane >> 3) & 1), cu = lane >> 4;
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks)
@@ -192,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
   for (int dt = 0; dt < DT; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
   float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
-  const float sscale = p.score_scale;
+  const float sscale = p.score_scale * (F8 ? __ldg(p.k_scale) : 1.f);
   const int min_pos = __shfl_sync(0xffffffffu, pos[0], 0);  // row 0 of the warp: smallest
 
   bool ok = true;
@@ -212,15 +245,33 @@ __global__ void __launch_bounds__(kThreads, 2)
       // k-steps outermost: the eight n-tiles are eight independent accumulation
       // chains, so consecutive MMAs do not wait on each other.
       const int mi = lane >> 3, rr = lane & 7;
+      if constexpr (F8) {
+        // One ldmatrix.x4: 16 tokens x two 16-dimension steps of E4M3 codes.
 #pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
+        for (int k2 = 0; k2 < KS / 2; ++k2) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int t = 16 * q + rr + 8 * (mi >> 1);
-          uint32_t b[4];
-          ldsm_x4(b, kst + kv_offset<D>(t, 2 * ks + (mi & 1), bs));
-          Mma<T>::run(s[2 * q], qa[ks], b[0], b[1]);
-          Mma<T>::run(s[2 * q + 1], qa[ks], b[2], b[3]);
+          for (int q = 0; q < 4; ++q) {
+            const int t = 16 * q + rr + 8 * (mi >> 1);
+            uint32_t b[4];
+            ldsm_x4(b, kst + kv_offset<C::kRowB, C::kPieceB>(t, 2 * k2 + (mi & 1), bs));
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              const uint32_t b0 = e4m3x2_to_f16x2(b[x]), b1 = e4m3x2_to_f16x2(b[x] >> 16);
+              Mma<M>::run(s[2 * q + (x >> 1)], qa[2 * k2 + (x & 1)], b0, b1);
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int t = 16 * q + rr + 8 * (mi >> 1);
+            uint32_t b[4];
+            ldsm_x4(b, kst + kv_offset<C::kRowB, C::kPieceB>(t, 2 * ks + (mi & 1), bs));
+            Mma<M>::run(s[2 * q], qa[ks], b[0], b[1]);
+            Mma<M>::run(s[2 * q + 1], qa[ks], b[2], b[3]);
+          }
         }
       }
     }
@@ -262,8 +313,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       const float p0 = fast_exp2(s[nt][0] - msub[0]), p1 = fast_exp2(s[nt][1] - msub[0]);
       const float p2 = fast_exp2(s[nt][2] - msub[1]), p3 = fast_exp2(s[nt][3] - msub[1]);
       float r0, r1, r2, r3;  // the rounded values enter the row sums, as the MMA sees them
-      const uint32_t lo = Mma<T>::pack(p0, p1, r0, r1);
-      const uint32_t hi = Mma<T>::pack(p2, p3, r2, r3);
+      const uint32_t lo = Mma<M>::pack(p0, p1, r0, r1);
+      const uint32_t hi = Mma<M>::pack(p2, p3, r2, r3);
       l[0] += r0 + r1;
       l[1] += r2 + r3;
       pa[nt >> 1][(nt & 1) * 2 + 0] = lo;
@@ -282,12 +333,33 @@ __global__ void __launch_bounds__(kThreads, 2)
           keep0 = (ta < kv_end ? 0x0000ffffu : 0u) | (ta + 1 < kv_end ? 0xffff0000u : 0u);
           keep1 = (tb < kv_end ? 0x0000ffffu : 0u) | (tb + 1 < kv_end ? 0xffff0000u : 0u);
         }
+        if constexpr (F8) {
+          // Per 8 x 16-byte matrix a lane holds dims (2g0, 2g0+1) of tokens
+          // (2cq, 2cq+1); the byte permute gives the pair of tokens at dim 2g0
+          // (low half) and at dim 2g0+1 (high half): the even and the odd
+          // n-tile of the matrix's 16 dimensions. Masks act on the codes.
 #pragma unroll
-        for (int dp = 0; dp < DT / 2; ++dp) {
-          uint32_t b[4];
-          ldsm_x4_t(b, vst + kv_offset<D>(t, 2 * dp + (mi >> 1), bs));
-          Mma<T>::run(o[2 * dp], pa[kk], b[0] & keep0, b[1] & keep1);
-          Mma<T>::run(o[2 * dp + 1], pa[kk], b[2] & keep0, b[3] & keep1);
+          for (int dq = 0; dq < D / 32; ++dq) {
+            uint32_t b[4];
+            ldsm_x4_t(b, vst + kv_offset<C::kRowB, C::kPieceB>(t, 2 * dq + (mi >> 1), bs));
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              const uint32_t lo = __byte_perm(b[2 * half] & keep0, 0, 0x3120);
+              const uint32_t hi = __byte_perm(b[2 * half + 1] & keep1, 0, 0x3120);
+              const int c16 = 2 * dq + half;  // 16-dimension group
+              Mma<M>::run(o[2 * c16], pa[kk], e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi));
+              Mma<M>::run(o[2 * c16 + 1], pa[kk], e4m3x2_to_f16x2(lo >> 16),
+                          e4m3x2_to_f16x2(hi >> 16));
+            }
+          }
+        } else {
+#pragma unroll
+          for (int dp = 0; dp < DT / 2; ++dp) {
+            uint32_t b[4];
+            ldsm_x4_t(b, vst + kv_offset<C::kRowB, C::kPieceB>(t, 2 * dp + (mi >> 1), bs));
+            Mma<M>::run(o[2 * dp], pa[kk], b[0] & keep0, b[1] & keep1);
+            Mma<M>::run(o[2 * dp + 1], pa[kk], b[2] & keep0, b[3] & keep1);
+          }
         }
       }
     }
@@ -303,24 +375,37 @@ __global__ void __launch_bounds__(kThreads, 2)
     lx += __shfl_xor_sync(0xffffffffu, lx, 2);
     const int r = row0 + 16 * w + g0 + 8 * x;
     if (r >= rows) continue;
-    const float inv = lx > 0.f ? 1.f / lx : 0.f;
+    const float inv = lx > 0.f ? (F8 ? __ldg(p.v_scale) : 1.f) / lx : 0.f;
     const int tok = r / g, j = r - tok * g;
-    T* dst = static_cast<T*>(p.out) + ((int64_t)(q0 + tok) * Hq + h * g + j) * D + 2 * cq;
+    T* row = static_cast<T*>(p.out) + ((int64_t)(q0 + tok) * Hq + h * g + j) * D;
+    if constexpr (F8) {
+      // n-tiles 2c and 2c + 1 hold dims 16c + 4cq + {0, 2} and {1, 3}.
 #pragma unroll
-    for (int dt = 0; dt < DT; ++dt) {
-      float a, b;
-      *reinterpret_cast<uint32_t*>(dst + 8 * dt) =
-          Mma<T>::pack(o[dt][2 * x] * inv, o[dt][2 * x + 1] * inv, a, b);
+      for (int c16 = 0; c16 < D / 16; ++c16) {
+        float a, b;
+        uint2 w;
+        w.x = Mma<T>::pack(o[2 * c16][2 * x] * inv, o[2 * c16 + 1][2 * x] * inv, a, b);
+        w.y = Mma<T>::pack(o[2 * c16][2 * x + 1] * inv, o[2 * c16 + 1][2 * x + 1] * inv, a, b);
+        *reinterpret_cast<uint2*>(row + 16 * c16 + 4 * cq) = w;
+      }
+    } else {
+      T* dst = row + 2 * cq;
+#pragma unroll
+      for (int dt = 0; dt < DT; ++dt) {
+        float a, b;
+        *reinterpret_cast<uint32_t*>(dst + 8 * dt) =
+            Mma<T>::pack(o[dt][2 * x] * inv, o[dt][2 * x + 1] * inv, a, b);
+      }
     }
   }
 }
 
-template <typename T, int D>
+template <typename T, int D, bool F8>
 cudaError_t launch_t(const PrefillParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
                      int max_q_len, int num_seqs, cudaStream_t stream) {
-  constexpr int NS = D == 128 ? 2 : 4;
-  using C = Cfg<D, NS>;
-  auto kernel = prefill_tc_kernel<T, D, NS>;
+  constexpr int NS = (D == 128 && !F8) ? 2 : 4;  // stages of 32 KB (16-bit, D 128) or less
+  using C = Cfg<D, NS, F8 ? 1 : 2>;
+  auto kernel = prefill_tc_kernel<T, D, NS, F8>;
   static std::atomic<int> opted_in[64];  // the shared-memory opt-in, once per device
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
@@ -358,7 +443,8 @@ extern "C" int paged_attention_prefill(void* out, const void* query, const void*
                                        int num_seqs, int num_q_tokens, int max_q_len,
                                        int num_heads, int num_kv_heads, int head_dim,
                                        int block_size, int max_blocks_per_seq, int64_t num_blocks,
-                                       float scale, int q_dtype, int cache_dtype, unsigned flags,
+                                       float scale, int q_dtype, int cache_dtype,
+                                       const float* k_scale, const float* v_scale, unsigned flags,
                                        void* stream) {
   using namespace pkv;
   if (num_seqs < 0 || num_q_tokens < 0 || max_q_len < 0 || num_kv_heads <= 0 ||
@@ -368,24 +454,30 @@ extern "C" int paged_attention_prefill(void* out, const void* query, const void*
     return PKV_ERR_SHAPE;
   if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
   if (block_size != 8 && block_size != 16 && block_size != 32) return PKV_ERR_UNSUPPORTED;
-  if ((q_dtype != PKV_BF16 && q_dtype != PKV_F16) || cache_dtype != q_dtype)
+  if ((q_dtype != PKV_BF16 && q_dtype != PKV_F16) ||
+      (cache_dtype != q_dtype && cache_dtype != PKV_FP8_E4M3))
     return PKV_ERR_DTYPE;
+  const bool f8 = cache_dtype == PKV_FP8_E4M3;
   if (num_seqs == 0 || num_q_tokens == 0 || max_q_len == 0) return PKV_OK;
   if (!out || !query || !k_cache || !v_cache || !block_table || !seq_lens || !query_start)
     return PKV_ERR_NULL;
+  if (f8 && (!k_scale || !v_scale)) return PKV_ERR_NULL;
   if (((uintptr_t)out | (uintptr_t)query | (uintptr_t)k_cache | (uintptr_t)v_cache) & 15u ||
       ((uintptr_t)block_table | (uintptr_t)seq_lens | (uintptr_t)query_start) & 3u)
     return PKV_ERR_ALIGN;
   const int64_t tiles = ((int64_t)max_q_len * (num_heads / num_kv_heads) + pf::kRows - 1) /
                         pf::kRows;
   if (tiles > INT32_MAX) return PKV_ERR_SHAPE;
-  const CUtensorMapDataType dt =
-      q_dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  const bool tc5 = !(flags & PKV_PREFILL_MMA_SYNC) && pf::prefill_tc5_supported(head_dim);
+  const CUtensorMapDataType dt = f8                   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : q_dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  // E4M3 caches run on the mma.sync kernel, widened in registers.
+  const bool tc5 = !f8 && !(flags & PKV_PREFILL_MMA_SYNC) && pf::prefill_tc5_supported(head_dim);
+  const int e = f8 ? 1 : 2;
   CUtensorMap mk, mv;
-  if (!tcx::encode_pool_map(&mk, k_cache, dt, 2, head_dim, block_size, num_kv_heads, num_blocks,
+  if (!tcx::encode_pool_map(&mk, k_cache, dt, e, head_dim, block_size, num_kv_heads, num_blocks,
                             tc5) ||
-      !tcx::encode_pool_map(&mv, v_cache, dt, 2, head_dim, block_size, num_kv_heads, num_blocks,
+      !tcx::encode_pool_map(&mv, v_cache, dt, e, head_dim, block_size, num_kv_heads, num_blocks,
                             tc5))
     return PKV_ERR_CUDA;
   pf::PrefillParams p;
@@ -402,15 +494,24 @@ extern "C" int paged_attention_prefill(void* out, const void* query, const void*
   p.max_q_len = max_q_len;
   p.num_blocks = (int)num_blocks;
   p.score_scale = scale * 1.4426950408889634f;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e;
+  cudaError_t err;
+  const bool bf16 = q_dtype == PKV_BF16, d128 = head_dim == 128;
   if (tc5)
-    e = pf::launch_prefill_tc5(p, mk, mv, head_dim, q_dtype == PKV_BF16, num_seqs, st);
-  else if (q_dtype == PKV_BF16)
-    e = head_dim == 128 ? pf::launch_t<__nv_bfloat16, 128>(p, mk, mv, max_q_len, num_seqs, st)
-                        : pf::launch_t<__nv_bfloat16, 64>(p, mk, mv, max_q_len, num_seqs, st);
+    err = pf::launch_prefill_tc5(p, mk, mv, head_dim, bf16, num_seqs, st);
+  else if (f8 && bf16)
+    err = d128 ? pf::launch_t<__nv_bfloat16, 128, true>(p, mk, mv, max_q_len, num_seqs, st)
+               : pf::launch_t<__nv_bfloat16, 64, true>(p, mk, mv, max_q_len, num_seqs, st);
+  else if (f8)
+    err = d128 ? pf::launch_t<__half, 128, true>(p, mk, mv, max_q_len, num_seqs, st)
+               : pf::launch_t<__half, 64, true>(p, mk, mv, max_q_len, num_seqs, st);
+  else if (bf16)
+    err = d128 ? pf::launch_t<__nv_bfloat16, 128, false>(p, mk, mv, max_q_len, num_seqs, st)
+               : pf::launch_t<__nv_bfloat16, 64, false>(p, mk, mv, max_q_len, num_seqs, st);
   else
-    e = head_dim == 128 ? pf::launch_t<__half, 128>(p, mk, mv, max_q_len, num_seqs, st)
-                        : pf::launch_t<__half, 64>(p, mk, mv, max_q_len, num_seqs, st);
-  return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    err = d128 ? pf::launch_t<__half, 128, false>(p, mk, mv, max_q_len, num_seqs, st)
+               : pf::launch_t<__half, 64, false>(p, mk, mv, max_q_len, num_seqs, st);
+  return err == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }

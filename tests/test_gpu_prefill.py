@@ -17,7 +17,9 @@ pytestmark = pytest.mark.gpu
 TORCH = {"bf16": torch.bfloat16, "f16": torch.float16}
 
 
-def make_case(lens, qlens, Hq, Hkv, D, bs, dt, dev, seed=0, spare=5):
+def make_case(lens, qlens, Hq, Hkv, D, bs, dt, dev, seed=0, spare=5, cache=None):
+    """Pools for the given lengths (cache: None = the query dtype, or "e4m3":
+    codes drawn as in workloads.py with k_scale = v_scale = 5/448)."""
     rng = np.random.default_rng(seed)
     gen = torch.Generator().manual_seed(seed)
     nbs = [-(-L // bs) for L in lens]
@@ -29,20 +31,29 @@ def make_case(lens, qlens, Hq, Hkv, D, bs, dt, dev, seed=0, spare=5):
     for i, k in enumerate(nbs):
         bt[i, :k] = ids[n:n + k]
         n += k
-    kc = torch.randn((nb, bs, Hkv, D), generator=gen).to(TORCH[dt])
-    vc = torch.randn((nb, bs, Hkv, D), generator=gen).to(TORCH[dt])
+    cache = cache or dt
+    if cache == "e4m3":
+        def codes():
+            x = (torch.randn((nb, bs, Hkv, D), generator=gen) * W.FP8_CODE_SIGMA).clamp(-448, 448)
+            return x.to(torch.float8_e4m3fn).view(torch.uint8)
+        kc, vc = codes(), codes()
+    else:
+        kc = torch.randn((nb, bs, Hkv, D), generator=gen).to(TORCH[dt])
+        vc = torch.randn((nb, bs, Hkv, D), generator=gen).to(TORCH[dt])
     # Slots past every sequence's length hold NaN: they must never reach the output.
     used = np.zeros((nb, bs), bool)
     for i, L in enumerate(lens):
         for t in range(L):
             used[bt[i, t // bs], t % bs] = True
     mask = torch.from_numpy(~used)
-    kc[mask] = float("nan")
-    vc[mask] = float("nan")
+    nan = 0x7F if cache == "e4m3" else float("nan")
+    kc[mask] = nan
+    vc[mask] = nan
     qs = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
     q = torch.randn((int(qs[-1]), Hq, D), generator=gen).to(TORCH[dt])
+    sc = W.FP8_SCALE if cache == "e4m3" else 1.0
     return dict(kc=kc.to(dev), vc=vc.to(dev), bt=bt, lens=np.asarray(lens, np.int32), qs=qs,
-                q=q.to(dev), Hq=Hq, Hkv=Hkv, D=D, bs=bs, dt=dt, dev=dev)
+                q=q.to(dev), Hq=Hq, Hkv=Hkv, D=D, bs=bs, dt=dt, dev=dev, cache=cache, sc=sc)
 
 
 def run_gpu(c, max_q_len=None, bt=None, fill=float("nan"), status=0, flags=0):
@@ -50,10 +61,14 @@ def run_gpu(c, max_q_len=None, bt=None, fill=float("nan"), status=0, flags=0):
     out = torch.full(tuple(c["q"].shape), fill, dtype=c["q"].dtype, device=dev)
     bt = c["bt"] if bt is None else bt
     mq = int(np.diff(c["qs"]).max()) if max_q_len is None else max_q_len
+    ks = vs = None
+    if c["cache"] == "e4m3":
+        ks = torch.tensor([c["sc"]], dtype=torch.float32, device=dev)
+        vs = torch.tensor([c["sc"]], dtype=torch.float32, device=dev)
     pkv.paged_attention_prefill(out, c["q"], c["kc"], c["vc"], torch.from_numpy(bt).to(dev),
                                 torch.from_numpy(c["lens"]).to(dev),
                                 torch.from_numpy(c["qs"]).to(dev), max_q_len=mq,
-                                scale=c["D"] ** -0.5, flags=flags)
+                                scale=c["D"] ** -0.5, k_scale=ks, v_scale=vs, flags=flags)
     torch.cuda.synchronize()
     assert pkv.pkv_device_status(clear=True) == status
     return out
@@ -64,7 +79,7 @@ def run_oracle(c, bt=None):
     want, _ = oracle.prefill(W.host(c["q"]), W.host(c["kc"]), W.host(c["vc"]), bt, c["lens"],
                              c["qs"], num_heads=c["Hq"], num_kv_heads=c["Hkv"], head_dim=c["D"],
                              block_size=c["bs"], scale=c["D"] ** -0.5, q_dtype=c["dt"],
-                             cache_dtype=c["dt"])
+                             cache_dtype=c["cache"], k_scale=c["sc"], v_scale=c["sc"])
     return want
 
 
@@ -187,3 +202,44 @@ def test_block_ids_outside_the_pool_read_as_zeros(cuda_dev, flags):
     bt[0, 1] = nb + 7
     bt[1, 0] = -3
     check(run_gpu(c, bt=bt, status=2, flags=flags), run_oracle(c, bt=bt), "bf16")  # reported
+
+
+@pytest.mark.parametrize("case", list(CASES))
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (32, 8), (16, 1), (12, 2)])
+@pytest.mark.parametrize("D", [64, 128])
+def test_prefill_fp8_cache_parity(cuda_dev, case, Hq, Hkv, D):
+    # E4M3 caches: codes widened in registers, k_scale folded into the scores,
+    # v_scale into the output; the tcgen05 flag has no effect on this path.
+    lens, qlens = CASES[case]
+    c = make_case(lens, qlens, Hq, Hkv, D, 16, "bf16", cuda_dev, seed=Hq + D, cache="e4m3")
+    check(run_gpu(c), run_oracle(c), "e4m3")
+
+
+@pytest.mark.parametrize("bs", [8, 16, 32])
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+@pytest.mark.parametrize("D", [64, 128])
+def test_prefill_fp8_cache_blocks_dtypes(cuda_dev, bs, dt, D):
+    c = make_case([400, 90, 33], [200, 90, 5], 16, 4, D, bs, dt, cuda_dev, seed=D + bs + 1,
+                  cache="e4m3")
+    check(run_gpu(c, flags=pkv.PKV_PREFILL_MMA_SYNC), run_oracle(c), "e4m3")
+
+
+def test_prefill_fp8_out_of_pool_and_prefix_hit_matches_decode(cuda_dev):
+    # Out-of-pool ids read as zeros and are reported; a one-token chunk over an
+    # FP8 cache equals the FP8 decode of the same token.
+    c = make_case([70, 33, 500], [20, 33, 1], 16, 4, 128, 16, "bf16", cuda_dev, seed=8,
+                  cache="e4m3")
+    bt = c["bt"].copy()
+    bt[0, 1] = c["kc"].shape[0] + 7
+    check(run_gpu(c, bt=bt, status=2), run_oracle(c, bt=bt), "e4m3")
+    got = run_gpu(c)
+    last = int(c["qs"][-1]) - 1
+    q1 = c["q"][last:last + 1]
+    out = torch.empty_like(q1)
+    sc = torch.tensor([c["sc"]], dtype=torch.float32, device=cuda_dev)
+    pkv.paged_attention_decode(out, q1, c["kc"], c["vc"],
+                               torch.from_numpy(c["bt"][2:3].copy()).to(cuda_dev),
+                               torch.from_numpy(c["lens"][2:3].copy()).to(cuda_dev),
+                               max_seq_len=500, scale=128 ** -0.5, k_scale=sc, v_scale=sc)
+    torch.cuda.synchronize()
+    assert (got[last:last + 1].float() - out.float()).abs().max().item() <= 2 * TOL["e4m3"][0]

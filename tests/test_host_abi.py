@@ -177,7 +177,7 @@ def prefill(lib, **kw):
     a = dict(out=A, query=A, k_cache=A, v_cache=A, block_table=A, seq_lens=A, query_start=A,
              num_seqs=2, num_q_tokens=10, max_q_len=8, num_heads=8, num_kv_heads=2, head_dim=128,
              block_size=16, max_blocks_per_seq=8, num_blocks=100, scale=0.1, q_dtype=BF16,
-             cache_dtype=BF16, flags=0, stream=None)
+             cache_dtype=BF16, k_scale=A, v_scale=A, flags=0, stream=None)
     a.update(kw)
     return lib.paged_attention_prefill(*a.values())
 
@@ -189,7 +189,9 @@ def prefill(lib, **kw):
     (dict(num_blocks=0), ESHAPE), (dict(max_blocks_per_seq=0), ESHAPE),
     (dict(scale=float("nan")), ESHAPE), (dict(num_seqs=70000), ESHAPE),
     (dict(head_dim=96), EUNSUP), (dict(block_size=4), EUNSUP),
-    (dict(cache_dtype=FP8), EDTYPE), (dict(q_dtype=F32, cache_dtype=F32), EDTYPE),
+    (dict(q_dtype=F32, cache_dtype=F32), EDTYPE), (dict(q_dtype=F32, cache_dtype=FP8), EDTYPE),
+    (dict(cache_dtype=F16), EDTYPE), (dict(cache_dtype=FP8, k_scale=None), ENULL),
+    (dict(cache_dtype=FP8, v_scale=None), ENULL),
     (dict(query=A + 8), EALIGN), (dict(query_start=A + 2), EALIGN), (dict(flags=2), ESHAPE),
 ])
 def test_prefill_rejects_bad_arguments(lib, kw, code):

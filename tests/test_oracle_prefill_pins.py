@@ -108,3 +108,38 @@ def test_single_token_chunks_equal_decode(orc):
     out = run_prefill(orc, q, kc, vc, bt, lens, [0, 1, 2, 3], Hq, Hkv, D, bs, 0.1)
     dec = oracle_f32(orc, q, kc, vc, bt, lens, Hq, Hkv, D, bs, 0.1)
     assert np.array_equal(out, dec)
+
+
+def test_prefill_over_e4m3_codes_matches_brute_force_with_scales(orc):
+    # E4M3 pool: K[t] = code value * k_scale, V[t] = code value * v_scale. The
+    # brute force decodes the codes with torch's float8_e4m3fn (not the oracle's
+    # decoder) and takes the bf16 query values from torch as well.
+    import torch
+    rng = np.random.default_rng(11)
+    D, bs, Hq, Hkv = 32, 8, 4, 2
+    lens, qlens = [23, 40], [23, 6]
+    qs = np.concatenate([[0], np.cumsum(qlens)])
+    bt, nb = _layout(rng, lens, bs)
+    codes_k = rng.integers(0, 256, size=(nb, bs, Hkv, D), dtype=np.uint8)
+    codes_v = rng.integers(0, 256, size=(nb, bs, Hkv, D), dtype=np.uint8)
+    for c in (codes_k, codes_v):      # no NaN codes (S.1111.111)
+        c[(c & 0x7F) == 0x7F] = 0x3A
+    qb = torch.randn((int(qs[-1]), Hq, D), generator=torch.Generator().manual_seed(3)).to(
+        torch.bfloat16)
+    ks, vs = 0.0625, 0.375             # exact in binary32
+    out, _ = orc.prefill(qb.view(torch.int16).numpy().view(np.uint16), codes_k, codes_v, bt,
+                         np.asarray(lens, np.int32), qs.astype(np.int32), num_heads=Hq,
+                         num_kv_heads=Hkv, head_dim=D, block_size=bs, scale=0.25,
+                         q_dtype="bf16", cache_dtype="e4m3", k_scale=ks, v_scale=vs)
+    dec = lambda c: torch.from_numpy(c).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    kv, vv = dec(codes_k) * ks, dec(codes_v) * vs
+    qv = qb.to(torch.float64).numpy()
+    g = Hq // Hkv
+    for i, (L, n) in enumerate(zip(lens, qlens)):
+        rows_k = np.stack([kv[bt[i, t // bs], t % bs] for t in range(L)])
+        rows_v = np.stack([vv[bt[i, t // bs], t % bs] for t in range(L)])
+        pos = np.arange(L - n, L)
+        for j in range(Hq):
+            want = brute_causal(qv[qs[i]:qs[i + 1], j], rows_k[:, j // g], rows_v[:, j // g],
+                                pos, 0.25)
+            assert np.max(np.abs(out[qs[i]:qs[i + 1], j] - want)) <= 1e-12
