@@ -73,11 +73,14 @@ def parse_args():
     ap.add_argument("--plain-launch", action="store_true",
                     help="decode without PKV_DECODE_ZEROED_WORKSPACE | PKV_DECODE_EARLY_START "
                          "(zero the counters every call; no programmatic dependent launch)")
-    ap.add_argument("--op", default="decode", choices=["decode", "blocks", "blocksize", "prefill"],
+    ap.add_argument("--op", default="decode",
+                    choices=["decode", "blocks", "blocksize", "prefill", "kernels"],
                     help="blocks: time the block copies (copy-on-write, swap) and the host "
                          "block manager; blocksize: decode time and pool fragmentation for "
                          "block sizes 8/16/32; prefill: causal multi-token queries over the "
-                         "paged cache (one JSON line each) instead of the decode step")
+                         "paged cache; kernels: the tensor-core decode kernel against the "
+                         "CUDA-core one on the MHA and GQA workloads (one JSON line each) "
+                         "instead of the decode step")
     return ap.parse_args()
 
 
@@ -130,14 +133,16 @@ def profiled_traffic(workload: str):
 
 
 class ClockSampler:
-    """Polls SM clock and clock-event reasons through NVML while running."""
+    """SM clock and clock-event reasons through NVML: one sample when entered,
+    one every `period` seconds while running, one when left."""
 
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x2: "applications_clocks_setting", 0x10: "sync_boost"}
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, period: float = 0.0005):
         self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period
         self._stop = threading.Event()
         try:
             import pynvml
@@ -154,29 +159,36 @@ class ClockSampler:
             self._nv = None
         self._t = threading.Thread(target=self._run, daemon=True)
 
+    def sample(self):
+        if self._nv is None:
+            return
+        try:
+            self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+            r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
     def _run(self):
-        while not self._stop.is_set() and self._nv is not None:
-            try:
-                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
-                r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-                for bit, name in self.REASONS.items():
-                    if r & bit:
-                        self.reasons.add(name)
-            except Exception:
-                pass
-            time.sleep(0.005)
+        while not self._stop.wait(self.period):
+            self.sample()
 
     def __enter__(self):
+        self.sample()
         self._t.start()
         return self
 
     def __exit__(self, *exc):
         self._stop.set()
         self._t.join()
+        self.sample()
 
     def summary(self):
         return {"sm_mhz": float(np.median(self.samples)) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "sm_mhz_min": float(np.min(self.samples)) if self.samples else None,
                 "reasons": sorted(self.reasons)}
 
 
@@ -217,6 +229,132 @@ def step_bytes(wl):
 
 # ------------------------------------------------------------------ our arm ----
 
+def kernel_time_ms(pre, call, n=16, reps=5):
+    """Mean device time of call() per launch: a CUDA graph of n x (pre(), event,
+    call(), event) is replayed `reps` times and the events' spans averaged. The
+    events are graph nodes (recorded as external events), so the span is the
+    launch's own time with no host gap. Falls back to events around eager
+    launches if the graph cannot be built. Returns (ms, how)."""
+    stream = torch.cuda.current_stream()
+    try:
+        evs = [(torch.cuda.Event(enable_timing=True, external=True),
+                torch.cuda.Event(enable_timing=True, external=True)) for _ in range(n)]
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            for _ in range(3):
+                pre()
+                call()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for a, b in evs:
+                pre()
+                a.record()
+                call()
+                b.record()
+        g.replay()
+        torch.cuda.synchronize()
+        spans = []
+        for _ in range(reps):
+            g.replay()
+            torch.cuda.synchronize()
+            spans += [a.elapsed_time(b) for a, b in evs]
+        del g
+        return float(np.mean(spans)), (f"CUDA events as graph nodes around each of {n} launches "
+                                        f"per graph replay, {reps} replays")
+    except Exception as e:  # noqa: BLE001 - report how it was timed instead
+        torch.cuda.synchronize()
+        reason = f"{type(e).__name__}"
+    m = max(n * reps, 20)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(m)]
+    for a, b in ev:
+        pre()
+        a.record(stream)
+        call()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return (float(np.mean([a.elapsed_time(b) for a, b in ev])),
+            f"CUDA events around {m} eager launches (graph events unavailable: {reason})")
+
+
+def e2e_time_ms(args, wl, append, decode, out, world):
+    """Per-step time of the step through the public API with host buffers.
+
+    Every step copies its inputs (query, new K/V, slot mapping, block table,
+    lengths), packed in one pinned host buffer, to the device in one copy, runs
+    paged_kv_append and paged_attention_decode through the binding, and copies
+    the output back to pinned host memory. Inputs and outputs are double
+    buffered and the copies run on their own streams, so step k+1's inputs and
+    step k-1's output move while step k computes; the timed region spans the
+    first input copy to the last output copy."""
+    K = args.steps
+    KE = args.e2e_steps or max(min(K, 200), 50)
+    parts = [wl.query, wl.new_key, wl.new_value, torch.from_numpy(wl.slot_mapping),
+             torch.from_numpy(wl.block_table), torch.from_numpy(wl.seq_lens)]
+    offs, total = [], 0
+    for t in parts:
+        total = (total + 255) // 256 * 256
+        offs.append(total)
+        total += t.numel() * t.element_size()
+    h_in = [torch.empty(total, dtype=torch.uint8).pin_memory() for _ in range(2)]
+    d_in = [torch.empty(total, dtype=torch.uint8, device=out.device) for _ in range(2)]
+    views = []
+    for b in range(2):
+        v = []
+        for t, o in zip(parts, offs):
+            nb = t.numel() * t.element_size()
+            h_in[b][o:o + nb].copy_(t.detach().cpu().contiguous().view(-1).view(torch.uint8))
+            v.append(d_in[b][o:o + nb].view(t.dtype).view(t.shape))
+        views.append(v)
+    outs = [out, torch.empty_like(out)]
+    h_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    h2d, d2h = total, out.numel() * out.element_size()
+    compute = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_used = [torch.cuda.Event() for _ in range(2)]     # step done with its inputs
+    ev_out = [torch.cuda.Event() for _ in range(2)]      # output ready
+    ev_read = [torch.cuda.Event() for _ in range(2)]     # output copied to the host
+
+    def run(steps):
+        for k in range(steps):
+            b = k & 1
+            if k >= 2:
+                s_in.wait_event(ev_used[b])
+            with torch.cuda.stream(s_in):
+                d_in[b].copy_(h_in[b], non_blocking=True)
+                ev_in[b].record(s_in)
+            compute.wait_event(ev_in[b])
+            if k >= 2:
+                compute.wait_event(ev_read[b])
+            q, nk, nv, sl, bt, ln = views[b]
+            append(nk, nv, sl)
+            decode(q, bt, ln, outs[b])
+            ev_used[b].record(compute)
+            ev_out[b].record(compute)
+            s_out.wait_event(ev_out[b])
+            with torch.cuda.stream(s_out):
+                h_out[b].copy_(outs[b], non_blocking=True)
+                ev_read[b].record(s_out)
+
+    run(4)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(compute)
+    s_in.wait_stream(compute)
+    run(KE)
+    compute.wait_stream(s_out)
+    e1.record(compute)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / KE, KE, h2d, d2h, h_out[(KE - 1) & 1]
+
+
+
 def run_ours(args, rank, world, dev):
     cfg = W.CONFIGS[args.workload]
     cfg = cfg.replace(seed=replica_seed(cfg.seed, rank))
@@ -247,8 +385,10 @@ def run_ours(args, rank, world, dev):
                                            pkv.PKV_DECODE_EARLY_START)
     first = [True]
 
-    def decode(q, bt_t, lens_t, out_t):
+    def decode(q, bt_t, lens_t, out_t, early=True):
         flags = args.flags | (0 if first[0] else serving)
+        if not early:
+            flags &= ~pkv.PKV_DECODE_EARLY_START
         first[0] = False
         pkv.paged_attention_decode(out_t, q, wl.k_cache, wl.v_cache, bt_t, lens_t, max_seq_len=msl,
                                    scale=c.scale, partition_size=P, workspace=ws, k_scale=ks,
@@ -292,53 +432,16 @@ def run_ours(args, rank, world, dev):
     step_ms = t0.elapsed_time(t1) / K
     if world > 1:
         torch.distributed.barrier()
-    # The decode kernel alone: CUDA events around eager launches of the same call.
-    KD = min(K, 200)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(KD)]
-    for k in range(KD):
-        append(wl.new_key, wl.new_value, slots)
-        ev[k][0].record(stream)
-        decode(wl.query, bt, lens, out)
-        ev[k][1].record(stream)
-    torch.cuda.synchronize()
-    decode_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    # The decode kernel alone: CUDA events recorded around each decode launch
+    # inside a CUDA graph of several steps (append, event, decode, event), so no
+    # host launch gap is timed; eager launches if the graph cannot hold events.
+    decode_ms, decode_timing = kernel_time_ms(
+        lambda: append(wl.new_key, wl.new_value, slots),
+        lambda: decode(wl.query, bt, lens, out, early=False), reps=max(1, min(K // 20, 10)))
     status = pkv.pkv_device_status(clear=True)
     assert status == 0, f"device wait expired (status {status})"
 
-    # End to end: per-step inputs start in pinned host memory, the output ends there.
-    KE = args.e2e_steps or min(K, 200)
-    h_q = wl.query.cpu().pin_memory()
-    h_k, h_v = wl.new_key.cpu().pin_memory(), wl.new_value.cpu().pin_memory()
-    h_slots = torch.from_numpy(wl.slot_mapping).pin_memory()
-    h_bt = torch.from_numpy(wl.block_table).pin_memory()
-    h_lens = torch.from_numpy(wl.seq_lens).pin_memory()
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    d_q, d_k, d_v = torch.empty_like(wl.query), torch.empty_like(wl.new_key), torch.empty_like(wl.new_value)
-    d_slots, d_bt, d_lens = torch.empty_like(slots), torch.empty_like(bt), torch.empty_like(lens)
-    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_bt, h_lens))
-    d2h = h_out.numel() * h_out.element_size()
-
-    def e2e_step():
-        for d, h in ((d_q, h_q), (d_k, h_k), (d_v, h_v), (d_slots, h_slots), (d_bt, h_bt),
-                     (d_lens, h_lens)):
-            d.copy_(h, non_blocking=True)
-        append(d_k, d_v, d_slots)
-        decode(d_q, d_bt, d_lens, out)
-        h_out.copy_(out, non_blocking=True)
-
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(KE):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / KE
+    e2e_ms, KE, h2d, d2h, h_out = e2e_time_ms(args, wl, append, decode, out, world)
     assert torch.isfinite(h_out.float()).all(), "non-finite decode output"
 
     if world > 1:
@@ -358,15 +461,22 @@ def run_ours(args, rank, world, dev):
         "tokens_per_s": round(world * c.num_seqs / (step_ms * 1e-3), 1),
         "pct_of_8TBs_nominal": round(100 * value / world / NOMINAL_HBM_GBS, 2),
         "decode_ms": round(decode_ms, 5),
+        "decode_timing": decode_timing,
         "bytes_per_step": {"decode": dec_b, "append": app_b},
         "roofline": {"bound": "hbm", "kernel": "paged_attention_decode (decode kernel" +
                      (", counter memset)" if args.plain_launch else ", counters left zero by the previous call)"),
                      "achieved": round(achieved, 2), "peak": peak, "peak_source": peak_src,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": profiled_traffic(c.name)},
-        "e2e": {"value": round(world * dec_b / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "e2e": {"value": round(world * (dec_b + app_b) / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "steps": KE, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h,
+                "how": "each step: one H2D copy of the step's packed inputs (query, new K/V, "
+                       "slot mapping, block table, lengths) from pinned host memory, "
+                       "paged_kv_append and paged_attention_decode through the Python binding, "
+                       "one D2H copy of the output to pinned host memory; copies run on two "
+                       "copy streams, double-buffered, so step k+1's inputs and step k-1's "
+                       "output move while step k computes"},
         "gpu_launches": K * launches_per_step,
         "timing": "CUDA graph replay of one step" if graph is not None else "eager launches",
         "decode_flags": "plain" if args.plain_launch else
@@ -632,6 +742,57 @@ def run_block_sizes(args, dev):
     return lines
 
 
+def run_decode_kernels(args, dev):
+    """The tensor-core decode kernel against the CUDA-core one (PKV_DECODE_FORCE_SIMT)
+    on the MHA (one query head per KV head) and the GQA (eight) workloads, each
+    timed alone per launch (events inside a CUDA graph), same inputs and split."""
+    peak, peak_src = measured_hbm_peak()
+    lines = []
+    for name in ("llama2_13b_mha", "gqa70b"):
+        cfg = W.CONFIGS[name]
+        wl = W.make_workload(cfg, device=dev)
+        c = wl.cfg
+        bt = torch.from_numpy(wl.block_table).to(dev)
+        sl = torch.from_numpy(wl.seq_lens).to(dev)
+        slots = torch.from_numpy(wl.slot_mapping).to(dev)
+        pkv.paged_kv_append(wl.new_key, wl.new_value, wl.k_cache, wl.v_cache, slots)
+        P = c.partition_size
+        nbytes = pkv.paged_attention_workspace_size(c.num_seqs, c.num_heads, c.num_kv_heads,
+                                                    c.head_dim, wl.max_seq_len, P)
+        ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+        out = torch.empty_like(wl.query)
+        dec, _ = step_bytes(wl)
+        for flags, kname in ((0, "decode_tc_kernel: mma.sync m16n8k16, S^T = K Q^T"),
+                             (pkv.PKV_DECODE_FORCE_SIMT, "decode_simt_kernel: CUDA cores")):
+            def call(f=flags):
+                pkv.paged_attention_decode(out, wl.query, wl.k_cache, wl.v_cache, bt, sl,
+                                           max_seq_len=wl.max_seq_len, scale=c.scale,
+                                           partition_size=P, workspace=ws,
+                                           flags=f | pkv.PKV_DECODE_ZEROED_WORKSPACE)
+            pkv.paged_attention_decode(out, wl.query, wl.k_cache, wl.v_cache, bt, sl,
+                                       max_seq_len=wl.max_seq_len, scale=c.scale,
+                                       partition_size=P, workspace=ws, flags=flags)
+            if args.no_graph:  # eager launches (e.g. under a profiler): warmup, then steps
+                ms, how = _event_time_ms(call, args.steps, args.warmup), "CUDA events, eager launches"
+            else:
+                ms, how = kernel_time_ms(lambda: None, call, reps=max(3, args.steps // 50))
+            assert pkv.pkv_device_status(clear=True) == 0, "device wait expired"
+            gbs = dec / ms / 1e6
+            lines.append({"metric": "paged decode attention HBM GB/s by kernel", "value": round(gbs, 1),
+                          "unit": "GB/s", "higher_is_better": True, "kernel": kname,
+                          "us_per_launch": round(ms * 1e3, 2), "timing": how,
+                          "group_size": c.num_heads // c.num_kv_heads, "dtype": c.q_dtype,
+                          "data": "synthetic",
+                          "config": {"workload": WORKLOAD_TEXT[name], "partition_size": P},
+                          "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
+                                       "peak_source": peak_src, "unit": "GB/s",
+                                       "frac": round(gbs / peak, 4), "traffic": None,
+                                       "bytes": dec}})
+        del wl, out, ws
+        torch.cuda.empty_cache()
+    return lines
+
+
 def measured_bf16_peak():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -714,10 +875,10 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=dev)
     try:
-        if args.op in ("blocks", "blocksize", "prefill"):
+        if args.op in ("blocks", "blocksize", "prefill", "kernels"):
             if rank == 0:
                 fn = {"blocks": run_block_ops, "blocksize": run_block_sizes,
-                      "prefill": run_prefill}[args.op]
+                      "prefill": run_prefill, "kernels": run_decode_kernels}[args.op]
                 for line in fn(args, dev):
                     print(json.dumps(line), flush=True)
             return

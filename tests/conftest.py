@@ -10,8 +10,24 @@ if ROOT not in sys.path:
 GOLDEN = os.path.join(ROOT, "tests", "golden")
 
 
+_PARITY_REPORT = []
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
+
+
+@pytest.fixture(scope="session")
+def parity_report():
+    """Lines (one per checked workload) printed in the session's summary."""
+    return _PARITY_REPORT
+
+
+def pytest_terminal_summary(terminalreporter):
+    if _PARITY_REPORT:
+        terminalreporter.write_sep("-", "parity against the fp64 oracle")
+        for line in _PARITY_REPORT:
+            terminalreporter.write_line(line)
 
 
 def read_golden(name: str) -> dict:

@@ -200,3 +200,15 @@ def test_fp8_cache_group_sizes(cuda_dev, Hq, Hkv, qdt, flags):
                                   lens=("uniform", 1, 400), prefix_len=0, partition_size=64,
                                   seed=91)
     _check(cfg, cuda_dev, flags=flags)
+
+
+@pytest.mark.parametrize("qdt", ["bf16", "f16", "f32"])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("flags", FLAGS)
+def test_fp8_cache_head_dims_and_query_dtypes(cuda_dev, qdt, D, flags):
+    # head_dim 64 over an E4M3 cache runs the CUDA-core kernel; so does an fp32
+    # query over an E4M3 cache (the new tokens are quantised from fp32 too).
+    cfg = C["fp8_prefix"].replace(num_seqs=6, num_heads=32, num_kv_heads=8, head_dim=D,
+                                  q_dtype=qdt, lens=("uniform", 1, 500), prefix_len=0,
+                                  partition_size=64, seed=93 + D)
+    _check(cfg, cuda_dev, flags=flags)
