@@ -743,15 +743,26 @@ def run_block_sizes(args, dev):
 
 
 def run_decode_kernels(args, dev):
-    """The tensor-core decode kernel against the CUDA-core one (PKV_DECODE_FORCE_SIMT)
-    on the MHA (one query head per KV head) and the GQA (eight) workloads, each
-    timed alone per launch (events inside a CUDA graph), same inputs and split."""
+    """Where the decode's products run: the TMA-fed kernel with Q K^T and P V on
+    the tensor cores (mma.sync) or on the CUDA cores (fp32 FMA), and the plain
+    CUDA-core kernel without TMA staging (PKV_DECODE_FORCE_SIMT), on the MHA
+    workload (one query head per KV head), the 70B-class shape with 4 query heads
+    per KV head, and the 70B-class GQA workload (8). Each timed alone per launch
+    (events inside a CUDA graph), same inputs and split."""
     peak, peak_src = measured_hbm_peak()
     lines = []
-    for name in ("llama2_13b_mha", "gqa70b"):
-        cfg = W.CONFIGS[name]
+    cases = [("llama2_13b_mha", W.CONFIGS["llama2_13b_mha"]),
+             ("gqa70b_g4", W.CONFIGS["gqa70b"].replace(num_heads=32)),
+             ("gqa70b", W.CONFIGS["gqa70b"])]
+    kernels = [(pkv.PKV_DECODE_TENSOR_CORES, "decode_tc_kernel, products on the tensor cores "
+                                             "(mma.sync m16n8k16, S^T = K Q^T)"),
+               (pkv.PKV_DECODE_CUDA_CORES, "decode_tc_kernel, products on the CUDA cores "
+                                           "(fp32 FMA, lanes over head_dim)"),
+               (pkv.PKV_DECODE_FORCE_SIMT, "decode_simt_kernel: CUDA cores, plain loads (no TMA)")]
+    for name, cfg in cases:
         wl = W.make_workload(cfg, device=dev)
         c = wl.cfg
+        g = c.num_heads // c.num_kv_heads
         bt = torch.from_numpy(wl.block_table).to(dev)
         sl = torch.from_numpy(wl.seq_lens).to(dev)
         slots = torch.from_numpy(wl.slot_mapping).to(dev)
@@ -762,8 +773,9 @@ def run_decode_kernels(args, dev):
         ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
         out = torch.empty_like(wl.query)
         dec, _ = step_bytes(wl)
-        for flags, kname in ((0, "decode_tc_kernel: mma.sync m16n8k16, S^T = K Q^T"),
-                             (pkv.PKV_DECODE_FORCE_SIMT, "decode_simt_kernel: CUDA cores")):
+        for flags, kname in kernels:
+            if flags == pkv.PKV_DECODE_CUDA_CORES and g > 4:
+                continue  # the CUDA-core products serve groups of up to 4 heads
             def call(f=flags):
                 pkv.paged_attention_decode(out, wl.query, wl.k_cache, wl.v_cache, bt, sl,
                                            max_seq_len=wl.max_seq_len, scale=c.scale,
@@ -778,12 +790,12 @@ def run_decode_kernels(args, dev):
                 ms, how = kernel_time_ms(lambda: None, call, reps=max(3, args.steps // 50))
             assert pkv.pkv_device_status(clear=True) == 0, "device wait expired"
             gbs = dec / ms / 1e6
+            text = WORKLOAD_TEXT.get(name, WORKLOAD_TEXT["gqa70b"].replace("64 q / 8 KV", "32 q / 8 KV"))
             lines.append({"metric": "paged decode attention HBM GB/s by kernel", "value": round(gbs, 1),
                           "unit": "GB/s", "higher_is_better": True, "kernel": kname,
                           "us_per_launch": round(ms * 1e3, 2), "timing": how,
-                          "group_size": c.num_heads // c.num_kv_heads, "dtype": c.q_dtype,
-                          "data": "synthetic",
-                          "config": {"workload": WORKLOAD_TEXT[name], "partition_size": P},
+                          "group_size": g, "dtype": c.q_dtype, "data": "synthetic",
+                          "config": {"workload": text, "partition_size": P},
                           "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
                                        "peak_source": peak_src, "unit": "GB/s",
                                        "frac": round(gbs / peak, 4), "traffic": None,

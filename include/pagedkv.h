@@ -80,6 +80,16 @@ typedef enum {
  * tokens) and does not touch `out` or the workspace. Without a preceding
  * kernel, or on the CUDA-core path, it changes nothing. */
 #define PKV_DECODE_EARLY_START 4u
+/* Where the TMA-fed decode kernel (16-bit caches, head_dim 64/128) runs its
+ * Q K^T and P V products. By default every group size uses the tensor cores
+ * (mma.sync, tokens on M): measured on B200, even one query head per KV head
+ * runs faster there than with fp32 FMA on the CUDA cores, since the CUDA-core
+ * form needs several times the instructions. CUDA_CORES selects the CUDA-core
+ * form for groups of up to 4 heads (wider groups stay on the tensor cores);
+ * TENSOR_CORES states the default. Both set is an error. Comparison and testing
+ * knobs. */
+#define PKV_DECODE_TENSOR_CORES 8u
+#define PKV_DECODE_CUDA_CORES 16u
 
 /*
  * paged_kv_append — write new tokens' K/V into their slots ("reshape and cache").

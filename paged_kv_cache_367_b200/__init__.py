@@ -20,7 +20,8 @@ __all__ = ["paged_kv_append", "paged_attention_decode", "paged_attention_workspa
            "pkv_device_status", "pkv_selftest_expired_wait", "pkv_status_string", "pkv_version",
            "load_library", "PagedKVError",
            "PKV_F32", "PKV_F16", "PKV_BF16", "PKV_FP8_E4M3", "PKV_DECODE_FORCE_SIMT",
-           "PKV_DECODE_ZEROED_WORKSPACE", "PKV_DECODE_EARLY_START", "PKV_PREFILL_MMA_SYNC",
+           "PKV_DECODE_ZEROED_WORKSPACE", "PKV_DECODE_EARLY_START", "PKV_DECODE_TENSOR_CORES",
+           "PKV_DECODE_CUDA_CORES", "PKV_PREFILL_MMA_SYNC",
            "LIB_PATH", "EXPORTED_SYMBOLS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedkv.so")
@@ -29,6 +30,8 @@ PKV_F32, PKV_F16, PKV_BF16, PKV_FP8_E4M3 = 0, 1, 2, 3
 PKV_DECODE_FORCE_SIMT = 1
 PKV_DECODE_ZEROED_WORKSPACE = 2
 PKV_DECODE_EARLY_START = 4
+PKV_DECODE_TENSOR_CORES = 8
+PKV_DECODE_CUDA_CORES = 16
 PKV_PREFILL_MMA_SYNC = 1
 
 EXPORTED_SYMBOLS = ("paged_kv_append", "paged_attention_workspace_size",

@@ -250,10 +250,196 @@ struct ChunkDesc {
 };
 constexpr int kFirst = 1, kLast = 2, kEnd = 4;
 
+// 16-bit pair (bf16 or f16, low element first) to two floats.
+template <typename T> __device__ __forceinline__ float2 pair_to_f32(uint32_t v);
+template <> __device__ __forceinline__ float2 pair_to_f32<__nv_bfloat16>(uint32_t v) {
+  return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+template <> __device__ __forceinline__ float2 pair_to_f32<__half>(uint32_t v) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&v));
+}
+
+// Consumer warps on the CUDA cores, for narrow groups (g <= G query heads per
+// KV head, where Q K^T is a matrix-vector product rather than a dense
+// contraction). Warp w takes tokens [16 w, 16 w + 16) of each chunk, as the
+// tensor-core consumers do; inside the warp, LPT = D / 8 lanes hold one token's
+// row, eight dimensions (one 16-byte unit of the 128B-swizzled tile) each, so
+// TPS = 32 / LPT tokens are read per step with conflict-free 16-byte shared
+// loads. A token's score is the LPT-lane sum of the lanes' partial dot
+// products (xor shuffles); the online softmax runs per 16-token slice in fp32
+// (P is not rounded); each lane accumulates P V for its eight dimensions over
+// its tokens, and the TPS lane groups are summed at the end of a segment.
+// Slots past the segment's end are neither read nor counted.
+template <typename T, int D, int G, int NS, int H>
+__device__ void consumer_cuda_cores(const DecodeParams& prm, uint8_t* ring, int stage_bytes,
+                                    int kv_bytes, const ChunkDesc* desc, uint64_t* full,
+                                    uint64_t* empty, float* red, int red_floats, int red_o,
+                                    ChunkDesc* hdesc, uint64_t* rfull, uint64_t* rempty,
+                                    volatile int* abort, int w, int lane) {
+  constexpr int LPT = D / 8, TPS = 32 / LPT, STEPS = 16 / TPS;
+  const int grp = lane / LPT, ln = lane % LPT;
+  const int bs = prm.block_size, g = prm.num_heads / prm.num_kv_heads;
+  const int tile = bs * D * 2;                // bytes of one (block, head) tile
+  const int plane = ln >> 3, unit = ln & 7;   // 128-byte piece of the row, 16-byte unit in it
+  const float sscale = prm.score_scale;
+  uint32_t kc = 0;
+  int sidx = 0;
+  float q[G][8], acc[G][8], m[G], l[G];
+  for (;;) {
+    const int stage = (int)(kc % NS);
+    const uint32_t phase = (kc / NS) & 1u;
+    ++kc;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(full + stage, phase, abort));
+    if (!ok) break;
+    const ChunkDesc d = desc[stage];
+    if (d.flags & kEnd) break;
+    const uint8_t* st = ring + stage * stage_bytes;
+    if (d.flags & kFirst) {
+      // This lane's eight dimensions of each query row, pre-scaled.
+      const uint8_t* qs = st + 2 * kv_bytes;
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        m[j] = -INFINITY;
+        l[j] = 0.f;
+        uint4 raw = make_uint4(0, 0, 0, 0);
+        if (j < g) raw = *reinterpret_cast<const uint4*>(qs + (j * D + 8 * ln) * 2);
+        const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = pair_to_f32<T>(u[k]);
+          q[j][2 * k] = f.x * sscale;
+          q[j][2 * k + 1] = f.y * sscale;
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[j][k] = 0.f;
+      }
+    }
+    const int nv = min(16, max(0, d.t1 - (d.c0 + 16 * w)));
+    if (nv > 0) {
+      // Scores of this lane group's tokens (base-2 domain).
+      float sc[G][STEPS];
+#pragma unroll
+      for (int s = 0; s < STEPS; ++s) {
+        const int tw = s * TPS + grp, t = 16 * w + tw;
+        const int tt = t % bs;
+        const uint32_t off = (uint32_t)((t / bs) * tile + plane * (bs * 128) + tt * 128 +
+                                        ((unit ^ (tt & 7)) << 4));
+        uint4 raw = make_uint4(0, 0, 0, 0);
+        if (tw < nv) raw = *reinterpret_cast<const uint4*>(st + off);
+        const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
+        float kf[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = pair_to_f32<T>(u[k]);
+          kf[2 * k] = f.x;
+          kf[2 * k + 1] = f.y;
+        }
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+          float dot = 0.f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) dot = fmaf(q[j][k], kf[k], dot);
+#pragma unroll
+          for (int o = LPT / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+          sc[j][s] = tw < nv ? dot : -INFINITY;
+        }
+      }
+      // Online softmax over the warp's slice of the chunk.
+      float p[G][STEPS];
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        float mx = sc[j][0];
+#pragma unroll
+        for (int s = 1; s < STEPS; ++s) mx = fmaxf(mx, sc[j][s]);
+#pragma unroll
+        for (int o = LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float mn = fmaxf(m[j], mx);
+        const float mu = mn == -INFINITY ? 0.f : mn;
+        const float alpha = fast_exp2(m[j] - mu);
+        m[j] = mn;
+        float ls = 0.f;
+#pragma unroll
+        for (int s = 0; s < STEPS; ++s) {
+          p[j][s] = fast_exp2(sc[j][s] - mu);
+          ls += p[j][s];
+        }
+        l[j] = l[j] * alpha + ls;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[j][k] *= alpha;
+      }
+      // P V for this lane's eight dimensions.
+#pragma unroll
+      for (int s = 0; s < STEPS; ++s) {
+        const int tw = s * TPS + grp, t = 16 * w + tw;
+        const int tt = t % bs;
+        const uint32_t off = (uint32_t)((t / bs) * tile + plane * (bs * 128) + tt * 128 +
+                                        ((unit ^ (tt & 7)) << 4));
+        if (tw < nv) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(st + kv_bytes + off);
+          const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = pair_to_f32<T>(u[k]);
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+              acc[j][2 * k] = fmaf(p[j][s], f.x, acc[j][2 * k]);
+              acc[j][2 * k + 1] = fmaf(p[j][s], f.y, acc[j][2 * k + 1]);
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty + stage);
+    if (d.flags & kLast) {
+      // ---- hand the warp's state to the epilogue warp ----
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+#pragma unroll
+        for (int o = LPT; o < 32; o <<= 1) {
+          l[j] += __shfl_xor_sync(0xffffffffu, l[j], o);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[j][k] += __shfl_xor_sync(0xffffffffu, acc[j][k], o);
+        }
+      }
+      const int rb = sidx & 1;
+      const uint32_t use = (uint32_t)(sidx >> 1);
+      ++sidx;
+      mbar_wait(rempty + rb, (use & 1u) ^ 1u, abort);  // read two segments ago
+      if (w == 0 && lane == 0) hdesc[rb] = d;
+      float* ro = red + rb * red_floats + (w * H) * D;
+      float* rm = red + rb * red_floats + red_o;
+      float* rl = rm + 4 * H;
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        if (j < g && grp == 0) {
+          *reinterpret_cast<float4*>(ro + j * D + 8 * ln) =
+              make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+          *reinterpret_cast<float4*>(ro + j * D + 8 * ln + 4) =
+              make_float4(acc[j][4], acc[j][5], acc[j][6], acc[j][7]);
+        }
+        if (j < g && lane == 0) {
+          rm[w * H + j] = m[j];
+          rl[w * H + j] = l[j];
+        }
+      }
+      mbar_arrive(rfull + rb);
+    }
+  }
+  // Tell the epilogue warp there is nothing more.
+  const int rb = sidx & 1;
+  const uint32_t use = (uint32_t)(sidx >> 1);
+  mbar_wait(rempty + rb, (use & 1u) ^ 1u, abort);
+  if (w == 0 && lane == 0) hdesc[rb].flags = kEnd;
+  mbar_arrive(rfull + rb);
+}
+
 // T: query/output type (bf16 or f16). F8: the cache holds E4M3 codes; the
 // products then run in f16 (exact for E4M3 values) with k_scale folded into the
 // score scale and v_scale applied to the output.
-template <typename T, int D, int NT, int NS, int MINB, bool F8>
+// CC > 0: the products run on the CUDA cores (consumer_cuda_cores) for groups
+// of at most CC query heads; 16-bit caches only.
+template <typename T, int D, int NT, int NS, int MINB, bool F8, int CC>
 __global__ void __launch_bounds__(kThreads, MINB)
     decode_tc_kernel(const DecodeParams prm, const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v) {
@@ -542,6 +728,13 @@ __global__ void __launch_bounds__(kThreads, MINB)
 
   // -------------------------------------------------------------- consumers ----
   // Warp w takes tokens [16 w, 16 w + 16) of every 64-token chunk.
+  if constexpr (CC > 0) {
+    static_assert(!F8, "CUDA-core products: 16-bit caches");
+    consumer_cuda_cores<T, D, CC, NS, H>(prm, ring, C::kStage, C::kKV, desc, full, empty, red,
+                                         C::kRed / 4, C::kRedO, hdesc, rfull, rempty, abort, warp,
+                                         lane);
+    return;
+  }
   const int w = warp;
   const int g0 = lane >> 2, cq = lane & 3, x7 = lane & 7;
   const int kt = 16 * w + ((lane >> 3) & 1) * 8 + x7;  // token row this lane addresses for K
@@ -829,6 +1022,14 @@ int tc_timeout_flag(bool clear, int* value) {
   return 0;
 }
 
+// Largest group whose products run on the CUDA cores by default (see
+// launch_decode_tc): none. Measured on B200 with the same TMA pipeline, the
+// CUDA-core products take 2.8x the instructions of mma.sync at one query head
+// per KV head (the dot products need per-element conversions and cross-lane
+// sums), hold each stage longer, and run the MHA decode 1.46x slower (DRAM
+// throughput 52% against 76%); at four heads per KV head 2.2x slower.
+constexpr int kCudaCoreMaxGroup = 0;
+
 bool tc_supported(int q_dtype, int cache_dtype, int head_dim, int group) {
   if (q_dtype != PKV_BF16 && q_dtype != PKV_F16) return false;
   if (group < 1 || group > 16) return false;
@@ -836,12 +1037,12 @@ bool tc_supported(int q_dtype, int cache_dtype, int head_dim, int group) {
   return cache_dtype == PKV_FP8_E4M3 && head_dim == 128;
 }
 
-template <typename T, int D, int NT, int NS, int MINB, bool F8>
+template <typename T, int D, int NT, int NS, int MINB, bool F8, int CC>
 static cudaError_t launch_tc_t(const DecodeParams& prm, const CUtensorMap& mk,
                                const CUtensorMap& mv, int max_ctas, int num_sms,
                                bool early_start, cudaStream_t stream) {
   using C = tc::Cfg<D, NT, NS, F8 ? 1 : 2>;
-  auto kernel = tc::decode_tc_kernel<T, D, NT, NS, MINB, F8>;
+  auto kernel = tc::decode_tc_kernel<T, D, NT, NS, MINB, F8, CC>;
   // The shared-memory opt-in is a per-device setting: done, and the residency
   // queried, once per device.
   static std::atomic<int> occ_of[64];
@@ -888,23 +1089,38 @@ static cudaError_t launch_tc_t(const DecodeParams& prm, const CUtensorMap& mk,
   return cudaGetLastError();
 }
 
+// cc > 0: products on the CUDA cores for a group of at most cc heads (1, 2, 4).
 template <typename T, int D, bool F8>
 static cudaError_t launch_tc_d(const DecodeParams& prm, const CUtensorMap& mk,
                                const CUtensorMap& mv, int max_ctas, int num_sms,
-                               bool early_start, cudaStream_t stream) {
+                               bool early_start, int cc, cudaStream_t stream) {
   // Two CTAs per SM (two producers keep more copies in flight than one) where
   // shared memory allows; head_dim 128 with more than 8 heads per group runs one.
   const int g = prm.num_heads / prm.num_kv_heads;
   // E4M3 stages are half the size: four of them per CTA.
   constexpr int kNS = F8 ? 4 : (D == 128 ? 2 : 4);
-  if (g <= 8) return launch_tc_t<T, D, 1, kNS, 2, F8>(prm, mk, mv, max_ctas, num_sms, early_start, stream);
-  if (D == 64 || F8) return launch_tc_t<T, D, 2, 4, 2, F8>(prm, mk, mv, max_ctas, num_sms, early_start, stream);
-  return launch_tc_t<T, D, 2, 4, 1, F8>(prm, mk, mv, max_ctas, num_sms, early_start, stream);
+  if constexpr (!F8) {
+    if (cc == 1)
+      return launch_tc_t<T, D, 1, kNS, 2, F8, 1>(prm, mk, mv, max_ctas, num_sms, early_start, stream);
+    if (cc == 2)
+      return launch_tc_t<T, D, 1, kNS, 2, F8, 2>(prm, mk, mv, max_ctas, num_sms, early_start, stream);
+    if (cc == 4)
+      return launch_tc_t<T, D, 1, kNS, 2, F8, 4>(prm, mk, mv, max_ctas, num_sms, early_start, stream);
+  }
+  if (g <= 8) return launch_tc_t<T, D, 1, kNS, 2, F8, 0>(prm, mk, mv, max_ctas, num_sms, early_start, stream);
+  if (D == 64 || F8) return launch_tc_t<T, D, 2, 4, 2, F8, 0>(prm, mk, mv, max_ctas, num_sms, early_start, stream);
+  return launch_tc_t<T, D, 2, 4, 1, F8, 0>(prm, mk, mv, max_ctas, num_sms, early_start, stream);
 }
 
 cudaError_t launch_decode_tc(const DecodeParams& prm, int q_dtype, int cache_dtype, int max_ctas,
-                             int num_sms, bool early_start, cudaStream_t stream) {
+                             int num_sms, bool early_start, int products, cudaStream_t stream) {
   const bool f8 = cache_dtype == PKV_FP8_E4M3;
+  // Where the products run: the CUDA cores for narrow groups of a 16-bit cache
+  // (by default up to kCudaCoreMaxGroup heads; products > 0 forces them up to
+  // 4), else the tensor cores (products < 0 forces them).
+  const int g = prm.num_heads / prm.num_kv_heads;
+  const int cc_max = products > 0 ? 4 : products < 0 ? 0 : kCudaCoreMaxGroup;
+  const int cc = f8 || g > cc_max ? 0 : (g == 1 ? 1 : g == 2 ? 2 : 4);
   const CUtensorMapDataType dt = f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                  : q_dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -917,16 +1133,16 @@ cudaError_t launch_decode_tc(const DecodeParams& prm, int q_dtype, int cache_dty
     return cudaErrorInvalidValue;
   if (f8) {
     return q_dtype == PKV_BF16
-               ? launch_tc_d<__nv_bfloat16, 128, true>(prm, mk, mv, max_ctas, num_sms, early_start, stream)
-               : launch_tc_d<__half, 128, true>(prm, mk, mv, max_ctas, num_sms, early_start, stream);
+               ? launch_tc_d<__nv_bfloat16, 128, true>(prm, mk, mv, max_ctas, num_sms, early_start, cc, stream)
+               : launch_tc_d<__half, 128, true>(prm, mk, mv, max_ctas, num_sms, early_start, cc, stream);
   }
   if (q_dtype == PKV_BF16) {
     return prm.head_dim == 128
-               ? launch_tc_d<__nv_bfloat16, 128, false>(prm, mk, mv, max_ctas, num_sms, early_start, stream)
-               : launch_tc_d<__nv_bfloat16, 64, false>(prm, mk, mv, max_ctas, num_sms, early_start, stream);
+               ? launch_tc_d<__nv_bfloat16, 128, false>(prm, mk, mv, max_ctas, num_sms, early_start, cc, stream)
+               : launch_tc_d<__nv_bfloat16, 64, false>(prm, mk, mv, max_ctas, num_sms, early_start, cc, stream);
   }
-  return prm.head_dim == 128 ? launch_tc_d<__half, 128, false>(prm, mk, mv, max_ctas, num_sms, early_start, stream)
-                             : launch_tc_d<__half, 64, false>(prm, mk, mv, max_ctas, num_sms, early_start, stream);
+  return prm.head_dim == 128 ? launch_tc_d<__half, 128, false>(prm, mk, mv, max_ctas, num_sms, early_start, cc, stream)
+                             : launch_tc_d<__half, 64, false>(prm, mk, mv, max_ctas, num_sms, early_start, cc, stream);
 }
 
 }  // namespace pkv

@@ -13,7 +13,8 @@ cudaError_t launch_decode_simt(const DecodeParams& prm, int q_dtype, int cache_d
                                int max_ctas, int num_sms, cudaStream_t stream);
 bool tc_supported(int q_dtype, int cache_dtype, int head_dim, int group);
 cudaError_t launch_decode_tc(const DecodeParams& prm, int q_dtype, int cache_dtype,
-                             int max_ctas, int num_sms, bool early_start, cudaStream_t stream);
+                             int max_ctas, int num_sms, bool early_start, int products,
+                             cudaStream_t stream);
 int tc_timeout_flag(bool clear, int* value);
 int pf_timeout_flag(bool clear, int* value);
 int simt_status_flag(bool clear, int* value);
@@ -146,7 +147,9 @@ int paged_attention_decode(void* out, const void* query, const void* k_cache,
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 ||
       max_blocks_per_seq <= 0 || num_blocks <= 0 || max_seq_len < 0 || partition_size < 0 ||
       max_ctas < 0 || !isfinite(scale) ||
-      (flags & ~(PKV_DECODE_FORCE_SIMT | PKV_DECODE_ZEROED_WORKSPACE | PKV_DECODE_EARLY_START)))
+      (flags & ~(PKV_DECODE_FORCE_SIMT | PKV_DECODE_ZEROED_WORKSPACE | PKV_DECODE_EARLY_START |
+                 PKV_DECODE_TENSOR_CORES | PKV_DECODE_CUDA_CORES)) ||
+      ((flags & PKV_DECODE_TENSOR_CORES) && (flags & PKV_DECODE_CUDA_CORES)))
     return PKV_ERR_SHAPE;
   if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
   if (block_size != 8 && block_size != 16 && block_size != 32) return PKV_ERR_UNSUPPORTED;
@@ -210,7 +213,9 @@ int paged_attention_decode(void* out, const void* query, const void* k_cache,
   }
   if (!(flags & PKV_DECODE_FORCE_SIMT) && tc_supported(q_dtype, cache_dtype, head_dim, group))
     e = launch_decode_tc(prm, q_dtype, cache_dtype, max_ctas, sms,
-                         (flags & PKV_DECODE_EARLY_START) != 0, st);
+                         (flags & PKV_DECODE_EARLY_START) != 0,
+                         (flags & PKV_DECODE_CUDA_CORES) ? 1 : (flags & PKV_DECODE_TENSOR_CORES) ? -1 : 0,
+                         st);
   else
     e = launch_decode_simt(prm, q_dtype, cache_dtype, max_ctas, sms, st);
   if (e != cudaSuccess) return PKV_ERR_CUDA;

@@ -212,3 +212,34 @@ def test_fp8_cache_head_dims_and_query_dtypes(cuda_dev, qdt, D, flags):
                                   q_dtype=qdt, lens=("uniform", 1, 500), prefix_len=0,
                                   partition_size=64, seed=93 + D)
     _check(cfg, cuda_dev, flags=flags)
+
+
+PRODUCTS = [pkv.PKV_DECODE_TENSOR_CORES, pkv.PKV_DECODE_CUDA_CORES]
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 8), (12, 4), (16, 4), (32, 4), (16, 16)])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+@pytest.mark.parametrize("flags", PRODUCTS)
+def test_products_on_tensor_or_cuda_cores(cuda_dev, Hq, Hkv, D, dt, flags):
+    # The TMA-fed kernel with its products on the tensor cores (mma.sync) or on
+    # the CUDA cores (groups of up to 4 heads; wider ones stay on the tensor
+    # cores), split and unsplit sequences, ragged tails.
+    cfg = C["gqa70b"].replace(num_seqs=7, num_heads=Hq, num_kv_heads=Hkv, head_dim=D, q_dtype=dt,
+                              cache_dtype=dt, lens=("uniform", 1, 700), partition_size=128,
+                              seed=Hq * 3 + Hkv + D)
+    _check(cfg, cuda_dev, flags=flags)
+
+
+@pytest.mark.parametrize("bs", [8, 16, 32])
+@pytest.mark.parametrize("flags", PRODUCTS)
+def test_mha_products_block_sizes(cuda_dev, bs, flags):
+    _check(SMALL["llama2_13b_mha"].replace(block_size=bs), cuda_dev, flags=flags)
+
+
+@pytest.mark.parametrize("flags", PRODUCTS)
+def test_mha_products_single_token_exact(cuda_dev, flags):
+    cfg = C["llama2_13b_mha"].replace(num_seqs=3, lens=("fixed", [1, 1, 1]), seed=22)
+    wl = W.make_workload(cfg, device=cuda_dev)
+    out = gpu_step(wl, cuda_dev, flags=flags)
+    assert torch.equal(out, wl.new_value)

@@ -199,5 +199,6 @@ def test_prefill_rejects_bad_arguments(lib, kw, code):
 
 
 def test_decode_rejects_unknown_flags(lib):
-    assert decode(lib, flags=8) == ESHAPE
+    assert decode(lib, flags=32) == ESHAPE
     assert decode(lib, flags=1 << 31) == ESHAPE
+    assert decode(lib, flags=8 | 16) == ESHAPE          # tensor cores and CUDA cores at once
