@@ -10,7 +10,8 @@
 //  * One CTA per SM (persistent) takes a balanced, contiguous share of the
 //    (sequence, KV head) work (schedule.cuh).
 //  * A producer warp walks the same segments and streams 64-token chunks of K
-//    and V into a ring of shared-memory stages. Each physical block is one TMA
+//    and V into a ring of shared-memory stages (marked evict-first in L2: each
+//    tile is read once). Each physical block is one TMA
 //    tensor copy: the pool [num_blocks, bs, Hkv, D] is described as a 5-D tensor
 //    (d_lo 64, token, d_hi, head, block) so a (block, head) tile lands as
 //    128-byte rows with the 128B swizzle; a block id outside the pool is out of
@@ -489,9 +490,9 @@ __global__ void __launch_bounds__(kThreads, MINB)
     // ------------------------------------------------------------ producer ----
     // Streams the chunks of every segment of this CTA's static range, then of
     // each dynamic range it takes, in order, into the ring, with a descriptor
-    // per chunk. The block ids of the next segment are loaded while the current
-    // one is issued; the lane holding a block's id issues that block's K and V
-    // tile copies. A final descriptor marks the end.
+    // per chunk. The next segment is found, and its block ids loaded, once the
+    // current segment's first chunk is issued; the lane holding a block's id
+    // issues that block's K and V tile copies. A final descriptor marks the end.
     uint32_t kc = 0;  // chunk counter: stage kc % NS, phase (kc / NS) & 1
     uint32_t armed = 0, last_parity = 0;
     bool ok = true, waited = false;
@@ -500,6 +501,9 @@ __global__ void __launch_bounds__(kThreads, MINB)
     int ci = sched->d_i;            // forward cursor for dynamic ranges
     int64_t cbase = sched->d_base;
     int* const dyn_counter = prm.ws_done + (int64_t)prm.num_seqs * Hkv;
+    // K/V tiles are read once: evicted from L2 first, so the lengths, block
+    // tables, query rows and split partials stay there.
+    const uint64_t kv_policy = l2_evict_first_policy();
     for (;;) {
       Segment seg, nseg;
       bool have = walker.next(seg);
@@ -514,13 +518,8 @@ __global__ void __launch_bounds__(kThreads, MINB)
         const int lb0 = seg.t0 / bs;
         const int nlb = (seg.t1 + bs - 1) / bs - lb0;
         int nxt = lane + 32 < nlb ? __ldg(bt + lb0 + 32 + lane) : 0;
-        const bool have_next = walker.next(nseg);
+        bool have_next = false;
         int ncur = 0;
-        if (have_next) {
-          const int32_t* nbt = prm.block_table + (int64_t)nseg.seq * prm.max_blocks_per_seq;
-          const int nlb0 = nseg.t0 / bs, nnlb = (nseg.t1 + bs - 1) / bs - nlb0;
-          ncur = lane < nnlb ? __ldg(nbt + nlb0 + lane) : 0;
-        }
         int batch = 0;
         for (int c0 = seg.t0; c0 < seg.t1; c0 += kChunk, ++kc) {
           const int stage = (int)(kc % NS);
@@ -566,12 +565,21 @@ __global__ void __launch_bounds__(kThreads, MINB)
             // An id outside the pool reads as zeros (the copy's bounds fill);
             // it is also reported in the status word (bit 1).
             if (cur < 0 || (int64_t)cur >= prm.num_blocks) atomicOr(&g_tc_timeout, 2);
-            tma_load_5d(st + b * tile, &tmap_k, 0, 0, 0, seg.head, cur, full + stage);
-            tma_load_5d(st + C::kKV + b * tile, &tmap_v, 0, 0, 0, seg.head, cur, full + stage);
+            tma_load_5d_hint(st + b * tile, &tmap_k, 0, 0, 0, seg.head, cur, full + stage, kv_policy);
+            tma_load_5d_hint(st + C::kKV + b * tile, &tmap_v, 0, 0, 0, seg.head, cur, full + stage,
+                             kv_policy);
           }
           if (ok) {
             armed |= 1u << stage;
             last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          }
+          if (first) {
+            have_next = walker.next(nseg);
+            if (have_next) {
+              const int32_t* nbt = prm.block_table + (int64_t)nseg.seq * prm.max_blocks_per_seq;
+              const int nlb0 = nseg.t0 / bs, nnlb = (nseg.t1 + bs - 1) / bs - nlb0;
+              ncur = lane < nnlb ? __ldg(nbt + nlb0 + lane) : 0;
+            }
           }
         }
         seg = nseg;
