@@ -588,7 +588,14 @@ __global__ void __launch_bounds__(kThreads, MINB)
       }
       if (!ok || cuts.Rd == 0) break;
       int64_t nr = 0;
-      if (lane == 0) nr = cuts.G + atomicAdd(dyn_counter, 1);
+      if (lane == 0) {
+        const int64_t taken = atomicAdd(dyn_counter, 1);
+        // Every CTA asks until it is refused once, so the counter ends at Rd + G:
+        // the last refusal (no other CTA asks after it) leaves it at zero for
+        // the next call on this workspace.
+        if (taken == cuts.Rd + cuts.G - 1) atomicExch(dyn_counter, 0);
+        nr = cuts.G + taken;
+      }
       nr = __shfl_sync(0xffffffffu, nr, 0);
       if (nr >= cuts.R()) break;
       r = nr;
@@ -1070,16 +1077,20 @@ static cudaError_t launch_tc_t(const DecodeParams& prm, const CUtensorMap& mk,
   int grid = occ * num_sms;
   if (grid > kMaxRanges) grid = kMaxRanges;
   if (max_ctas > 0 && max_ctas < grid) grid = max_ctas;
-  // Dynamic ranges (work handed out at run time to whichever CTA is free) are
-  // supported by the kernel but off: on the measured workloads the extra pieces
-  // they cut, with their merges and per-range start-up, cost more than the
-  // tail they save. kDynRanges > 0 turns them on (up to kMaxRanges in total).
-  constexpr int kDynRanges = 0;
+  // Dynamic ranges: the last (1024 - kStaticShare) / 1024 of the work cut into
+  // kDynPerCta4 / 4 ranges per CTA, handed out at run time to whichever CTA is
+  // free; only where units may be split (a workspace exists). Off: CTAs do
+  // stream at unequal rates (with static ranges the last one finishes about
+  // 7 us after the median on the 70B-class workload), but measured on B200 the
+  // dynamic ranges cost more than that: each starts with a search of the
+  // lengths and a fresh block-table read, and they cut long units into many
+  // small pieces whose merges land at the end (116 against 110 us there, 333
+  // against 317 us on the long-context workload).
+  constexpr int kDynPerCta4 = 0, kStaticShare = 870;
   DecodeParams p = prm;
-  p.dyn_ranges = prm.ws_done && kDynRanges > 0
-                     ? (kDynRanges < kMaxRanges - grid ? kDynRanges : kMaxRanges - grid)
-                     : 0;
-  p.static_share = 870;
+  const int dyn = grid * kDynPerCta4 / 4;
+  p.dyn_ranges = prm.ws_done ? (dyn < kMaxRanges - grid ? dyn : kMaxRanges - grid) : 0;
+  p.static_share = kStaticShare;
   if (early_start) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
