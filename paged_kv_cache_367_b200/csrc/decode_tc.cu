@@ -109,7 +109,7 @@ __device__ void warp_merge_unit(const DecodeParams& prm, const Cuts& cu, int64_t
   const int Hq = prm.num_heads, g = Hq / prm.num_kv_heads;
   const int rowf = g * D;                 // floats of one piece's partial rows
   const int B = stage_floats / rowf;      // pieces per staging round (>= 4)
-  const int64_t nparts = (s.len + P - 1) / P;
+  const int64_t nparts = div_nn(s.len + P - 1, P);
   const int64_t r0 = cu.owner(s.first);
   const int64_t r1 = cu.owner(s.first + (nparts - 1) * P);
   // Writes the slots of pieces [b0, b0 + 32) to wslot; returns the piece count.

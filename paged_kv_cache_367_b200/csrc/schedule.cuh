@@ -57,13 +57,21 @@ struct DecodeParams {
 
 constexpr int64_t kNoSplit = int64_t(1) << 30;
 
+// a / b for a >= 0, b > 0: a 32-bit division when both fit (a 64-bit one is
+// several times longer on the GPU, and the set-up runs a chain of them).
+__host__ __device__ __forceinline__ int64_t div_nn(int64_t a, int64_t b) {
+  if ((((uint64_t)a | (uint64_t)b) >> 32) == 0) return (int64_t)((uint32_t)a / (uint32_t)b);
+  return a / b;
+}
+
 __host__ __device__ __forceinline__ int clamp_len(int L, int cap) {
   return L < 0 ? 0 : (L > cap ? cap : L);
 }
 
 // Work of a unit of L tokens (0 for an empty unit).
 __host__ __device__ __forceinline__ int64_t unit_work(int L, int cost, int round) {
-  return L > 0 ? (int64_t)(L + round - 1) / round * round + cost : 0;
+  return L > 0 ? (int64_t)(((uint32_t)L + (uint32_t)round - 1u) / (uint32_t)round * (uint32_t)round) + cost
+               : 0;
 }
 
 __host__ __device__ __forceinline__ int load_len(const int32_t* p) {
@@ -82,13 +90,13 @@ struct Cuts {
   __host__ __device__ int64_t R() const { return G + Rd; }
   // First work offset of range r (r in [0, R]).
   __host__ __device__ int64_t lo(int64_t r) const {
-    if (r <= G) return (Ws * r + G - 1) / G;
-    return Ws + ((W - Ws) * (r - G) + Rd - 1) / Rd;
+    if (r <= G) return div_nn(Ws * r + G - 1, G);
+    return Ws + div_nn((W - Ws) * (r - G) + Rd - 1, Rd);
   }
   // Range holding offset off (0 <= off < W).
   __host__ __device__ int64_t owner(int64_t off) const {
-    if (off < Ws) return off * G / Ws;
-    return G + (off - Ws) * Rd / (W - Ws);
+    if (off < Ws) return div_nn(off * G, Ws);
+    return G + div_nn((off - Ws) * Rd, W - Ws);
   }
 };
 
@@ -114,7 +122,7 @@ struct Segment {
 __host__ __device__ __forceinline__ int64_t range_first_part(const Cuts& cu, int64_t r,
                                                              int64_t first, int64_t P) {
   const int64_t lo = cu.lo(r);
-  return lo <= first ? 0 : (lo - first + P - 1) / P;
+  return lo <= first ? 0 : div_nn(lo - first + P - 1, P);
 }
 
 // Workspace slot of the piece of a unit held by range r; r0 owns partition 0.
@@ -131,7 +139,7 @@ __host__ __device__ __forceinline__ int own_piece_slot(int64_t r, const Segment&
 // in token order.
 template <typename F>
 __host__ __device__ void for_each_piece(const Cuts& cu, int64_t P, int64_t first, int L, F f) {
-  const int64_t nparts = (L + P - 1) / P;
+  const int64_t nparts = div_nn(L + P - 1, P);
   const int64_t r0 = cu.owner(first);
   const int64_t r1 = cu.owner(first + (nparts - 1) * P);
   for (int64_t r = r0; r <= r1; ++r) {
@@ -188,8 +196,8 @@ struct SegmentWalker {
       if (p * P >= L) { ++h; p = 0; continue; }  // unit's rest belongs to earlier ranges
       const int64_t first = base + (int64_t)h * unit_work(L, cost, round) + cost;
       if (first + p * P >= hi) { done = true; break; }
-      const int64_t nparts = (L + P - 1) / P;
-      int64_t q = (hi - 1 - first) / P;
+      const int64_t nparts = div_nn(L + P - 1, P);
+      int64_t q = div_nn(hi - 1 - first, P);
       if (q > nparts - 1) q = nparts - 1;
       s.seq = i;
       s.head = h;
@@ -243,20 +251,20 @@ __host__ __device__ __forceinline__ void start_range(SegmentWalker& w, int64_t l
   w.Lnext = fLnext;
   const int64_t fw = unit_work(fL, w.cost, w.round);
   const int64_t rel = lo - fbase;
-  w.h = (int)(rel / fw);
+  w.h = (int)div_nn(rel, fw);
   const int64_t r = rel - (int64_t)w.h * fw;  // offset inside unit (fi, h)
-  w.p = r <= w.cost ? 0 : (r - w.cost + w.P - 1) / w.P;
+  w.p = r <= w.cost ? 0 : div_nn(r - w.cost + w.P - 1, w.P);
   w.has_head = w.p > 0 && w.p * w.P < fL && fbase + (int64_t)w.h * fw + w.cost + w.p * w.P < hi;
   // The tail: the last item lies in a unit that starts at or after lo and
   // continues past hi.
   if (li < 0 || lL <= 0) return;
   const int64_t lw = unit_work(lL, w.cost, w.round);
   const int64_t lrel = (hi - 1) - lbase;
-  const int hh = (int)(lrel / lw);
+  const int hh = (int)div_nn(lrel, lw);
   const int64_t first = lbase + (int64_t)hh * lw + w.cost;
   if (hi - 1 < first || first < lo) return;
-  const int64_t nparts = (lL + w.P - 1) / w.P;
-  const int64_t q = (hi - 1 - first) / w.P;
+  const int64_t nparts = div_nn(lL + w.P - 1, w.P);
+  const int64_t q = div_nn(hi - 1 - first, w.P);
   if (q >= nparts - 1) return;  // the unit ends inside the range
   w.tail.seq = li;
   w.tail.head = hh;
