@@ -14,23 +14,26 @@
 //    and an MMA warp (the whole warp runs the issue loop on warp-uniform
 //    operands; one elected thread issues every MMA and commit).
 //  * The producer streams the causal range in 64-token chunks through a
-//    three-stage ring shared by both tiles. Each (block, KV head) tile is
-//    copied as one TMA box per 64-element piece of head_dim, so in shared
-//    memory a chunk's K (and V) is, per piece, 64 token rows of 128 bytes in
-//    the 128B swizzle: K is a K-major operand and V an MN-major operand of the
-//    tensor core as it lands.
-//  * S = Q K^T of a tile (M 128, N 64, K 16 per instruction) lands in the
-//    tile's S columns of tensor memory; the MMA warp issues the next chunk's S
-//    as soon as the softmax threads have read this one, so it overlaps their
-//    softmax. They apply the causal mask (only in chunks that reach past a
-//    row's position) and the scale, and keep a running maximum that is only
-//    raised (and O rescaled in tensor memory) when a chunk's maximum exceeds it
-//    by more than 2^8, so rescaling is rare and P = 2^(s - m) stays below 256.
-//  * P goes back to tensor memory as 16-bit pairs, and O += P [V | 1] (A from
-//    tensor memory, M 128, N head_dim + 16) accumulates in the tile's O
-//    columns: the extra operand piece holds a column of ones, so the row sums
-//    of the rounded P come out of the tensor core beside O, rescaled with it.
-//    At the end each thread reads its row of O and its sum, divides and
+//    four-stage ring shared by both tiles. Each (block, KV head) tile is copied
+//    as one TMA box per 64-element piece of head_dim, so in shared memory a
+//    chunk's K (and V) is, per piece, 64 token rows of 128 bytes in the 128B
+//    swizzle: K is a K-major operand and V an MN-major operand of the tensor
+//    core as it lands.
+//  * Each tile has two S buffers in tensor memory (chunk c uses buffer c % 2):
+//    S = Q K^T of the next chunk (M 128, N 64, K 16 per instruction) is
+//    computed into one while the softmax threads work on the other, so a
+//    softmax thread finds its next S ready instead of waiting for it. The
+//    threads read S with tcgen05.ld, apply the causal mask (only in chunks that
+//    reach past a row's position) and the scale, keep a running maximum that
+//    is only raised (and O rescaled in tensor memory) when a chunk's maximum
+//    exceeds it by more than 2^8, so rescaling is rare and P = 2^(s - m) stays
+//    below 256, and sum the rounded P into their row sums.
+//  * P goes back over the first 32 columns of its own S buffer as 16-bit pairs,
+//    and O += P V (A from tensor memory, M 128, N head_dim) accumulates in the
+//    tile's O columns. The MMA warp issues, per chunk c and tile t, the PV of
+//    chunk c and then S of chunk c + 2 into the same buffer: MMAs of a CTA run
+//    in issue order, so S(c + 2) overwrites P(c) only after the PV that read
+//    it. At the end each thread reads its row of O, divides by its row sum and
 //    stores it.
 //  * Slots past the causal range are masked in S and zeroed in V before the
 //    last PV, so stale or poisoned memory never reaches the output.
@@ -60,7 +63,7 @@ constexpr int kSoftWarps = 4 * kTiles;
 constexpr int kProducerWarp = kSoftWarps;
 constexpr int kMmaWarp = kSoftWarps + 1;
 constexpr int kThreads = (kSoftWarps + 2) * 32;
-constexpr int kNS = 3;          // K/V stages
+constexpr int kNS = 4;          // K/V stages
 constexpr uint32_t kTmemCols = 512;
 
 __device__ __forceinline__ float max3f(float a, float b, float c) {
@@ -87,17 +90,17 @@ struct Cfg5 {
   static constexpr int kPlanes = D / 64;          // 128-byte pieces of head_dim
   static constexpr int kPlaneKV = kChunk * 128;   // one piece of a K (or V) chunk
   static constexpr int kKV = kPlanes * kPlaneKV;
-  // K pieces, V pieces, then one more V piece whose first column is 1 and the
-  // rest 0: O += P [V | 1] yields the row sums of P in the column after O.
-  static constexpr int kStage = 2 * kKV + kPlaneKV;
+  static constexpr int kStage = 2 * kKV;          // K pieces, then V pieces
   static constexpr int kPlaneQ = kRows * 128;
   static constexpr int kQ = kPlanes * kPlaneQ;    // Q of one tile
-  // Tensor-memory columns: S of tile t at 64 t, P of tile t (bf16 pairs, 32
-  // columns) at 128 + 32 t, O of tile t at 192 + t (D + 32): D columns of O,
-  // the row sum, and padding to a whole group of 32.
-  static constexpr uint32_t kColP = 128, kColO = 192, kOCols = D + 32;
-  static_assert(kColO + kTiles * kOCols <= kTmemCols, "tensor memory per CTA");
-  static constexpr int kBars = 2 * kNS + 4 * kTiles + 2;  // full, empty, s_full, s_free, p_full, o_done, q_full, drain
+  // Tensor-memory columns: two S buffers of 64 columns per tile (chunk c uses
+  // buffer c % 2, at 128 t + 64 (c % 2); P of the chunk is written, as 16-bit
+  // pairs, over the first 32 columns of its buffer), and O of tile t at
+  // 256 + t D.
+  static constexpr uint32_t kColO = 256;
+  static_assert(kColO + kTiles * D <= kTmemCols, "tensor memory per CTA");
+  // full, empty, s_full [tile][buffer], p_full [tile], o_done [tile], q_full, drain
+  static constexpr int kBars = 2 * kNS + 4 * kTiles + 2;
   static constexpr int kSmem = 1024 + kNS * kStage + kTiles * kQ + kBars * 8 + 16;
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA exceeds 227 KB");
 };
@@ -231,16 +234,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* ring = smem;                          // kNS stages: K pieces, V pieces, ones piece
+  uint8_t* ring = smem;                          // kNS stages: K pieces, V pieces
   uint8_t* qs = ring + kNS * C::kStage;          // Q pieces of tile 0, then of tile 1
   uint64_t* full = reinterpret_cast<uint64_t*>(qs + kTiles * C::kQ);
   uint64_t* empty = full + kNS;
-  uint64_t* s_full = empty + kNS;       // [tile] S of the tile's chunk is in tensor memory
-  uint64_t* s_free = s_full + kTiles;   // [tile] the tile's softmax warps have read S
-  uint64_t* p_full = s_free + kTiles;   // [tile] P of the tile's chunk is in tensor memory
-  uint64_t* o_done = p_full + kTiles;   // [tile] the tile's PV of the chunk has completed
-  uint64_t* q_full = o_done + kTiles;   // Q is staged
-  uint64_t* drain = q_full + 1;         // the MMA warp's last MMAs have completed
+  uint64_t* s_full = empty + kNS;        // [tile][buffer] S of a chunk is in tensor memory
+  uint64_t* p_full = s_full + 2 * kTiles; // [tile] P of the tile's chunk is in tensor memory
+  uint64_t* o_done = p_full + kTiles;    // [tile] the tile's PV of a chunk has completed
+  uint64_t* q_full = o_done + kTiles;    // Q is staged
+  uint64_t* drain = q_full + 1;          // every MMA issued has completed
   uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
 
@@ -266,8 +268,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(empty + s, 1);
     }
     for (int t = 0; t < kTiles; ++t) {
-      mbar_init(s_full + t, 1);
-      mbar_init(s_free + t, kRows);
+      mbar_init(s_full + 2 * t, 1);
+      mbar_init(s_full + 2 * t + 1, 1);
       mbar_init(p_full + t, kRows);
       mbar_init(o_done + t, 1);
     }
@@ -328,63 +330,74 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------------- MMA ----
-    // S = Q K^T of each tile for chunk c + 1 as soon as the tile's softmax has
-    // read S of chunk c, so it overlaps that softmax; then O += P [V | 1] of
-    // each tile for chunk c once its P is in tensor memory, which also frees
-    // the chunk's stage. The whole warp runs the loop and computes every
-    // operand (warp-uniform values); one elected thread issues each group of
-    // MMAs and the commit that tracks them.
+    // S of the first two chunks up front (one S buffer each), then per chunk c
+    // and tile t: O_t += P_t(c) V(c) once the tile's softmax has written P(c)
+    // over its S buffer, then S_t(c + 2) into that same buffer. MMAs of a CTA
+    // run in issue order, so S(c + 2) overwrites P(c) only after the PV that
+    // read it, while S(c + 1), in the other buffer, was computed during the
+    // softmax of chunk c. The whole warp runs the loop on warp-uniform operands;
+    // one elected thread issues.
     constexpr uint32_t idS = idesc<T>(kRows, kChunk, false);
-    constexpr uint32_t idO = idesc<T>(kRows, D + 16, true);  // O and the row sums
+    constexpr uint32_t idO = idesc<T>(kRows, D, true);
     const uint32_t q_addr = smem_u32(qs), r_addr = smem_u32(ring);
     const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
-    const bool leader = elect_one();  // the same thread issues every MMA and commit
+    const bool leader = elect_one();
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, wait5(bar, parity, abort));
     };
+    auto issue_s = [&](int c, int t) {  // S_t(c) = Q_t K(c)^T into buffer c % 2
+      const uint32_t k = r_addr + (c % kNS) * C::kStage;
+#pragma unroll
+      for (int s = 0; s < D / 16; ++s) {
+        const int pc = s / 4, off = (s % 4) * 32;
+        umma(tm + 128 * t + 64 * (c & 1), sdesc(q_addr + t * C::kQ + pc * C::kPlaneQ + off, 16),
+             sdesc(k + pc * C::kPlaneKV + off, 16), idS, s > 0 ? 1u : 0u);
+      }
+      umma_commit(s_full + 2 * t + (c & 1));
+    };
+    auto issue_pv = [&](int c, int t) {  // O_t += P_t(c) V(c)
+      const uint32_t v = r_addr + (c % kNS) * C::kStage + C::kKV;
+#pragma unroll
+      for (int s = 0; s < kChunk / 16; ++s)
+        umma_ts(tm + C::kColO + t * D, tm + 128 * t + 64 * (c & 1) + 8 * s,
+                sdesc(v + s * 16 * 128, C::kPlaneKV), idO, (c > 0 || s > 0) ? 1u : 0u);
+      umma_commit(o_done + t);
+    };
     bool ok = wait_warp(q_full, 0);
     tc_fence_after();
-    auto issue_qk = [&](int c) -> bool {
-      const int stage = c % kNS;
-      if (!wait_warp(full + stage, (uint32_t)(c / kNS) & 1u)) return false;
-      const uint32_t k = r_addr + stage * C::kStage;
-      for (int t = 0; t < ntiles; ++t) {
-        if (c > 0 && !wait_warp(s_free + t, (uint32_t)(c - 1) & 1u)) return false;
+    for (int c = 0; c < 2 && c < nchunks && ok; ++c) {
+      ok = wait_warp(full + c % kNS, (uint32_t)(c / kNS) & 1u);
+      if (!ok) break;
+      tc_fence_after();
+      if (leader)
+        for (int t = 0; t < ntiles; ++t) issue_s(c, t);
+      __syncwarp();
+    }
+    for (int c = 0; c < nchunks && ok; ++c) {
+      const bool more = c + 2 < nchunks;
+      for (int t = 0; t < ntiles && ok; ++t) {
+        ok = wait_warp(p_full + t, (uint32_t)c & 1u);
+        if (!ok) break;
         tc_fence_after();
         if (leader) {
-#pragma unroll
-          for (int s = 0; s < D / 16; ++s) {
-            const int pc = s / 4, off = (s % 4) * 32;
-            umma(tm + 64 * t, sdesc(q_addr + t * C::kQ + pc * C::kPlaneQ + off, 16),
-                 sdesc(k + pc * C::kPlaneKV + off, 16), idS, s > 0 ? 1u : 0u);
-          }
-          umma_commit(s_full + t);
-        }
-        __syncwarp();
-      }
-      return true;
-    };
-    auto issue_pv = [&](int c) -> bool {
-      const uint32_t v = r_addr + (c % kNS) * C::kStage + C::kKV;
-      for (int t = 0; t < ntiles; ++t) {
-        if (!wait_warp(p_full + t, (uint32_t)c & 1u)) return false;
-        tc_fence_after();
-        if (leader) {
-#pragma unroll
-          for (int s = 0; s < kChunk / 16; ++s)
-            umma_ts(tm + C::kColO + t * C::kOCols, tm + C::kColP + 32 * t + 8 * s,
-                    sdesc(v + s * 16 * 128, C::kPlaneKV), idO, (c > 0 || s > 0) ? 1u : 0u);
-          umma_commit(o_done + t);
+          issue_pv(c, t);
+          // The stage of chunk c is free once both tiles' PV of it (and, issued
+          // earlier, their S) have completed.
           if (t == ntiles - 1) umma_commit(empty + c % kNS);
         }
         __syncwarp();
+        if (more) {
+          // K of chunk c + 2 (waited for only now, so the PV above never waits
+          // on a copy).
+          if (t == 0) {
+            ok = wait_warp(full + (c + 2) % kNS, (uint32_t)((c + 2) / kNS) & 1u);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          if (leader) issue_s(c + 2, t);
+          __syncwarp();
+        }
       }
-      return true;
-    };
-    if (ok) ok = issue_qk(0);
-    for (int c = 0; c < nchunks && ok; ++c) {
-      if (c + 1 < nchunks) ok = issue_qk(c + 1);
-      if (ok) ok = issue_pv(c);
     }
     // Whatever happened, wait (bounded) until every MMA issued has completed.
     if (leader) {
@@ -403,8 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tok = valid ? R / g : 0, j = valid ? R - tok * g : 0;
     const int pos = valid ? base_pos + tok : -1;
     const uint32_t trow = tmem + ((uint32_t)(32 * (warp % 4)) << 16);
-    const uint32_t tS = trow + 64 * t, tP = trow + C::kColP + 32 * t,
-                   tO = trow + C::kColO + t * C::kOCols;
+    const uint32_t tO = trow + C::kColO + t * D;
     // Stage this row of Q (zeros past the chunk) in the operand layout.
     {
       uint8_t* qt = qs + t * C::kQ;
@@ -416,30 +428,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<uint4*>(qt + (u >> 3) * C::kPlaneQ + sw(r, u & 7)) = v;
       }
     }
-    // The ones piece of every stage (written once; the copies never touch it).
-    for (int e = threadIdx.x; e < kNS * kChunk * 8; e += kSoftWarps * 32) {
-      const int st = e / (kChunk * 8), tk = (e / 8) % kChunk, u = e % 8;
-      const uint16_t one = std::is_same<T, __nv_bfloat16>::value ? 0x3F80u : 0x3C00u;
-      const uint32_t w0 = (u == (tk & 7)) ? (uint32_t)one : 0u;  // element 0 of the row
-      *reinterpret_cast<uint4*>(ring + st * C::kStage + 2 * C::kKV + tk * 128 + u * 16) =
-          make_uint4(w0, 0u, 0u, 0u);
-    }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     mbar_arrive(q_full);
     const float sscale = p.score_scale;
-    float m_use = -INFINITY;
+    float m_use = -INFINITY, l0 = 0.f, l1 = 0.f;
     bool ok = t < ntiles;
     for (int c = 0; c < nchunks && ok; ++c) {
-      ok = wait5(s_full + t, (uint32_t)c & 1u, abort);
+      ok = wait5(s_full + 2 * t + (c & 1), (uint32_t)(c >> 1) & 1u, abort);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      const uint32_t tS = trow + 128 * t + 64 * (c & 1);
       float s[64];
       tmem_ld64(tS, s);
-      tc_fence_before();
-      mbar_arrive(s_free + t);  // the next S of this tile may overwrite it
       const int c0 = c * kChunk;
       // Raw scores; the causal mask only where the chunk reaches past a row's
       // position. The scale is applied with the exponent (it is positive, so the
@@ -452,9 +455,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Raise the running maximum only when this chunk exceeds it by 2^8.
       const bool raise = mx > m_use + 8.f;
       const bool rescale = raise && m_use != -INFINITY;
+      // The PV of the previous chunk must have completed before O is rescaled
+      // (and it is waited for once per chunk in any case, below, so that the
+      // tile's PV barrier is never more than one phase ahead of this thread).
       bool pv_waited = false;
       if (__any_sync(0xffffffffu, rescale)) {
-        if (c > 0) {  // the last PV must have landed in O
+        if (c > 0) {
           ok = wait5(o_done + t, (uint32_t)(c - 1) & 1u, abort);
           if (!__all_sync(0xffffffffu, ok)) {
             ok = false;
@@ -464,8 +470,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           pv_waited = true;
         }
         const float alpha = rescale ? fast_exp2(m_use - mx) : 1.f;
+        l0 *= alpha;
+        l1 *= alpha;
 #pragma unroll
-        for (int q = 0; q <= D / 32; ++q) {  // O and, in the last group, the row sums
+        for (int q = 0; q < D / 32; ++q) {
           float o[32];
           tmem_ld32(tO + 32 * q, o);
 #pragma unroll
@@ -487,18 +495,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rr) : "l"(xy), "l"(sc), "l"(mm));
           asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(rr));
         }
-        const float p0 = fast_exp2(x0);
-        const float p1 = fast_exp2(x1);
-        float lo, hi;  // (the row sums come from the tensor core, of the rounded P)
-        pk[i] = Mma<T>::pack(p0, p1, lo, hi);
+        float lo, hi;  // the row sums take P as the tensor cores see it (rounded)
+        pk[i] = Mma<T>::pack(fast_exp2(x0), fast_exp2(x1), lo, hi);
+        l0 += lo;
+        l1 += hi;
       }
-      if (c > 0 && !pv_waited) {  // the PV that read P of the previous chunk has completed
+      if (c > 0 && !pv_waited) {
         ok = wait5(o_done + t, (uint32_t)(c - 1) & 1u, abort);
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
         }
-        tc_fence_after();
       }
       if (t == 0 && c == nchunks - 1 && c0 + kChunk > kv_end) {
         // Zero V rows past the range (stale or poisoned) before the last PVs
@@ -512,7 +519,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
-      tmem_st32(tP, pk);
+      // P over the first 32 columns of this chunk's S buffer (S is in registers).
+      tmem_st32(tS, pk);
       tc_fence_before();
       mbar_arrive(p_full + t);
     }
@@ -522,9 +530,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) {
       tc_fence_after();
-      float ls[32];
-      tmem_ld32(tO + D, ls);  // column D of the tile's O: the row sum of P
-      const float inv = ls[0] > 0.f ? 1.f / ls[0] : 0.f;
+      const float lsum = l0 + l1;
+      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
       T* dst = static_cast<T*>(p.out) + ((int64_t)(q0 + tok) * Hq + h * g + j) * D;
 #pragma unroll
       for (int q = 0; q < D / 32; ++q) {
