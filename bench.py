@@ -709,16 +709,18 @@ def run_block_sizes(args, dev):
             ks = torch.tensor([wl.k_scale], device=dev)
             vs = torch.tensor([wl.v_scale], device=dev)
 
-        def call():
+        def call(flags=pkv.PKV_DECODE_ZEROED_WORKSPACE):
             pkv.paged_attention_decode(out, wl.query, wl.k_cache, wl.v_cache, bt, sl,
                                        max_seq_len=wl.max_seq_len, scale=c.scale,
-                                       partition_size=P, workspace=ws, k_scale=ks, v_scale=vs)
-        ms = _event_time_ms(call, reps, warmup)
+                                       partition_size=P, workspace=ws, k_scale=ks, v_scale=vs,
+                                       flags=flags)
+        call(0)  # zeroes the split counters; every call leaves them zero
+        ms, how = kernel_time_ms(lambda: None, call, reps=max(3, reps // 4))
         dec, _ = step_bytes(wl)
         gbs = dec / ms / 1e6
         lines.append({"metric": "paged decode attention HBM GB/s by block size", "value": round(gbs, 1),
                       "unit": "GB/s", "higher_is_better": True, "block_size": bs,
-                      "us_per_launch": round(ms * 1e3, 2), "dtype": c.q_dtype,
+                      "us_per_launch": round(ms * 1e3, 2), "timing": how, "dtype": c.q_dtype,
                       "data": "synthetic", "config": {"workload": WORKLOAD_TEXT.get(
                           args.workload, args.workload).replace("block 16", f"block {bs}")},
                       "fragmentation": round(FR.fixed_block_fragmentation(wl.seq_lens, bs), 5),
@@ -851,12 +853,12 @@ def run_prefill(args, dev):
             def call():
                 pkv.paged_attention_prefill(out, q, kc, vc, btd, lensd, qsd, max_q_len=max(qlen),
                                             scale=D ** -0.5, flags=flags)
-            ms = _event_time_ms(call, reps, warmup)
+            ms, how = kernel_time_ms(lambda: None, call, n=8, reps=max(3, reps // 8))
             assert pkv.pkv_device_status(clear=True) == 0, "device wait expired"
             tflops = flops / ms / 1e9
             lines.append({"metric": "paged causal multi-token attention TFLOP/s",
                           "value": round(tflops, 1), "unit": "TFLOP/s", "higher_is_better": True,
-                          "us_per_launch": round(ms * 1e3, 1),
+                          "us_per_launch": round(ms * 1e3, 1), "timing": how,
                           "tokens_per_s": round(T / ms * 1e3, 0), "dtype": "bf16",
                           "data": "synthetic",
                           "config": {"workload": name + f"; {Hq} q / {Hkv} KV heads, head_dim {D}, "
