@@ -30,11 +30,16 @@
 //    below 256, and sum the rounded P into their row sums.
 //  * P goes back over the first 32 columns of its own S buffer as 16-bit pairs,
 //    and O += P V (A from tensor memory, M 128, N head_dim) accumulates in the
-//    tile's O columns. The MMA warp issues, per chunk c and tile t, the PV of
-//    chunk c and then S of chunk c + 2 into the same buffer: MMAs of a CTA run
-//    in issue order, so S(c + 2) overwrites P(c) only after the PV that read
-//    it. At the end each thread reads its row of O, divides by its row sum and
-//    stores it.
+//    tile's O columns. The MMA warp issues, per chunk c, the PV of chunk c for
+//    both tiles and then S of chunk c + 2 for both tiles into the buffers
+//    those PVs read: MMAs of a CTA run in issue order, so S(c + 2) overwrites
+//    P(c) only after the PV that read it, and no S directly follows the PV of
+//    its own buffer (that pairing stalls the tensor pipe). At the end each
+//    thread reads its row of O, divides by its row sum and stores it.
+//  * The commit after S(c + 2) (past the last chunk, a commit alone) also
+//    tells a tile's softmax that PV(c) has completed: it is what O's rescale
+//    and the final read of O wait for. P has a barrier per S buffer, so a
+//    softmax that runs a chunk ahead never completes a phase twice.
 //  * Slots past the causal range are masked in S and zeroed in V before the
 //    last PV, so stale or poisoned memory never reaches the output.
 //  * Every wait is bounded; on expiry the CTA records it, stops, waits (bounded)
@@ -99,7 +104,7 @@ struct Cfg5 {
   // 256 + t D.
   static constexpr uint32_t kColO = 256;
   static_assert(kColO + kTiles * D <= kTmemCols, "tensor memory per CTA");
-  // full, empty, s_full [tile][buffer], p_full [tile], o_done [tile], q_full, drain
+  // full, empty, s_full [tile][buffer], p_full [tile][buffer], q_full, drain
   static constexpr int kBars = 2 * kNS + 4 * kTiles + 2;
   static constexpr int kSmem = 1024 + kNS * kStage + kTiles * kQ + kBars * 8 + 16;
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA exceeds 227 KB");
@@ -239,9 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(qs + kTiles * C::kQ);
   uint64_t* empty = full + kNS;
   uint64_t* s_full = empty + kNS;        // [tile][buffer] S of a chunk is in tensor memory
-  uint64_t* p_full = s_full + 2 * kTiles; // [tile] P of the tile's chunk is in tensor memory
-  uint64_t* o_done = p_full + kTiles;    // [tile] the tile's PV of a chunk has completed
-  uint64_t* q_full = o_done + kTiles;    // Q is staged
+  uint64_t* p_full = s_full + 2 * kTiles; // [tile][buffer] P of a chunk is in tensor memory
+  uint64_t* q_full = p_full + 2 * kTiles; // Q is staged
   uint64_t* drain = q_full + 1;          // every MMA issued has completed
   uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
@@ -270,8 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < kTiles; ++t) {
       mbar_init(s_full + 2 * t, 1);
       mbar_init(s_full + 2 * t + 1, 1);
-      mbar_init(p_full + t, kRows);
-      mbar_init(o_done + t, 1);
+      mbar_init(p_full + 2 * t, kRows);
+      mbar_init(p_full + 2 * t + 1, kRows);
     }
     mbar_init(q_full, kSoftWarps * 32);
     mbar_init(drain, 1);
@@ -330,13 +334,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------------- MMA ----
-    // S of the first two chunks up front (one S buffer each), then per chunk c
-    // and tile t: O_t += P_t(c) V(c) once the tile's softmax has written P(c)
-    // over its S buffer, then S_t(c + 2) into that same buffer. MMAs of a CTA
-    // run in issue order, so S(c + 2) overwrites P(c) only after the PV that
-    // read it, while S(c + 1), in the other buffer, was computed during the
-    // softmax of chunk c. The whole warp runs the loop on warp-uniform operands;
-    // one elected thread issues.
+    // S of the first two chunks up front (one S buffer each), then per chunk c:
+    // O_t += P_t(c) V(c) for each tile once its softmax has written P(c) over
+    // its S buffer, then S_t(c + 2) for each tile into those buffers, while
+    // S(c + 1), in the other buffers, was computed during the softmax of chunk
+    // c. The whole warp runs the loop on warp-uniform operands; one elected
+    // thread issues.
     constexpr uint32_t idS = idesc<T>(kRows, kChunk, false);
     constexpr uint32_t idO = idesc<T>(kRows, D, true);
     const uint32_t q_addr = smem_u32(qs), r_addr = smem_u32(ring);
@@ -346,22 +349,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       return __all_sync(0xffffffffu, wait5(bar, parity, abort));
     };
     auto issue_s = [&](int c, int t) {  // S_t(c) = Q_t K(c)^T into buffer c % 2
-      const uint32_t k = r_addr + (c % kNS) * C::kStage;
+      // Base descriptors once; the K steps add compile-time offsets to the
+      // 14-bit address field (addresses stay below 256 KB, so it never carries).
+      const uint64_t a0 = sdesc(q_addr + t * C::kQ, 16);
+      const uint64_t b0 = sdesc(r_addr + (c % kNS) * C::kStage, 16);
+      const uint32_t dS = tm + 128 * t + 64 * (c & 1);
 #pragma unroll
       for (int s = 0; s < D / 16; ++s) {
         const int pc = s / 4, off = (s % 4) * 32;
-        umma(tm + 128 * t + 64 * (c & 1), sdesc(q_addr + t * C::kQ + pc * C::kPlaneQ + off, 16),
-             sdesc(k + pc * C::kPlaneKV + off, 16), idS, s > 0 ? 1u : 0u);
+        umma(dS, a0 + (uint64_t)((pc * C::kPlaneQ + off) >> 4),
+             b0 + (uint64_t)((pc * C::kPlaneKV + off) >> 4), idS, s > 0 ? 1u : 0u);
       }
       umma_commit(s_full + 2 * t + (c & 1));
     };
     auto issue_pv = [&](int c, int t) {  // O_t += P_t(c) V(c)
-      const uint32_t v = r_addr + (c % kNS) * C::kStage + C::kKV;
+      const uint64_t b0 = sdesc(r_addr + (c % kNS) * C::kStage + C::kKV, C::kPlaneKV);
+      const uint32_t dO = tm + C::kColO + t * D, aP = tm + 128 * t + 64 * (c & 1);
 #pragma unroll
       for (int s = 0; s < kChunk / 16; ++s)
-        umma_ts(tm + C::kColO + t * D, tm + 128 * t + 64 * (c & 1) + 8 * s,
-                sdesc(v + s * 16 * 128, C::kPlaneKV), idO, (c > 0 || s > 0) ? 1u : 0u);
-      umma_commit(o_done + t);
+        umma_ts(dO, aP + 8 * s, b0 + (uint64_t)((s * 16 * 128) >> 4), idO,
+                (c > 0 || s > 0) ? 1u : 0u);
     };
     bool ok = wait_warp(q_full, 0);
     tc_fence_after();
@@ -374,9 +381,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     }
     for (int c = 0; c < nchunks && ok; ++c) {
-      const bool more = c + 2 < nchunks;
       for (int t = 0; t < ntiles && ok; ++t) {
-        ok = wait_warp(p_full + t, (uint32_t)c & 1u);
+        ok = wait_warp(p_full + 2 * t + (c & 1), (uint32_t)(c >> 1) & 1u);
         if (!ok) break;
         tc_fence_after();
         if (leader) {
@@ -386,17 +392,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (t == ntiles - 1) umma_commit(empty + c % kNS);
         }
         __syncwarp();
-        if (more) {
-          // K of chunk c + 2 (waited for only now, so the PV above never waits
-          // on a copy).
-          if (t == 0) {
-            ok = wait_warp(full + (c + 2) % kNS, (uint32_t)((c + 2) / kNS) & 1u);
-            if (!ok) break;
-            tc_fence_after();
-          }
-          if (leader) issue_s(c + 2, t);
-          __syncwarp();
-        }
+      }
+      if (!ok) break;
+      // S of chunk c + 2 for both tiles after both PVs of chunk c, so no S
+      // directly follows the PV that reads its buffer. K of chunk c + 2 is
+      // waited for only now, so the PVs above never wait on a copy.
+      if (c + 2 < nchunks) {
+        ok = wait_warp(full + (c + 2) % kNS, (uint32_t)((c + 2) / kNS) & 1u);
+        if (!ok) break;
+        tc_fence_after();
+        if (leader)
+          for (int t = 0; t < ntiles; ++t) issue_s(c + 2, t);
+        __syncwarp();
+      } else if (leader) {
+        for (int t = 0; t < ntiles; ++t)
+          umma_commit(s_full + 2 * t + (c & 1));  // stand-in for S(c + 2): PV(c) has completed
       }
     }
     // Whatever happened, wait (bounded) until every MMA issued has completed.
@@ -431,7 +441,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     mbar_arrive(q_full);
     const float sscale = p.score_scale;
-    float m_use = -INFINITY, l0 = 0.f, l1 = 0.f;
+    float m_use = -INFINITY;
+    uint64_t lsum2 = 0;
     bool ok = t < ntiles;
     for (int c = 0; c < nchunks && ok; ++c) {
       ok = wait5(s_full + 2 * t + (c & 1), (uint32_t)(c >> 1) & 1u, abort);
@@ -455,23 +466,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Raise the running maximum only when this chunk exceeds it by 2^8.
       const bool raise = mx > m_use + 8.f;
       const bool rescale = raise && m_use != -INFINITY;
-      // The PV of the previous chunk must have completed before O is rescaled
-      // (and it is waited for once per chunk in any case, below, so that the
-      // tile's PV barrier is never more than one phase ahead of this thread).
-      bool pv_waited = false;
+      // The PV of the previous chunk must have completed before O is rescaled:
+      // the commit of S(c + 1) (or of its stand-in) follows it.
       if (__any_sync(0xffffffffu, rescale)) {
         if (c > 0) {
-          ok = wait5(o_done + t, (uint32_t)(c - 1) & 1u, abort);
+          ok = wait5(s_full + 2 * t + ((c + 1) & 1), (uint32_t)((c + 1) >> 1) & 1u, abort);
           if (!__all_sync(0xffffffffu, ok)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          pv_waited = true;
         }
         const float alpha = rescale ? fast_exp2(m_use - mx) : 1.f;
-        l0 *= alpha;
-        l1 *= alpha;
+        {
+          uint64_t aa;
+          asm("mov.b64 %0, {%1, %1};" : "=l"(aa) : "f"(alpha));
+          asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(lsum2) : "l"(aa));
+        }
 #pragma unroll
         for (int q = 0; q < D / 32; ++q) {
           float o[32];
@@ -497,14 +508,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         float lo, hi;  // the row sums take P as the tensor cores see it (rounded)
         pk[i] = Mma<T>::pack(fast_exp2(x0), fast_exp2(x1), lo, hi);
-        l0 += lo;
-        l1 += hi;
-      }
-      if (c > 0 && !pv_waited) {
-        ok = wait5(o_done + t, (uint32_t)(c - 1) & 1u, abort);
-        if (!__all_sync(0xffffffffu, ok)) {
-          ok = false;
-          break;
+        {
+          uint64_t pp;
+          asm("mov.b64 %0, {%1, %2};" : "=l"(pp) : "f"(lo), "f"(hi));
+          asm("add.rn.f32x2 %0, %0, %1;" : "+l"(lsum2) : "l"(pp));
         }
       }
       if (t == 0 && c == nchunks - 1 && c0 + kChunk > kv_end) {
@@ -522,14 +529,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P over the first 32 columns of this chunk's S buffer (S is in registers).
       tmem_st32(tS, pk);
       tc_fence_before();
-      mbar_arrive(p_full + t);
+      mbar_arrive(p_full + 2 * t + (c & 1));
     }
-    if (ok) {
-      ok = wait5(o_done + t, (uint32_t)(nchunks - 1) & 1u, abort);
+    if (ok) {  // the stand-in commit of "chunk n + 1": every PV of the tile has completed
+      ok = wait5(s_full + 2 * t + ((nchunks + 1) & 1), (uint32_t)((nchunks + 1) >> 1) & 1u, abort);
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
       tc_fence_after();
+      float l0, l1;
+      asm("mov.b64 {%0, %1}, %2;" : "=f"(l0), "=f"(l1) : "l"(lsum2));
       const float lsum = l0 + l1;
       const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
       T* dst = static_cast<T*>(p.out) + ((int64_t)(q0 + tok) * Hq + h * g + j) * D;
