@@ -9,10 +9,12 @@
 // How:
 //  * A CTA owns 256 query rows — (token, query head of the group) pairs of one
 //    (sequence, KV head) — as two tiles of 128, each the M of one tcgen05.mma.
-//    Ten warps: eight softmax warps (warp w serves tile w / 4 and owns tensor-
-//    memory lanes 32 (w % 4) .. +31, one row per thread), a TMA producer warp
-//    and an MMA warp (the whole warp runs the issue loop on warp-uniform
-//    operands; one elected thread issues every MMA and commit).
+//    Eleven warps: eight softmax warps (warp w serves tile w / 4 and owns
+//    tensor-memory lanes 32 (w % 4) .. +31, one row per thread), a TMA
+//    producer warp and one MMA warp per tile (each runs its tile's issue loop
+//    on warp-uniform operands; one elected thread issues every MMA and commit).
+//    With two issuing warps on different sub-partitions, one warp's barrier
+//    waits overlap the other's MMAs, so the tensor pipe rarely runs dry.
 //  * The producer streams the causal range in 64-token chunks through a
 //    four-stage ring shared by both tiles. Each (block, KV head) tile is copied
 //    as one TMA box per 64-element piece of head_dim, so in shared memory a
@@ -30,12 +32,12 @@
 //    below 256, and sum the rounded P into their row sums.
 //  * P goes back over the first 32 columns of its own S buffer as 16-bit pairs,
 //    and O += P V (A from tensor memory, M 128, N head_dim) accumulates in the
-//    tile's O columns. The MMA warp issues, per chunk c, the PV of chunk c for
-//    both tiles and then S of chunk c + 2 for both tiles into the buffers
-//    those PVs read: MMAs of a CTA run in issue order, so S(c + 2) overwrites
-//    P(c) only after the PV that read it, and no S directly follows the PV of
-//    its own buffer (that pairing stalls the tensor pipe). At the end each
-//    thread reads its row of O, divides by its row sum and stores it.
+//    tile's O columns. A tile's MMA warp issues, per chunk c, the PV of chunk
+//    c and then S of chunk c + 2 into the buffer that PV reads: the MMAs of a
+//    thread run in issue order, so S(c + 2) overwrites P(c) only after the PV
+//    that read it. A K/V stage is free once both tiles' warps have committed
+//    their PV of it. At the end each thread reads its row of O, divides by its
+//    row sum and stores it.
 //  * The commit after S(c + 2) (past the last chunk, a commit alone) also
 //    tells a tile's softmax that PV(c) has completed: it is what O's rescale
 //    and the final read of O wait for. P has a barrier per S buffer, so a
@@ -66,8 +68,8 @@ constexpr int kTiles = 2;       // tiles per CTA, sharing each K/V chunk
 constexpr int kCtaRows = kTiles * kRows;
 constexpr int kSoftWarps = 4 * kTiles;
 constexpr int kProducerWarp = kSoftWarps;
-constexpr int kMmaWarp = kSoftWarps + 1;
-constexpr int kThreads = (kSoftWarps + 2) * 32;
+constexpr int kMmaWarp = kSoftWarps + 1;  // MMA warps kMmaWarp + t, one per tile
+constexpr int kThreads = (kSoftWarps + 1 + kTiles) * 32;
 constexpr int kNS = 4;          // K/V stages
 constexpr uint32_t kTmemCols = 512;
 
@@ -269,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNS; ++s) {
       mbar_init(full + s, 1);
-      mbar_init(empty + s, 1);
+      mbar_init(empty + s, ntiles);  // one commit per tile's MMA warp
     }
     for (int t = 0; t < kTiles; ++t) {
       mbar_init(s_full + 2 * t, 1);
@@ -278,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(p_full + 2 * t + 1, kRows);
     }
     mbar_init(q_full, kSoftWarps * 32);
-    mbar_init(drain, 1);
+    mbar_init(drain, kTiles);
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -332,14 +334,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (clock64() - t0 > kWaitCycles) break;
       }
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp >= kMmaWarp) {
     // ----------------------------------------------------------------- MMA ----
-    // S of the first two chunks up front (one S buffer each), then per chunk c:
-    // O_t += P_t(c) V(c) for each tile once its softmax has written P(c) over
-    // its S buffer, then S_t(c + 2) for each tile into those buffers, while
-    // S(c + 1), in the other buffers, was computed during the softmax of chunk
-    // c. The whole warp runs the loop on warp-uniform operands; one elected
-    // thread issues.
+    // Warp kMmaWarp + t serves tile t: S of the first two chunks up front (one
+    // S buffer each), then per chunk c: O_t += P_t(c) V(c) once the tile's
+    // softmax has written P(c) over its S buffer, then S_t(c + 2) into that
+    // buffer, while S(c + 1), in the other buffer, was computed during the
+    // softmax of chunk c. The whole warp runs the loop on warp-uniform
+    // operands; one elected thread issues.
     constexpr uint32_t idS = idesc<T>(kRows, kChunk, false);
     constexpr uint32_t idO = idesc<T>(kRows, D, true);
     const uint32_t q_addr = smem_u32(qs), r_addr = smem_u32(ring);
@@ -370,43 +372,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_ts(dO, aP + 8 * s, b0 + (uint64_t)((s * 16 * 128) >> 4), idO,
                 (c > 0 || s > 0) ? 1u : 0u);
     };
-    bool ok = wait_warp(q_full, 0);
+    const int t = warp - kMmaWarp;  // this warp issues the MMAs of tile t
+    bool ok = t < ntiles && wait_warp(q_full, 0);
     tc_fence_after();
     for (int c = 0; c < 2 && c < nchunks && ok; ++c) {
       ok = wait_warp(full + c % kNS, (uint32_t)(c / kNS) & 1u);
       if (!ok) break;
       tc_fence_after();
-      if (leader)
-        for (int t = 0; t < ntiles; ++t) issue_s(c, t);
+      if (leader) issue_s(c, t);
       __syncwarp();
     }
     for (int c = 0; c < nchunks && ok; ++c) {
-      for (int t = 0; t < ntiles && ok; ++t) {
-        ok = wait_warp(p_full + 2 * t + (c & 1), (uint32_t)(c >> 1) & 1u);
-        if (!ok) break;
-        tc_fence_after();
-        if (leader) {
-          issue_pv(c, t);
-          // The stage of chunk c is free once both tiles' PV of it (and, issued
-          // earlier, their S) have completed.
-          if (t == ntiles - 1) umma_commit(empty + c % kNS);
-        }
-        __syncwarp();
-      }
+      ok = wait_warp(p_full + 2 * t + (c & 1), (uint32_t)(c >> 1) & 1u);
       if (!ok) break;
-      // S of chunk c + 2 for both tiles after both PVs of chunk c, so no S
-      // directly follows the PV that reads its buffer. K of chunk c + 2 is
-      // waited for only now, so the PVs above never wait on a copy.
+      tc_fence_after();
+      if (leader) {
+        issue_pv(c, t);
+        umma_commit(empty + c % kNS);
+      }
+      __syncwarp();
       if (c + 2 < nchunks) {
         ok = wait_warp(full + (c + 2) % kNS, (uint32_t)((c + 2) / kNS) & 1u);
         if (!ok) break;
         tc_fence_after();
-        if (leader)
-          for (int t = 0; t < ntiles; ++t) issue_s(c + 2, t);
+        if (leader) issue_s(c + 2, t);
         __syncwarp();
       } else if (leader) {
-        for (int t = 0; t < ntiles; ++t)
-          umma_commit(s_full + 2 * t + (c & 1));  // stand-in for S(c + 2): PV(c) has completed
+        umma_commit(s_full + 2 * t + (c & 1));  // stand-in for S(c + 2): PV(c) has completed
       }
     }
     // Whatever happened, wait (bounded) until every MMA issued has completed.
@@ -514,9 +506,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           asm("add.rn.f32x2 %0, %0, %1;" : "+l"(lsum2) : "l"(pp));
         }
       }
-      if (t == 0 && c == nchunks - 1 && c0 + kChunk > kv_end) {
-        // Zero V rows past the range (stale or poisoned) before the last PVs
-        // (tile 0's goes first, so tile 1's comes after these stores too).
+      if (c == nchunks - 1 && c0 + kChunk > kv_end) {
+        // Zero V rows past the range (stale or poisoned) before this tile's
+        // last PV. Both tiles do it, as their PVs are issued independently
+        // (the other tile's stores write the same zeros).
         uint8_t* v = ring + (c % kNS) * C::kStage + C::kKV;
         const int t0 = kv_end - c0, per_row = 8 * C::kPlanes;
         for (int e = r; e < (kChunk - t0) * per_row; e += kRows) {
