@@ -240,9 +240,14 @@ int paged_attention_decode_static(void* out, const void* query, const void* k_ca
  * last max_q_len rows computed. Lengths are clamped to max_blocks_per_seq *
  * block_size and query_start to [0, num_q_tokens]. head_dim 64 or 128,
  * block_size 8/16/32. With a 16-bit cache the default kernel runs on the
- * tcgen05 tensor cores with tensor-memory accumulators (256 query rows per CTA
- * in two tiles); flags PKV_PREFILL_MMA_SYNC selects the mma.sync kernel (64
- * rows per CTA) instead; other flag bits are an error. An FP8-E4M3 cache runs on
+ * tcgen05 tensor cores with tensor-memory accumulators: a persistent kernel,
+ * one CTA per SM taking items of 256 query rows (two tiles) from a work counter
+ * in device memory. Each call takes the next of 64 such counters (the call's
+ * last CTA resets it), so up to 64 prefill calls may be in flight at once, on
+ * any streams; a CUDA graph that holds a call keeps that call's counter, so
+ * replays of one graph must not overlap each other. flags PKV_PREFILL_MMA_SYNC
+ * selects the mma.sync kernel (64 rows per CTA, no counter) instead; other flag
+ * bits are an error. An FP8-E4M3 cache runs on
  * the mma.sync kernel: codes widened exactly to f16 in registers, the query
  * rounded to f16, k_scale folded into the score scale and v_scale into the
  * output.

@@ -7,21 +7,33 @@
 // + r and attends over tokens 0..pos of its sequence.
 //
 // How:
-//  * A CTA owns 256 query rows — (token, query head of the group) pairs of one
-//    (sequence, KV head) — as two tiles of 128, each the M of one tcgen05.mma.
-//    Eleven warps: eight softmax warps (warp w serves tile w / 4 and owns
+//  * The work is items of 256 query rows — (token, query head of the group)
+//    pairs of one (sequence, KV head) — each two tiles of 128, each tile the M
+//    of one tcgen05.mma. The kernel is persistent: one CTA per SM takes items
+//    from a work counter as it becomes free, the items of a few (sequence, KV
+//    head) pairs at a time, longest causal ranges first within them, so their
+//    K/V stays in L2 and the shortest items come last. Within a CTA every role
+//    walks the same sequence of items and 64-token chunks, so a chunk's place
+//    in it names its K/V stage, S buffer and barrier phases in every role,
+//    and the next item's Q and K/V stream in while the current one finishes.
+//  * Eleven warps: eight softmax warps (warp w serves tile w / 4 and owns
 //    tensor-memory lanes 32 (w % 4) .. +31, one row per thread), a TMA
 //    producer warp and one MMA warp per tile (each runs its tile's issue loop
 //    on warp-uniform operands; one elected thread issues every MMA and commit).
 //    With two issuing warps on different sub-partitions, one warp's barrier
 //    waits overlap the other's MMAs, so the tensor pipe rarely runs dry.
-//  * The producer streams the causal range in 64-token chunks through a
-//    four-stage ring shared by both tiles. Each (block, KV head) tile is copied
-//    as one TMA box per 64-element piece of head_dim, so in shared memory a
-//    chunk's K (and V) is, per piece, 64 token rows of 128 bytes in the 128B
-//    swizzle: K is a K-major operand and V an MN-major operand of the tensor
-//    core as it lands.
-//  * Each tile has two S buffers in tensor memory (chunk c uses buffer c % 2):
+//  * The producer takes items from the counter, publishes their records to the
+//    other roles through a small ring in shared memory, starts each item's Q
+//    on its way into L2, and streams the causal range of each item in 64-token
+//    chunks through a four-stage ring shared by both tiles. Each (block, KV
+//    head) tile is copied as one TMA box per 64-element piece of head_dim, so
+//    in shared memory a chunk's K (and V) is, per piece, 64 token rows of 128
+//    bytes in the 128B swizzle: K is a K-major operand and V an MN-major
+//    operand of the tensor core as it lands. A tile's Q (when g divides 128,
+//    whole tokens) is one TMA box per piece of head_dim in the same layout,
+//    loaded by one softmax thread as soon as the tile's last S of the previous
+//    item has completed; otherwise the softmax threads copy their rows.
+//  * Each tile has two S buffers in tensor memory (chunk j uses buffer j % 2):
 //    S = Q K^T of the next chunk (M 128, N 64, K 16 per instruction) is
 //    computed into one while the softmax threads work on the other, so a
 //    softmax thread finds its next S ready instead of waiting for it. The
@@ -32,21 +44,25 @@
 //    below 256, and sum the rounded P into their row sums.
 //  * P goes back over the first 32 columns of its own S buffer as 16-bit pairs,
 //    and O += P V (A from tensor memory, M 128, N head_dim) accumulates in the
-//    tile's O columns. A tile's MMA warp issues, per chunk c, the PV of chunk
-//    c and then S of chunk c + 2 into the buffer that PV reads: the MMAs of a
-//    thread run in issue order, so S(c + 2) overwrites P(c) only after the PV
-//    that read it. A K/V stage is free once both tiles' warps have committed
-//    their PV of it. At the end each thread reads its row of O, divides by its
-//    row sum and stores it.
-//  * The commit after S(c + 2) (past the last chunk, a commit alone) also
-//    tells a tile's softmax that PV(c) has completed: it is what O's rescale
-//    and the final read of O wait for. P has a barrier per S buffer, so a
-//    softmax that runs a chunk ahead never completes a phase twice.
+//    tile's O columns. A tile's MMA warp issues, per chunk j, the PV of chunk
+//    j and then S of chunk j + 2 (of the next item past this one's end) into
+//    the buffer that PV reads: the MMAs of a thread run in issue order, so
+//    S(j + 2) overwrites P(j) only after the PV that read it. A K/V stage is
+//    free once both tiles' warps have committed their PV of it. After an
+//    item's last PV each thread reads its row of O, divides by its row sum and
+//    stores it; the next item's first PV overwrites O only after that, as it
+//    needs P from the same threads.
+//  * The commit after S(j + 2) (past the last chunk, a commit alone) also
+//    tells a tile's softmax that PV(j) has completed: it is what O's rescale
+//    waits for. P has a barrier per S buffer, so a softmax that runs a chunk
+//    ahead never completes a phase twice.
 //  * Slots past the causal range are masked in S and zeroed in V before the
 //    last PV, so stale or poisoned memory never reaches the output.
 //  * Every wait is bounded; on expiry the CTA records it, stops, waits (bounded)
 //    for its own copies and MMAs in flight, and frees its tensor memory.
+#include <algorithm>
 #include <atomic>
+#include <climits>
 #include <type_traits>
 
 #include "common.cuh"
@@ -56,6 +72,9 @@
 namespace pkv {
 
 __device__ int g_pf5_status = 0;  // bit 0: a wait expired; bit 1: a block id outside the pool
+// Work counters of the tcgen05 prefill: per slot the next item to hand out and
+// the CTAs that have finished; the last CTA of a launch puts both back to 0.
+__device__ int g_pf5_sched[64][2];  // 64 = kSchedSlots
 
 namespace pf {
 namespace {
@@ -92,6 +111,15 @@ __device__ __forceinline__ float max64(const float (&s)[64]) {
   return max3f(max3f(u[0], u[1], u[2]), max3f(u[3], u[4], u[5]), fmaxf(u[6], u[7]));
 }
 
+// One unit of work: the 256 query rows row0 .. row0 + 255 of (sequence, KV
+// head); nchunks = 0 marks an empty one.
+struct Item {
+  int seq, h, q0, rows, row0, base_pos, kv_end, nchunks;
+};
+constexpr int kRing = 8;        // item records in flight from the producer to the other roles
+constexpr int kPairGroup = 8;   // (sequence, KV head) pairs whose items are handed out together
+constexpr int kSchedSlots = 64; // work counters, one per launch in flight
+
 template <int D>
 struct Cfg5 {
   static constexpr int kPlanes = D / 64;          // 128-byte pieces of head_dim
@@ -106,9 +134,10 @@ struct Cfg5 {
   // 256 + t D.
   static constexpr uint32_t kColO = 256;
   static_assert(kColO + kTiles * D <= kTmemCols, "tensor memory per CTA");
-  // full, empty, s_full [tile][buffer], p_full [tile][buffer], q_full, drain
-  static constexpr int kBars = 2 * kNS + 4 * kTiles + 2;
-  static constexpr int kSmem = 1024 + kNS * kStage + kTiles * kQ + kBars * 8 + 16;
+  // full, empty, s_full [tile][buffer], p_full [tile][buffer], q_full [tile], o_done [tile], drain
+  static constexpr int kBars = 2 * kNS + 6 * kTiles + 1;
+  static constexpr int kSmem = 1024 + kNS * kStage + kTiles * kQ + kBars * 8 + 16 +
+                               kRing * (16 + (int)sizeof(Item));
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA exceeds 227 KB");
 };
 
@@ -233,10 +262,98 @@ __device__ __forceinline__ uint32_t sw(int r, int j) {
   return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4));
 }
 
-template <typename T, int D>
+// Item i of a launch: the (sequence, KV head) pairs in groups of kPairGroup,
+// and within a group tile pair xr (counted from the end of the chunk, so the
+// longest causal ranges come first) of each pair in turn. CTAs take items in
+// this order as they become free, so the K/V of a few pairs is in use at a
+// time (it stays in L2) and the shortest items come last.
+__device__ __forceinline__ bool load_item(const PrefillParams& p, int num_seqs, int tiles, int i,
+                                          Item& it) {
+  const int Hkv = p.num_kv_heads, g = p.num_heads / Hkv;
+  const int per_group = kPairGroup * tiles, grp = i / per_group;
+  const int pg = min(kPairGroup, num_seqs * Hkv - grp * kPairGroup);
+  const int within = i - grp * per_group, xr = within / pg;
+  const int pair = grp * kPairGroup + within - xr * pg;
+  it.seq = pair / Hkv;
+  it.h = pair - it.seq * Hkv;
+  const int q1 = min(max(__ldg(p.query_start + it.seq + 1), 0), p.num_q_tokens);
+  it.q0 = max(min(max(__ldg(p.query_start + it.seq), 0), q1), q1 - p.max_q_len);
+  const int qn = q1 - it.q0;
+  it.rows = qn * g;
+  const int L = min(__ldg(p.seq_lens + it.seq), p.max_blocks_per_seq * p.block_size);
+  it.row0 = (tiles - 1 - xr) * kCtaRows;
+  if (qn <= 0 || it.row0 >= it.rows || L <= 0) return false;
+  it.base_pos = L - qn;
+  const int last_row = min(it.rows, it.row0 + kCtaRows) - 1;
+  it.kv_end = min(L, it.base_pos + last_row / g + 1);
+  if (it.kv_end <= 0) return false;
+  it.nchunks = (it.kv_end + kChunk - 1) / kChunk;
+  return true;
+}
+
+// The items of this CTA, as the producer publishes them in a ring of kRing
+// records, and their chunks, in order. Every role walks the same sequence, so
+// the position of a chunk in it (its index j) names the same K/V stage
+// (j % kNS), S buffer (j % 2) and barrier phases in every role. All lanes of a
+// warp call the methods; a record with no chunks ends the sequence.
+struct Walk {
+  const Item* ring;
+  uint64_t* full;
+  volatile int* abort;
+  int ii, c, nchunks;  // item number, chunk within it, its chunks
+  bool ok;             // a current chunk exists
+  __device__ __forceinline__ const Item& it() const { return ring[ii % kRing]; }
+  __device__ __forceinline__ void next_item() {
+    ++ii;
+    const int slot = ii % kRing;
+    const bool w = __all_sync(0xffffffffu, wait5(full + slot, (uint32_t)(ii / kRing) & 1u, abort));
+    nchunks = w ? ring[slot].nchunks : 0;
+    ok = nchunks > 0;
+    c = 0;
+  }
+  __device__ __forceinline__ void start(const Item* r, uint64_t* f, volatile int* a) {
+    ring = r;
+    full = f;
+    abort = a;
+    ii = -1;
+    next_item();
+  }
+  __device__ __forceinline__ void advance() {
+    if (++c >= nchunks) next_item();
+  }
+};
+
+// Q rows of a tile by TMA: box (64 elements of head_dim, g heads, 128 / g
+// tokens) of the query tensor (head_dim, heads, tokens), 128B swizzle.
+__device__ __forceinline__ void tma_load_q(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                           uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
+      "{%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_q(const CUtensorMap* map, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(map),
+               "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
+// 16 bytes global -> shared without registers; zeros when !valid.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+
+// QT: Q is copied by TMA (g divides 128, so a tile's rows are whole tokens);
+// otherwise the softmax threads copy their rows.
+template <typename T, int D, bool QT>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc5_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_k,
-                       const __grid_constant__ CUtensorMap tmap_v) {
+                       const __grid_constant__ CUtensorMap tmap_v,
+                       const __grid_constant__ CUtensorMap tmap_q, int num_seqs, int tiles,
+                       int n_items, int* sched) {
   using C = Cfg5<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -245,42 +362,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* qs = ring + kNS * C::kStage;          // Q pieces of tile 0, then of tile 1
   uint64_t* full = reinterpret_cast<uint64_t*>(qs + kTiles * C::kQ);
   uint64_t* empty = full + kNS;
-  uint64_t* s_full = empty + kNS;        // [tile][buffer] S of a chunk is in tensor memory
-  uint64_t* p_full = s_full + 2 * kTiles; // [tile][buffer] P of a chunk is in tensor memory
-  uint64_t* q_full = p_full + 2 * kTiles; // Q is staged
-  uint64_t* drain = q_full + 1;          // every MMA issued has completed
+  uint64_t* s_full = empty + kNS;         // [tile][buffer] S of a chunk is in tensor memory
+  uint64_t* p_full = s_full + 2 * kTiles;  // [tile][buffer] P of a chunk is in tensor memory
+  uint64_t* q_full = p_full + 2 * kTiles;  // [tile] Q of the tile's next item is staged
+  uint64_t* o_done = q_full + kTiles;      // [tile] every PV of the tile's item has completed
+  uint64_t* drain = o_done + kTiles;       // every MMA issued has completed
   uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
+  uint64_t* item_full = drain + 2;           // [kRing] a record is published
+  uint64_t* item_empty = item_full + kRing;  // [kRing] every role is done with a record
+  Item* ring_items = reinterpret_cast<Item*>(item_empty + kRing);
 
   const int Hq = p.num_heads, g = Hq / p.num_kv_heads, bs = p.block_size;
-  const int seq = blockIdx.y, h = blockIdx.z;
-  const int q1 = min(max(__ldg(p.query_start + seq + 1), 0), p.num_q_tokens);
-  const int q0 = max(min(max(__ldg(p.query_start + seq), 0), q1), q1 - p.max_q_len);
-  const int qn = q1 - q0, rows = qn * g;
-  const int L = min(__ldg(p.seq_lens + seq), p.max_blocks_per_seq * bs);
-  const int row0 = (int)(gridDim.x - 1 - blockIdx.x) * kCtaRows;  // longest causal ranges first
-  if (qn <= 0 || row0 >= rows || L <= 0) return;
-  const int base_pos = L - qn;
-  const int last_row = min(rows, row0 + kCtaRows) - 1;
-  const int kv_end = min(L, base_pos + last_row / g + 1);
-  if (kv_end <= 0) return;
-  const int nchunks = (kv_end + kChunk - 1) / kChunk;
-  const int ntiles = rows - row0 > kRows ? 2 : 1;  // the second tile only if it has rows
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNS; ++s) {
       mbar_init(full + s, 1);
-      mbar_init(empty + s, ntiles);  // one commit per tile's MMA warp
+      mbar_init(empty + s, kTiles);  // one commit per tile's MMA warp
     }
     for (int t = 0; t < kTiles; ++t) {
       mbar_init(s_full + 2 * t, 1);
       mbar_init(s_full + 2 * t + 1, 1);
       mbar_init(p_full + 2 * t, kRows);
       mbar_init(p_full + 2 * t + 1, kRows);
+      mbar_init(q_full + t, QT ? 1 : kRows);
+      mbar_init(o_done + t, 1);
     }
-    mbar_init(q_full, kSoftWarps * 32);
     mbar_init(drain, kTiles);
+    for (int s = 0; s < kRing; ++s) {
+      mbar_init(item_full + s, 1);
+      mbar_init(item_empty + s, kTiles + kSoftWarps);  // the MMA warps and the softmax warps
+    }
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -298,15 +411,51 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer ----
-    const int32_t* bt = p.block_table + (int64_t)seq * p.max_blocks_per_seq;
     const int piece = bs * 128;  // bytes of one (block, piece of head_dim) box
     uint32_t armed = 0, last_parity = 0;
     bool ok = true;
-    for (int c = 0; c < nchunks && ok; ++c) {
-      const int stage = c % kNS;
-      const uint32_t phase = (uint32_t)(c / kNS) & 1u;
+    // Takes the next item of the launch (lane 0, from the work counter),
+    // publishes its record (one with no chunks when the work is gone) and
+    // starts its Q on the way into L2.
+    int ii = -1;
+    Item cur;
+    auto publish = [&]() -> bool {
+      ++ii;
+      const int slot = ii % kRing;
+      if (lane == 0) ok = wait5(item_empty + slot, ((uint32_t)(ii / kRing) & 1u) ^ 1u, abort);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) return false;
+      if (lane == 0) {
+        Item it;
+        for (;;) {
+          const int i = atomicAdd(sched, 1);
+          if (i >= n_items) {
+            it.nchunks = 0;
+            break;
+          }
+          if (load_item(p, num_seqs, tiles, i, it)) break;
+        }
+        ring_items[slot] = it;
+        mbar_arrive(item_full + slot);
+        if (QT && it.nchunks > 0) {
+#pragma unroll
+          for (int t = 0; t < kTiles; ++t)
+#pragma unroll
+            for (int pc = 0; pc < C::kPlanes; ++pc)
+              tma_prefetch_q(&tmap_q, pc * 64, it.h * g, it.q0 + (it.row0 + kRows * t) / g);
+        }
+      }
+      __syncwarp();
+      cur = ring_items[slot];
+      return cur.nchunks > 0;
+    };
+    bool have = publish();
+    for (int j = 0, c = 0; have && ok; ++j) {
+      const int stage = j % kNS;
+      const uint32_t phase = (uint32_t)(j / kNS) & 1u;
       const int c0 = c * kChunk;
-      const int nblk = (min(kChunk, kv_end - c0) + bs - 1) / bs;
+      const int nblk = (min(kChunk, cur.kv_end - c0) + bs - 1) / bs;
+      const int32_t* bt = p.block_table + (int64_t)cur.seq * p.max_blocks_per_seq;
       const int blk = lane < nblk ? __ldg(bt + c0 / bs + lane) : 0;
       if (lane == 0) ok = wait5(empty + stage, phase ^ 1u, abort);
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -318,13 +467,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (blk < 0 || blk >= p.num_blocks) atomicOr(&g_pf5_status, 2);  // reads as zeros
 #pragma unroll
         for (int pc = 0; pc < C::kPlanes; ++pc) {
-          tma_load_5d(st + pc * C::kPlaneKV + lane * piece, &tmap_k, 0, 0, pc, h, blk, full + stage);
-          tma_load_5d(st + C::kKV + pc * C::kPlaneKV + lane * piece, &tmap_v, 0, 0, pc, h, blk,
+          tma_load_5d(st + pc * C::kPlaneKV + lane * piece, &tmap_k, 0, 0, pc, cur.h, blk,
                       full + stage);
+          tma_load_5d(st + C::kKV + pc * C::kPlaneKV + lane * piece, &tmap_v, 0, 0, pc, cur.h,
+                      blk, full + stage);
         }
       }
       armed |= 1u << stage;
       last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+      if (++c >= cur.nchunks) {
+        c = 0;
+        have = publish();
+      }
     }
     if (!ok && lane == 0) {  // wait, bounded, for this CTA's copies in flight
       for (int s = 0; s < kNS; ++s) {
@@ -336,70 +490,84 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kMmaWarp) {
     // ----------------------------------------------------------------- MMA ----
-    // Warp kMmaWarp + t serves tile t: S of the first two chunks up front (one
-    // S buffer each), then per chunk c: O_t += P_t(c) V(c) once the tile's
-    // softmax has written P(c) over its S buffer, then S_t(c + 2) into that
-    // buffer, while S(c + 1), in the other buffer, was computed during the
-    // softmax of chunk c. The whole warp runs the loop on warp-uniform
-    // operands; one elected thread issues.
+    // Warp kMmaWarp + t serves tile t over the chunk sequence of all this
+    // CTA's items: S of chunks 0 and 1 up front (one S buffer each), then per
+    // chunk j: O_t += P_t(j) V(j) once the tile's softmax has written P(j)
+    // over its S buffer, then S_t(j + 2) into that buffer (of the next item
+    // when j + 2 is past this one's end: its Q is waited for first), while
+    // S(j + 1), in the other buffer, was computed during the softmax of chunk
+    // j. Past the last chunk a commit alone stands in for S(j + 2). The whole
+    // warp runs the loop on warp-uniform operands; one elected thread issues.
     constexpr uint32_t idS = idesc<T>(kRows, kChunk, false);
     constexpr uint32_t idO = idesc<T>(kRows, D, true);
     const uint32_t q_addr = smem_u32(qs), r_addr = smem_u32(ring);
     const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
     const bool leader = elect_one();
+    const int t = warp - kMmaWarp;  // this warp issues the MMAs of tile t
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, wait5(bar, parity, abort));
     };
-    auto issue_s = [&](int c, int t) {  // S_t(c) = Q_t K(c)^T into buffer c % 2
+    auto issue_s = [&](int j) {  // S_t(j) = Q_t K(j)^T into buffer j % 2
       // Base descriptors once; the K steps add compile-time offsets to the
       // 14-bit address field (addresses stay below 256 KB, so it never carries).
       const uint64_t a0 = sdesc(q_addr + t * C::kQ, 16);
-      const uint64_t b0 = sdesc(r_addr + (c % kNS) * C::kStage, 16);
-      const uint32_t dS = tm + 128 * t + 64 * (c & 1);
+      const uint64_t b0 = sdesc(r_addr + (j % kNS) * C::kStage, 16);
+      const uint32_t dS = tm + 128 * t + 64 * (j & 1);
 #pragma unroll
       for (int s = 0; s < D / 16; ++s) {
         const int pc = s / 4, off = (s % 4) * 32;
         umma(dS, a0 + (uint64_t)((pc * C::kPlaneQ + off) >> 4),
              b0 + (uint64_t)((pc * C::kPlaneKV + off) >> 4), idS, s > 0 ? 1u : 0u);
       }
-      umma_commit(s_full + 2 * t + (c & 1));
+      umma_commit(s_full + 2 * t + (j & 1));
     };
-    auto issue_pv = [&](int c, int t) {  // O_t += P_t(c) V(c)
-      const uint64_t b0 = sdesc(r_addr + (c % kNS) * C::kStage + C::kKV, C::kPlaneKV);
-      const uint32_t dO = tm + C::kColO + t * D, aP = tm + 128 * t + 64 * (c & 1);
+    auto issue_pv = [&](int j, bool acc) {  // O_t (+)= P_t(j) V(j)
+      const uint64_t b0 = sdesc(r_addr + (j % kNS) * C::kStage + C::kKV, C::kPlaneKV);
+      const uint32_t dO = tm + C::kColO + t * D, aP = tm + 128 * t + 64 * (j & 1);
 #pragma unroll
       for (int s = 0; s < kChunk / 16; ++s)
         umma_ts(dO, aP + 8 * s, b0 + (uint64_t)((s * 16 * 128) >> 4), idO,
-                (c > 0 || s > 0) ? 1u : 0u);
+                (acc || s > 0) ? 1u : 0u);
     };
-    const int t = warp - kMmaWarp;  // this warp issues the MMAs of tile t
-    bool ok = t < ntiles && wait_warp(q_full, 0);
-    tc_fence_after();
-    for (int c = 0; c < 2 && c < nchunks && ok; ++c) {
-      ok = wait_warp(full + c % kNS, (uint32_t)(c / kNS) & 1u);
-      if (!ok) break;
-      tc_fence_after();
-      if (leader) issue_s(c, t);
-      __syncwarp();
-    }
-    for (int c = 0; c < nchunks && ok; ++c) {
-      ok = wait_warp(p_full + 2 * t + (c & 1), (uint32_t)(c >> 1) & 1u);
-      if (!ok) break;
-      tc_fence_after();
-      if (leader) {
-        issue_pv(c, t);
-        umma_commit(empty + c % kNS);
-      }
-      __syncwarp();
-      if (c + 2 < nchunks) {
-        ok = wait_warp(full + (c + 2) % kNS, (uint32_t)((c + 2) / kNS) & 1u);
-        if (!ok) break;
-        tc_fence_after();
-        if (leader) issue_s(c + 2, t);
+    Walk pv, sn;  // the chunk of the next PV, and of the next S (two ahead)
+    pv.start(ring_items, item_full, abort);
+    sn.start(ring_items, item_full, abort);
+    int js = 0, q_items = 0;
+    auto next_s = [&]() -> bool {
+      if (!sn.ok) {  // past the last chunk
+        if (leader) umma_commit(s_full + 2 * t + (js & 1));
         __syncwarp();
-      } else if (leader) {
-        umma_commit(s_full + 2 * t + (c & 1));  // stand-in for S(c + 2): PV(c) has completed
+        ++js;
+        return true;
       }
+      if (sn.c == 0) {  // the first S of an item: its Q must be staged
+        if (!wait_warp(q_full + t, (uint32_t)q_items & 1u)) return false;
+        ++q_items;
+      }
+      // K of chunk js (waited for only now, so the PV before never waits on a copy).
+      if (!wait_warp(full + js % kNS, (uint32_t)(js / kNS) & 1u)) return false;
+      tc_fence_after();
+      if (leader) issue_s(js);
+      __syncwarp();
+      ++js;
+      sn.advance();
+      return true;
+    };
+    bool ok = !pv.ok || (next_s() && next_s());
+    for (int j = 0; pv.ok && ok; ++j) {
+      ok = wait_warp(p_full + 2 * t + (j & 1), (uint32_t)(j >> 1) & 1u);
+      if (!ok) break;
+      tc_fence_after();
+      const bool last = pv.c == pv.nchunks - 1;
+      if (leader) {
+        issue_pv(j, pv.c > 0);
+        umma_commit(empty + j % kNS);
+        if (last) umma_commit(o_done + t);
+      }
+      __syncwarp();
+      ok = next_s();
+      if (last && lane == 0) mbar_arrive(item_empty + pv.ii % kRing);  // done with its record
+      pv.advance();
     }
     // Whatever happened, wait (bounded) until every MMA issued has completed.
     if (leader) {
@@ -413,145 +581,207 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------- softmax ----
     const int t = warp / 4;                 // this warp's tile
     const int r = 32 * (warp % 4) + lane;   // this thread's tensor-memory lane and row of the tile
-    const int R = row0 + kRows * t + r;
-    const bool valid = R < rows;
-    const int tok = valid ? R / g : 0, j = valid ? R - tok * g : 0;
-    const int pos = valid ? base_pos + tok : -1;
     const uint32_t trow = tmem + ((uint32_t)(32 * (warp % 4)) << 16);
     const uint32_t tO = trow + C::kColO + t * D;
-    // Stage this row of Q (zeros past the chunk) in the operand layout.
-    {
-      uint8_t* qt = qs + t * C::kQ;
+    const uint32_t qt = smem_u32(qs + t * C::kQ);
+    // This thread's row of Q of an item (zeros past its rows), copied into the
+    // operand layout without passing through registers; q_ready() publishes it.
+    auto stage_q = [&](const Item& it) {
+      const int R = it.row0 + kRows * t + r;
+      const bool valid = R < it.rows;
+      const int tok = valid ? R / g : 0, jh = valid ? R - tok * g : 0;
       const uint4* src = reinterpret_cast<const uint4*>(
-          static_cast<const T*>(p.query) + ((int64_t)(q0 + tok) * Hq + h * g + j) * D);
+          static_cast<const T*>(p.query) + ((int64_t)(it.q0 + tok) * Hq + it.h * g + jh) * D);
 #pragma unroll
-      for (int u = 0; u < D / 8; ++u) {
-        const uint4 v = valid ? __ldg(src + u) : make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(qt + (u >> 3) * C::kPlaneQ + sw(r, u & 7)) = v;
-      }
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_arrive(q_full);
+      for (int u = 0; u < D / 8; ++u)
+        cp_async16(qt + (u >> 3) * C::kPlaneQ + sw(r, u & 7), valid ? src + u : p.query, valid);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    auto q_ready = [&]() {
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(q_full + t);
+    };
+    // With TMA one thread of the tile loads (or prefetches into L2) an item's Q.
+    const bool q_thread = r == 0;
+    int q_loads = 0;  // Q copies this thread has issued
+    auto load_q_tma = [&](const Item& it) {
+      ++q_loads;
+      const int z = it.q0 + (it.row0 + kRows * t) / g;
+      mbar_expect_tx(q_full + t, (uint32_t)C::kQ);
+#pragma unroll
+      for (int pc = 0; pc < C::kPlanes; ++pc)
+        tma_load_q(qs + t * C::kQ + pc * C::kPlaneQ, &tmap_q, pc * 64, it.h * g, z, q_full + t);
+    };
     const float sscale = p.score_scale;
-    float m_use = -INFINITY;
-    uint64_t lsum2 = 0;
-    bool ok = t < ntiles;
-    for (int c = 0; c < nchunks && ok; ++c) {
-      ok = wait5(s_full + 2 * t + (c & 1), (uint32_t)(c >> 1) & 1u, abort);
-      if (!__all_sync(0xffffffffu, ok)) {
-        ok = false;
-        break;
+    Walk w;
+    w.start(ring_items, item_full, abort);
+    if (w.ok) {
+      if (QT) {
+        if (q_thread) load_q_tma(w.it());
+      } else {
+        stage_q(w.it());
+        q_ready();
       }
-      tc_fence_after();
-      const uint32_t tS = trow + 128 * t + 64 * (c & 1);
-      float s[64];
-      tmem_ld64(tS, s);
-      const int c0 = c * kChunk;
-      // Raw scores; the causal mask only where the chunk reaches past a row's
-      // position. The scale is applied with the exponent (it is positive, so the
-      // maximum of the raw scores gives the maximum of the scaled ones).
-      if (__any_sync(0xffffffffu, c0 + kChunk - 1 > pos)) {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) s[i] = c0 + i <= pos ? s[i] : -INFINITY;
-      }
-      const float mx = max64(s) * sscale;
-      // Raise the running maximum only when this chunk exceeds it by 2^8.
-      const bool raise = mx > m_use + 8.f;
-      const bool rescale = raise && m_use != -INFINITY;
-      // The PV of the previous chunk must have completed before O is rescaled:
-      // the commit of S(c + 1) (or of its stand-in) follows it.
-      if (__any_sync(0xffffffffu, rescale)) {
-        if (c > 0) {
-          ok = wait5(s_full + 2 * t + ((c + 1) & 1), (uint32_t)((c + 1) >> 1) & 1u, abort);
-          if (!__all_sync(0xffffffffu, ok)) {
-            ok = false;
-            break;
+    }
+    bool ok = true;
+    int j = 0, items = 0;
+    while (w.ok && ok) {
+      const int nchunks = w.it().nchunks, kv_end = w.it().kv_end;
+      const int R = w.it().row0 + kRows * t + r;
+      const bool valid = R < w.it().rows;
+      const int tok = valid ? R / g : 0, jh = valid ? R - tok * g : 0;
+      const int pos = valid ? w.it().base_pos + tok : -1;
+      T* const dst =
+          static_cast<T*>(p.out) + ((int64_t)(w.it().q0 + tok) * Hq + w.it().h * g + jh) * D;
+      __syncwarp();  // every lane has read the record
+      if (lane == 0) mbar_arrive(item_empty + w.ii % kRing);
+      float m_use = -INFINITY;
+      uint64_t lsum2 = 0;
+      bool q_pending = false;
+      for (int c = 0; c < nchunks; ++c, ++j) {
+        ok = wait5(s_full + 2 * t + (j & 1), (uint32_t)(j >> 1) & 1u, abort);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (c == nchunks - 1) w.next_item();  // w is the next item from here on
+        if (c == nchunks - 1 && w.ok) {
+          // Every S of this item has completed (this is its last), so Q's
+          // buffer is free: fetch the next item's rows while this chunk and
+          // the epilogue run.
+          if (QT) {
+            if (q_thread) load_q_tma(w.it());
+          } else {
+            stage_q(w.it());
+            q_pending = true;
           }
-          tc_fence_after();
         }
-        const float alpha = rescale ? fast_exp2(m_use - mx) : 1.f;
-        {
-          uint64_t aa;
-          asm("mov.b64 %0, {%1, %1};" : "=l"(aa) : "f"(alpha));
-          asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(lsum2) : "l"(aa));
+        const uint32_t tS = trow + 128 * t + 64 * (j & 1);
+        float s[64];
+        tmem_ld64(tS, s);
+        const int c0 = c * kChunk;
+        // Raw scores; the causal mask only where the chunk reaches past a row's
+        // position. The scale is applied with the exponent (it is positive, so the
+        // maximum of the raw scores gives the maximum of the scaled ones).
+        if (__any_sync(0xffffffffu, c0 + kChunk - 1 > pos)) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) s[i] = c0 + i <= pos ? s[i] : -INFINITY;
         }
+        const float mx = max64(s) * sscale;
+        // Raise the running maximum only when this chunk exceeds it by 2^8.
+        const bool raise = mx > m_use + 8.f;
+        const bool rescale = raise && m_use != -INFINITY;
+        // The PV of the previous chunk must have completed before O is rescaled:
+        // the commit of S(j + 1) (or of its stand-in) follows it. At an item's
+        // last chunk S(j + 1) is the next item's first, which needs its Q.
+        if (__any_sync(0xffffffffu, rescale)) {
+          if (c > 0) {
+            if (q_pending) {
+              q_ready();
+              q_pending = false;
+            }
+            ok = wait5(s_full + 2 * t + ((j + 1) & 1), (uint32_t)((j + 1) >> 1) & 1u, abort);
+            if (!__all_sync(0xffffffffu, ok)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          const float alpha = rescale ? fast_exp2(m_use - mx) : 1.f;
+          {
+            uint64_t aa;
+            asm("mov.b64 %0, {%1, %1};" : "=l"(aa) : "f"(alpha));
+            asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(lsum2) : "l"(aa));
+          }
 #pragma unroll
-        for (int q = 0; q < D / 32; ++q) {
-          float o[32];
-          tmem_ld32(tO + 32 * q, o);
+          for (int q = 0; q < D / 32; ++q) {
+            float o[32];
+            tmem_ld32(tO + 32 * q, o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(tO + 32 * q, o);
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(tO + 32 * q, o);
+          }
+        }
+        if (raise) m_use = mx;
+        const float msub = m_use == -INFINITY ? 0.f : m_use;
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          float x0, x1;  // s * scale - m for a pair, as one packed f32x2 FMA
+          {
+            uint64_t xy, sc, mm, rr;
+            asm("mov.b64 %0, {%1, %2};" : "=l"(xy) : "f"(s[2 * i]), "f"(s[2 * i + 1]));
+            asm("mov.b64 %0, {%1, %1};" : "=l"(sc) : "f"(sscale));
+            asm("mov.b64 %0, {%1, %1};" : "=l"(mm) : "f"(-msub));
+            asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rr) : "l"(xy), "l"(sc), "l"(mm));
+            asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(rr));
+          }
+          float lo, hi;  // the row sums take P as the tensor cores see it (rounded)
+          pk[i] = Mma<T>::pack(fast_exp2(x0), fast_exp2(x1), lo, hi);
+          {
+            uint64_t pp;
+            asm("mov.b64 %0, {%1, %2};" : "=l"(pp) : "f"(lo), "f"(hi));
+            asm("add.rn.f32x2 %0, %0, %1;" : "+l"(lsum2) : "l"(pp));
+          }
+        }
+        if (c == nchunks - 1 && c0 + kChunk > kv_end) {
+          // Zero V rows past the range (stale or poisoned) before this tile's
+          // last PV. Both tiles do it, as their PVs are issued independently
+          // (the other tile's stores write the same zeros).
+          uint8_t* v = ring + (j % kNS) * C::kStage + C::kKV;
+          const int t0 = kv_end - c0, per_row = 8 * C::kPlanes;
+          for (int e = r; e < (kChunk - t0) * per_row; e += kRows) {
+            const int tk = t0 + e / per_row, u = e % per_row;
+            *reinterpret_cast<uint4*>(v + (u >> 3) * C::kPlaneKV + tk * 128 + (u & 7) * 16) =
+                make_uint4(0, 0, 0, 0);
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
+        // P over the first 32 columns of this chunk's S buffer (S is in registers).
+        tmem_st32(tS, pk);
+        tc_fence_before();
+        mbar_arrive(p_full + 2 * t + (j & 1));
+        if (q_pending) {
+          q_ready();
+          q_pending = false;
         }
       }
-      if (raise) m_use = mx;
-      const float msub = m_use == -INFINITY ? 0.f : m_use;
-      uint32_t pk[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        float x0, x1;  // s * scale - m for a pair, as one packed f32x2 FMA
-        {
-          uint64_t xy, sc, mm, rr;
-          asm("mov.b64 %0, {%1, %2};" : "=l"(xy) : "f"(s[2 * i]), "f"(s[2 * i + 1]));
-          asm("mov.b64 %0, {%1, %1};" : "=l"(sc) : "f"(sscale));
-          asm("mov.b64 %0, {%1, %1};" : "=l"(mm) : "f"(-msub));
-          asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rr) : "l"(xy), "l"(sc), "l"(mm));
-          asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(rr));
-        }
-        float lo, hi;  // the row sums take P as the tensor cores see it (rounded)
-        pk[i] = Mma<T>::pack(fast_exp2(x0), fast_exp2(x1), lo, hi);
-        {
-          uint64_t pp;
-          asm("mov.b64 %0, {%1, %2};" : "=l"(pp) : "f"(lo), "f"(hi));
-          asm("add.rn.f32x2 %0, %0, %1;" : "+l"(lsum2) : "l"(pp));
-        }
-      }
-      if (c == nchunks - 1 && c0 + kChunk > kv_end) {
-        // Zero V rows past the range (stale or poisoned) before this tile's
-        // last PV. Both tiles do it, as their PVs are issued independently
-        // (the other tile's stores write the same zeros).
-        uint8_t* v = ring + (c % kNS) * C::kStage + C::kKV;
-        const int t0 = kv_end - c0, per_row = 8 * C::kPlanes;
-        for (int e = r; e < (kChunk - t0) * per_row; e += kRows) {
-          const int tk = t0 + e / per_row, u = e % per_row;
-          *reinterpret_cast<uint4*>(v + (u >> 3) * C::kPlaneKV + tk * 128 + (u & 7) * 16) =
-              make_uint4(0, 0, 0, 0);
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      }
-      // P over the first 32 columns of this chunk's S buffer (S is in registers).
-      tmem_st32(tS, pk);
-      tc_fence_before();
-      mbar_arrive(p_full + 2 * t + (c & 1));
-    }
-    if (ok) {  // the stand-in commit of "chunk n + 1": every PV of the tile has completed
-      ok = wait5(s_full + 2 * t + ((nchunks + 1) & 1), (uint32_t)((nchunks + 1) >> 1) & 1u, abort);
+      if (!ok) break;
+      // Every PV of the item has completed: O is final.
+      ok = wait5(o_done + t, (uint32_t)items & 1u, abort);
       ok = __all_sync(0xffffffffu, ok);
-    }
-    if (ok) {
+      ++items;
+      if (!ok) break;
       tc_fence_after();
       float l0, l1;
       asm("mov.b64 {%0, %1}, %2;" : "=f"(l0), "=f"(l1) : "l"(lsum2));
       const float lsum = l0 + l1;
       const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-      T* dst = static_cast<T*>(p.out) + ((int64_t)(q0 + tok) * Hq + h * g + j) * D;
 #pragma unroll
-      for (int q = 0; q < D / 32; ++q) {
-        float o[32];
-        tmem_ld32(tO + 32 * q, o);
+      for (int q = 0; q < D / 64; ++q) {
+        float o[64];
+        tmem_ld64(tO + 64 * q, o);  // two loads in flight, one wait
         if (valid) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            uint4 w;
+          for (int u = 0; u < 8; ++u) {
+            uint4 wv;
             float a, b;
-            w.x = Mma<T>::pack(o[8 * u + 0] * inv, o[8 * u + 1] * inv, a, b);
-            w.y = Mma<T>::pack(o[8 * u + 2] * inv, o[8 * u + 3] * inv, a, b);
-            w.z = Mma<T>::pack(o[8 * u + 4] * inv, o[8 * u + 5] * inv, a, b);
-            w.w = Mma<T>::pack(o[8 * u + 6] * inv, o[8 * u + 7] * inv, a, b);
-            *reinterpret_cast<uint4*>(dst + 32 * q + 8 * u) = w;
+            wv.x = Mma<T>::pack(o[8 * u + 0] * inv, o[8 * u + 1] * inv, a, b);
+            wv.y = Mma<T>::pack(o[8 * u + 2] * inv, o[8 * u + 3] * inv, a, b);
+            wv.z = Mma<T>::pack(o[8 * u + 4] * inv, o[8 * u + 5] * inv, a, b);
+            wv.w = Mma<T>::pack(o[8 * u + 6] * inv, o[8 * u + 7] * inv, a, b);
+            *reinterpret_cast<uint4*>(dst + 64 * q + 8 * u) = wv;
           }
         }
       }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // nothing left in flight on any path
+    if (QT && q_thread && q_loads > 0) {  // nor a Q copy (an aborted call may not have used it)
+      const long long t0 = clock64();
+      while (!mbar_try(q_full + t, (uint32_t)(q_loads - 1) & 1u))
+        if (clock64() - t0 > kWaitCycles) break;
     }
   }
   tc_fence_before();
@@ -561,27 +791,96 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(kTmemCols));
   }
+  if (threadIdx.x == 0) {  // the last CTA of the launch leaves the work counter at 0
+    __threadfence();
+    if (atomicAdd(sched + 1, 1) == (int)gridDim.x - 1) {
+      atomicExch(sched, 0);
+      atomicExch(sched + 1, 0);
+    }
+  }
 }
 
-template <typename T, int D>
+// The work counter of the next launch: each launch takes the next of
+// kSchedSlots (the last CTA of a launch resets its slot), so up to kSchedSlots
+// calls may be in flight at once, on any streams.
+cudaError_t next_sched_slot(int dev, int** sched) {
+  static std::atomic<unsigned> launches{0};
+  static std::atomic<int*> base[64];
+  int* b = base[dev].load(std::memory_order_relaxed);
+  if (!b) {
+    void* a = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&a, g_pf5_sched);
+    if (e != cudaSuccess) return e;
+    b = static_cast<int*>(a);
+    base[dev].store(b, std::memory_order_relaxed);
+  }
+  *sched = b + 2 * (int)(launches.fetch_add(1, std::memory_order_relaxed) % kSchedSlots);
+  return cudaSuccess;
+}
+
+template <typename T, int D, bool QT>
 cudaError_t launch5(const PrefillParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
-                    int num_seqs, cudaStream_t stream) {
+                    const CUtensorMap& mq, int num_seqs, cudaStream_t stream) {
   using C = Cfg5<D>;
-  auto kernel = prefill_tc5_kernel<T, D>;
+  auto kernel = prefill_tc5_kernel<T, D, QT>;
   static std::atomic<int> opted_in[64];  // the shared-memory opt-in, once per device
+  static std::atomic<int> sm_count[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!opted_in[dev].load(std::memory_order_relaxed)) {
-    const cudaError_t e =
+    cudaError_t e =
         cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
+    int n = 0;
+    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    sm_count[dev].store(n > 0 ? n : 1, std::memory_order_relaxed);
     opted_in[dev].store(1, std::memory_order_relaxed);
   }
   const int g = p.num_heads / p.num_kv_heads;
   const int64_t tiles = ((int64_t)p.max_q_len * g + kCtaRows - 1) / kCtaRows;
-  dim3 grid((unsigned)tiles, (unsigned)num_seqs, (unsigned)p.num_kv_heads);
-  kernel<<<grid, kThreads, C::kSmem, stream>>>(p, mk, mv);
+  const int64_t n_items = tiles * num_seqs * p.num_kv_heads;
+  if (n_items <= 0) return cudaSuccess;
+  if (n_items > (int64_t)INT32_MAX / 2) return cudaErrorInvalidValue;
+  // Persistent: one CTA per SM (a CTA fills one), each walking items
+  // blockIdx.x, + gridDim.x, ... so that the next item's Q and K/V stream in
+  // while the current one finishes.
+  // Persistent: one CTA per SM (a CTA fills one), each taking the launch's
+  // items from a work counter as it becomes free.
+  int* sched = nullptr;
+  const cudaError_t es = next_sched_slot(dev, &sched);
+  if (es != cudaSuccess) return es;
+  const int64_t grid = std::min<int64_t>(n_items, sm_count[dev].load(std::memory_order_relaxed));
+  kernel<<<(unsigned)grid, kThreads, C::kSmem, stream>>>(p, mk, mv, mq, num_seqs, (int)tiles,
+                                                         (int)n_items, sched);
   return cudaGetLastError();
+}
+
+// The query tensor (head_dim, heads, tokens) for Q tiles by TMA: box (64, g,
+// 128 / g) in the 128B swizzle. False when g does not divide 128.
+bool encode_q_map(CUtensorMap* map, const PrefillParams& p, int head_dim, bool bf16) {
+  const int g = p.num_heads / p.num_kv_heads;
+  if (kRows % g != 0) return false;
+  auto enc = tcx::tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)p.num_heads,
+                        (cuuint64_t)p.num_q_tokens};
+  cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, (cuuint64_t)p.num_heads * head_dim * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)g, (cuuint32_t)(kRows / g)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+             const_cast<void*>(p.query), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T, int D>
+cudaError_t launch5q(const PrefillParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
+                     int num_seqs, cudaStream_t stream) {
+  CUtensorMap mq;
+  if (encode_q_map(&mq, p, D, std::is_same<T, __nv_bfloat16>::value))
+    return launch5<T, D, true>(p, mk, mv, mq, num_seqs, stream);
+  return launch5<T, D, false>(p, mk, mv, mk, num_seqs, stream);  // mk unused as Q map
 }
 
 }  // namespace
@@ -591,10 +890,10 @@ bool prefill_tc5_supported(int head_dim) { return head_dim == 64 || head_dim == 
 cudaError_t launch_prefill_tc5(const PrefillParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
                                int head_dim, bool bf16, int num_seqs, cudaStream_t stream) {
   if (bf16)
-    return head_dim == 128 ? launch5<__nv_bfloat16, 128>(p, mk, mv, num_seqs, stream)
-                           : launch5<__nv_bfloat16, 64>(p, mk, mv, num_seqs, stream);
-  return head_dim == 128 ? launch5<__half, 128>(p, mk, mv, num_seqs, stream)
-                         : launch5<__half, 64>(p, mk, mv, num_seqs, stream);
+    return head_dim == 128 ? launch5q<__nv_bfloat16, 128>(p, mk, mv, num_seqs, stream)
+                           : launch5q<__nv_bfloat16, 64>(p, mk, mv, num_seqs, stream);
+  return head_dim == 128 ? launch5q<__half, 128>(p, mk, mv, num_seqs, stream)
+                         : launch5q<__half, 64>(p, mk, mv, num_seqs, stream);
 }
 
 }  // namespace pf
