@@ -243,3 +243,80 @@ def test_prefill_fp8_out_of_pool_and_prefix_hit_matches_decode(cuda_dev):
                                max_seq_len=500, scale=128 ** -0.5, k_scale=sc, v_scale=sc)
     torch.cuda.synchronize()
     assert (got[last:last + 1].float() - out.float()).abs().max().item() <= 2 * TOL["e4m3"][0]
+
+
+def _device_args(c):
+    dev = c["dev"]
+    return (torch.from_numpy(c["bt"]).to(dev), torch.from_numpy(c["lens"]).to(dev),
+            torch.from_numpy(c["qs"]).to(dev), int(np.diff(c["qs"]).max()))
+
+
+def test_prefill_repeated_calls_and_graph_replays_reuse_work_counters(cuda_dev):
+    # The tcgen05 kernel is persistent: its CTAs take items from a work counter
+    # that each call takes from a ring of 64 and that the call's last CTA puts
+    # back to zero. More calls than the ring holds, and replays of a captured
+    # graph (which keeps its calls' counters), must all compute every item.
+    c = make_case([300, 257, 64, 500, 33, 129], [300, 100, 64, 200, 33, 1], 32, 8, 128, 16,
+                  "bf16", cuda_dev, seed=5)
+    bt, lens, qs, mq = _device_args(c)
+    want = run_oracle(c)
+    outs = [torch.full(tuple(c["q"].shape), float("nan"), dtype=c["q"].dtype, device=cuda_dev)
+            for _ in range(3)]
+
+    def call(out):
+        pkv.paged_attention_prefill(out, c["q"], c["kc"], c["vc"], bt, lens, qs, max_q_len=mq,
+                                    scale=c["D"] ** -0.5)
+
+    call(outs[0])
+    torch.cuda.synchronize()
+    first = outs[0].clone()
+    check(first, want, "bf16")
+    for _ in range(70):
+        call(outs[0])
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], first)
+    for o in outs:
+        o.fill_(float("nan"))
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        call(outs[0])  # warm-up outside the capture
+        s.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for o in outs:
+                pkv.paged_attention_prefill(o, c["q"], c["kc"], c["vc"], bt, lens, qs,
+                                            max_q_len=mq, scale=c["D"] ** -0.5, stream=s)
+    for _ in range(5):
+        for o in outs:
+            o.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        for o in outs:
+            assert torch.equal(o, first)
+    assert pkv.pkv_device_status(clear=True) == 0
+
+
+def test_prefill_concurrent_calls_on_two_streams(cuda_dev):
+    # Calls in flight at the same time on different streams use different work
+    # counters and must not take each other's items.
+    a = make_case([700, 300, 90], [700, 40, 90], 16, 2, 128, 16, "bf16", cuda_dev, seed=21)
+    b = make_case([200, 1000, 64, 64], [200, 128, 1, 64], 64, 8, 64, 32, "f16", cuda_dev,
+                  seed=22)
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = []
+    for c, s in zip((a, b), streams):
+        bt, lens, qs, mq = _device_args(c)
+        o = [torch.full(tuple(c["q"].shape), float("nan"), dtype=c["q"].dtype, device=cuda_dev)
+             for _ in range(4)]
+        outs.append((c, bt, lens, qs, mq, s, o))
+    torch.cuda.synchronize()
+    for k in range(4):  # interleaved launches, no synchronisation between the streams
+        for c, bt, lens, qs, mq, s, o in outs:
+            pkv.paged_attention_prefill(o[k], c["q"], c["kc"], c["vc"], bt, lens, qs,
+                                        max_q_len=mq, scale=c["D"] ** -0.5, stream=s)
+    torch.cuda.synchronize()
+    assert pkv.pkv_device_status(clear=True) == 0
+    for c, bt, lens, qs, mq, s, o in outs:
+        want = run_oracle(c)
+        for k in range(4):
+            check(o[k], want, c["dt"])
