@@ -320,3 +320,13 @@ def test_prefill_concurrent_calls_on_two_streams(cuda_dev):
         want = run_oracle(c)
         for k in range(4):
             check(o[k], want, c["dt"])
+
+
+def test_prefill_many_one_chunk_items(cuda_dev):
+    # 300 short sequences give a few thousand one-chunk items: each CTA of the
+    # persistent kernel takes many more than its ring of item records holds.
+    rng = np.random.default_rng(9)
+    lens = [int(x) for x in rng.integers(1, 60, size=300)]
+    qlens = [int(min(L, q)) for L, q in zip(lens, rng.integers(1, 4, size=300))]
+    c = make_case(lens, qlens, 32, 8, 128, 16, "bf16", cuda_dev, seed=9)
+    check(run_gpu(c), run_oracle(c), "bf16")
