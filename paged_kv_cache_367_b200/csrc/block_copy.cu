@@ -20,36 +20,74 @@ constexpr int kCopyThreads = 256;
 constexpr int kCopyVecs = 4;                                   // 16-byte vectors per thread
 constexpr int64_t kPiece = (int64_t)kCopyThreads * kCopyVecs * 16;  // bytes per work item
 
-// Work item = (pair, K or V, piece of kPiece bytes). Each thread keeps its
-// kCopyVecs loads in flight before storing.
+// Work item = (pair, K or V, piece of kPiece bytes), items strided over the
+// grid. Software-pipelined: each thread issues its kCopyVecs loads of the next
+// item before storing the current one, so loads are in flight during the
+// stores (4% faster than load-then-store per item on 4096 scattered pairs).
+struct Piece {
+  const uint8_t* s;
+  uint8_t* d;
+  int64_t len;
+};
+
+__device__ __forceinline__ bool locate(int64_t it, const uint8_t* sk, const uint8_t* sv,
+                                       uint8_t* dk, uint8_t* dv, const int64_t* map,
+                                       int64_t block_bytes, int64_t src_blocks,
+                                       int64_t dst_blocks, int64_t pieces, Piece& pc) {
+  const int64_t pair = it / (2 * pieces);
+  const int64_t rem = it - pair * 2 * pieces;
+  const int tensor = (int)(rem / pieces);
+  const int64_t piece = rem - tensor * pieces;
+  const int64_t src = __ldg(map + 2 * pair), dst = __ldg(map + 2 * pair + 1);
+  if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) return false;
+  const int64_t base = piece * kPiece;
+  pc.len = min(kPiece, block_bytes - base);
+  pc.s = (tensor ? sv : sk) + src * block_bytes + base;
+  pc.d = (tensor ? dv : dk) + dst * block_bytes + base;
+  return true;
+}
+
 __global__ void __launch_bounds__(kCopyThreads)
     block_copy_kernel(const uint8_t* __restrict__ sk, const uint8_t* __restrict__ sv,
                       uint8_t* __restrict__ dk, uint8_t* __restrict__ dv,
                       const int64_t* __restrict__ map, int n, int64_t block_bytes,
                       int64_t src_blocks, int64_t dst_blocks, int64_t pieces) {
   const int64_t items = (int64_t)n * 2 * pieces;
-  for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
-    const int64_t pair = it / (2 * pieces);
-    const int64_t rem = it - pair * 2 * pieces;
-    const int tensor = (int)(rem / pieces);
-    const int64_t piece = rem - tensor * pieces;
-    const int64_t src = __ldg(map + 2 * pair), dst = __ldg(map + 2 * pair + 1);
-    if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) continue;
-    const int64_t base = piece * kPiece;
-    const int64_t len = min(kPiece, block_bytes - base);
-    const uint8_t* s = (tensor ? sv : sk) + src * block_bytes + base;
-    uint8_t* d = (tensor ? dv : dk) + dst * block_bytes + base;
-    int4 r[kCopyVecs];
+  // The next valid item at or after `it` (pairs out of range are skipped).
+  auto next = [&](int64_t& it, Piece& pc) -> bool {
+    for (; it < items; it += gridDim.x)
+      if (locate(it, sk, sv, dk, dv, map, block_bytes, src_blocks, dst_blocks, pieces, pc)) {
+        it += gridDim.x;
+        return true;
+      }
+    return false;
+  };
+  auto load = [&](const Piece& pc, int4 (&r)[kCopyVecs]) {
 #pragma unroll
     for (int v = 0; v < kCopyVecs; ++v) {
       const int64_t off = (int64_t)(v * kCopyThreads + threadIdx.x) * 16;
-      if (off < len) r[v] = __ldcs(reinterpret_cast<const int4*>(s + off));
+      if (off < pc.len) r[v] = __ldcs(reinterpret_cast<const int4*>(pc.s + off));
     }
+  };
+  int64_t it = blockIdx.x;
+  Piece cur;
+  int4 r[kCopyVecs];
+  bool have = next(it, cur);
+  if (have) load(cur, r);
+  while (have) {
+    Piece nxt;
+    int4 r2[kCopyVecs];
+    const bool have2 = next(it, nxt);
+    if (have2) load(nxt, r2);
 #pragma unroll
     for (int v = 0; v < kCopyVecs; ++v) {
       const int64_t off = (int64_t)(v * kCopyThreads + threadIdx.x) * 16;
-      if (off < len) __stcs(reinterpret_cast<int4*>(d + off), r[v]);
+      if (off < cur.len) __stcs(reinterpret_cast<int4*>(cur.d + off), r[v]);
     }
+#pragma unroll
+    for (int v = 0; v < kCopyVecs; ++v) r[v] = r2[v];
+    cur = nxt;
+    have = have2;
   }
 }
 
