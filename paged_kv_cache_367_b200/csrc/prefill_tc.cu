@@ -473,6 +473,8 @@ extern "C" int paged_attention_prefill(void* out, const void* query, const void*
                                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   // E4M3 caches run on the mma.sync kernel, widened in registers.
   const bool tc5 = !f8 && !(flags & PKV_PREFILL_MMA_SYNC) && pf::prefill_tc5_supported(head_dim);
+  // The tcgen05 kernel numbers its items (tile pairs x sequences x KV heads) in int.
+  if (tc5 && (tiles + 1) / 2 * num_seqs * num_kv_heads > INT32_MAX / 2) return PKV_ERR_SHAPE;
   const int e = f8 ? 1 : 2;
   CUtensorMap mk, mv;
   if (!tcx::encode_pool_map(&mk, k_cache, dt, e, head_dim, block_size, num_kv_heads, num_blocks,

@@ -270,9 +270,10 @@ __device__ __forceinline__ uint32_t sw(int r, int j) {
 __device__ __forceinline__ bool load_item(const PrefillParams& p, int num_seqs, int tiles, int i,
                                           Item& it) {
   const int Hkv = p.num_kv_heads, g = p.num_heads / Hkv;
-  const int per_group = kPairGroup * tiles, grp = i / per_group;
+  const int64_t per_group = (int64_t)kPairGroup * tiles;
+  const int grp = (int)(i / per_group);
   const int pg = min(kPairGroup, num_seqs * Hkv - grp * kPairGroup);
-  const int within = i - grp * per_group, xr = within / pg;
+  const int within = (int)(i - grp * per_group), xr = within / pg;
   const int pair = grp * kPairGroup + within - xr * pg;
   it.seq = pair / Hkv;
   it.h = pair - it.seq * Hkv;
