@@ -48,10 +48,12 @@
 //    j and then S of chunk j + 2 (of the next item past this one's end) into
 //    the buffer that PV reads: the MMAs of a thread run in issue order, so
 //    S(j + 2) overwrites P(j) only after the PV that read it. A K/V stage is
-//    free once both tiles' warps have committed their PV of it. After an
-//    item's last PV each thread reads its row of O, divides by its row sum and
-//    stores it; the next item's first PV overwrites O only after that, as it
-//    needs P from the same threads.
+//    free once both tiles' warps have committed their PV of it. Once an
+//    item's last PV has completed each thread reads its row of O, divides by
+//    its row sum and stores it: this epilogue runs after the next item's first
+//    chunk has been through the softmax and before that chunk's P is
+//    published, so the wait for the last PV overlaps useful work and the next
+//    item's first PV, which overwrites O, cannot start before O has been read.
 //  * The commit after S(j + 2) (past the last chunk, a commit alone) also
 //    tells a tile's softmax that PV(j) has completed: it is what O's rescale
 //    waits for. P has a barrier per S buffer, so a softmax that runs a chunk
@@ -627,6 +629,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     bool ok = true;
     int j = 0, items = 0;
+    // The previous item's O is read and stored (its epilogue) only after the
+    // next item's first chunk has been through the softmax and before that
+    // chunk's P is published: the wait for the previous item's last PV then
+    // overlaps useful work, and the next item's first PV, which overwrites O,
+    // cannot start before O has been read.
+    bool pending = false, prev_valid = false;
+    uint64_t prev_lsum = 0;
+    T* prev_dst = nullptr;
+    auto epilogue = [&]() -> bool {
+      pending = false;
+      bool okk = wait5(o_done + t, (uint32_t)items & 1u, abort);  // every PV of the item
+      okk = __all_sync(0xffffffffu, okk);
+      ++items;
+      if (!okk) return false;
+      tc_fence_after();
+      float l0, l1;
+      asm("mov.b64 {%0, %1}, %2;" : "=f"(l0), "=f"(l1) : "l"(prev_lsum));
+      const float lsum = l0 + l1;
+      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+#pragma unroll
+      for (int q = 0; q < D / 64; ++q) {
+        float o[64];
+        tmem_ld64(tO + 64 * q, o);  // two loads in flight, one wait
+        if (prev_valid) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            uint4 wv;
+            float a, b;
+            wv.x = Mma<T>::pack(o[8 * u + 0] * inv, o[8 * u + 1] * inv, a, b);
+            wv.y = Mma<T>::pack(o[8 * u + 2] * inv, o[8 * u + 3] * inv, a, b);
+            wv.z = Mma<T>::pack(o[8 * u + 4] * inv, o[8 * u + 5] * inv, a, b);
+            wv.w = Mma<T>::pack(o[8 * u + 6] * inv, o[8 * u + 7] * inv, a, b);
+            *reinterpret_cast<uint4*>(prev_dst + 64 * q + 8 * u) = wv;
+          }
+        }
+      }
+      return true;
+    };
     while (w.ok && ok) {
       const int nchunks = w.it().nchunks, kv_end = w.it().kv_end;
       const int R = w.it().row0 + kRows * t + r;
@@ -742,6 +782,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // P over the first 32 columns of this chunk's S buffer (S is in registers).
         tmem_st32(tS, pk);
+        if (c == 0 && pending && !epilogue()) {
+          ok = false;
+          break;
+        }
         tc_fence_before();
         mbar_arrive(p_full + 2 * t + (j & 1));
         if (q_pending) {
@@ -750,34 +794,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) break;
-      // Every PV of the item has completed: O is final.
-      ok = wait5(o_done + t, (uint32_t)items & 1u, abort);
-      ok = __all_sync(0xffffffffu, ok);
-      ++items;
-      if (!ok) break;
-      tc_fence_after();
-      float l0, l1;
-      asm("mov.b64 {%0, %1}, %2;" : "=f"(l0), "=f"(l1) : "l"(lsum2));
-      const float lsum = l0 + l1;
-      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-#pragma unroll
-      for (int q = 0; q < D / 64; ++q) {
-        float o[64];
-        tmem_ld64(tO + 64 * q, o);  // two loads in flight, one wait
-        if (valid) {
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            uint4 wv;
-            float a, b;
-            wv.x = Mma<T>::pack(o[8 * u + 0] * inv, o[8 * u + 1] * inv, a, b);
-            wv.y = Mma<T>::pack(o[8 * u + 2] * inv, o[8 * u + 3] * inv, a, b);
-            wv.z = Mma<T>::pack(o[8 * u + 4] * inv, o[8 * u + 5] * inv, a, b);
-            wv.w = Mma<T>::pack(o[8 * u + 6] * inv, o[8 * u + 7] * inv, a, b);
-            *reinterpret_cast<uint4*>(dst + 64 * q + 8 * u) = wv;
-          }
-        }
-      }
+      // This item's epilogue waits until the next item's first chunk has been
+      // through the softmax (or until the end).
+      prev_lsum = lsum2;
+      prev_dst = dst;
+      prev_valid = valid;
+      pending = true;
     }
+    if (ok && pending) ok = epilogue();
     asm volatile("cp.async.wait_all;" ::: "memory");  // nothing left in flight on any path
     if (QT && q_thread && q_loads > 0) {  // nor a Q copy (an aborted call may not have used it)
       const long long t0 = clock64();
