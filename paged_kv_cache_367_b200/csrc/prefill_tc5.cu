@@ -114,7 +114,8 @@ __device__ __forceinline__ float max64(const float (&s)[64]) {
 }
 
 // One unit of work: the 256 query rows row0 .. row0 + 255 of (sequence, KV
-// head); nchunks = 0 marks an empty one.
+// head) and the 64-token chunks of its causal range; a record with no chunks
+// tells the other roles that the work is gone.
 struct Item {
   int seq, h, q0, rows, row0, base_pos, kv_end, nchunks;
 };
@@ -136,7 +137,8 @@ struct Cfg5 {
   // 256 + t D.
   static constexpr uint32_t kColO = 256;
   static_assert(kColO + kTiles * D <= kTmemCols, "tensor memory per CTA");
-  // full, empty, s_full [tile][buffer], p_full [tile][buffer], q_full [tile], o_done [tile], drain
+  // full, empty, s_full [tile][buffer], p_full [tile][buffer], q_full [tile], o_done [tile],
+  // drain; then item_full and item_empty [kRing] and the ring of item records
   static constexpr int kBars = 2 * kNS + 6 * kTiles + 1;
   static constexpr int kSmem = 1024 + kNS * kStage + kTiles * kQ + kBars * 8 + 16 +
                                kRing * (16 + (int)sizeof(Item));
