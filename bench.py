@@ -867,7 +867,32 @@ def run_prefill(args, dev):
                                        "peak_source": peak_src, "unit": "TFLOP/s",
                                        "frac": round(tflops / peak, 4), "traffic": None,
                                        "flops": flops, "kernel": kname}})
-        del kc, vc, q, out
+        # The same queries over an E4M3 cache (codes as in the workload generator,
+        # per-tensor scales), on the tcgen05 kernel.
+        kc8 = (kc.float() * (448.0 / 4.0)).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+        vc8 = (vc.float() * (448.0 / 4.0)).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+        sc = torch.tensor([4.0 / 448.0], dtype=torch.float32, device=dev)
+
+        def call8():
+            pkv.paged_attention_prefill(out, q, kc8, vc8, btd, lensd, qsd, max_q_len=max(qlen),
+                                        scale=D ** -0.5, k_scale=sc, v_scale=sc)
+        ms, how = kernel_time_ms(lambda: None, call8, n=8, reps=max(3, reps // 8))
+        assert pkv.pkv_device_status(clear=True) == 0, "device wait expired"
+        tflops = flops / ms / 1e9
+        lines.append({"metric": "paged causal multi-token attention TFLOP/s",
+                      "value": round(tflops, 1), "unit": "TFLOP/s", "higher_is_better": True,
+                      "us_per_launch": round(ms * 1e3, 1), "timing": how,
+                      "tokens_per_s": round(T / ms * 1e3, 0),
+                      "dtype": "f16 MMAs over an e4m3 cache (bf16 query and output)",
+                      "data": "synthetic",
+                      "config": {"workload": name + f"; {Hq} q / {Hkv} KV heads, head_dim {D}, "
+                                                    f"block {bs}, shuffled pool, FP8-E4M3 cache"},
+                      "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak,
+                                   "peak_source": peak_src, "unit": "TFLOP/s",
+                                   "frac": round(tflops / peak, 4), "traffic": None,
+                                   "flops": flops,
+                                   "kernel": "tcgen05.mma over codes widened to f16 in shared memory"}})
+        del kc, vc, kc8, vc8, q, out
         torch.cuda.empty_cache()
     return lines
 

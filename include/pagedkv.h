@@ -247,10 +247,10 @@ int paged_attention_decode_static(void* out, const void* query, const void* k_ca
  * any streams; a CUDA graph that holds a call keeps that call's counter, so
  * replays of one graph must not overlap each other. flags PKV_PREFILL_MMA_SYNC
  * selects the mma.sync kernel (64 rows per CTA, no counter) instead; other flag
- * bits are an error. An FP8-E4M3 cache runs on
- * the mma.sync kernel: codes widened exactly to f16 in registers, the query
- * rounded to f16, k_scale folded into the score scale and v_scale into the
- * output.
+ * bits are an error. With an FP8-E4M3 cache the codes are widened exactly to
+ * f16 (in shared memory on the tcgen05 kernel, in registers on the mma.sync
+ * one), the query is rounded to f16, k_scale is folded into the score scale
+ * and v_scale into the output.
  * Errors: PKV_ERR_SHAPE, PKV_ERR_UNSUPPORTED, PKV_ERR_DTYPE, PKV_ERR_NULL,
  * PKV_ERR_ALIGN, PKV_ERR_CUDA.
  */

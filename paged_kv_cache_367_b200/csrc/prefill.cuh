@@ -25,7 +25,7 @@ struct PrefillParams {
 
 // Launch of the tcgen05 kernel (prefill_tc5.cu); mk / mv are per-plane pool maps.
 cudaError_t launch_prefill_tc5(const PrefillParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
-                               int head_dim, bool bf16, int num_seqs, cudaStream_t stream);
+                               int head_dim, bool bf16, bool f8, int num_seqs, cudaStream_t stream);
 bool prefill_tc5_supported(int head_dim);
 
 }  // namespace pf

@@ -471,8 +471,9 @@ extern "C" int paged_attention_prefill(void* out, const void* query, const void*
   const CUtensorMapDataType dt = f8                   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                  : q_dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  // E4M3 caches run on the mma.sync kernel, widened in registers.
-  const bool tc5 = !f8 && !(flags & PKV_PREFILL_MMA_SYNC) && pf::prefill_tc5_supported(head_dim);
+  // The tcgen05 kernel takes 16-bit and E4M3 caches (the latter widened to f16
+  // in shared memory); PKV_PREFILL_MMA_SYNC selects the mma.sync kernel.
+  const bool tc5 = !(flags & PKV_PREFILL_MMA_SYNC) && pf::prefill_tc5_supported(head_dim);
   // The tcgen05 kernel numbers its items (tile pairs x sequences x KV heads) in int.
   if (tc5 && (tiles + 1) / 2 * num_seqs * num_kv_heads > INT32_MAX / 2) return PKV_ERR_SHAPE;
   const int e = f8 ? 1 : 2;
@@ -502,7 +503,7 @@ extern "C" int paged_attention_prefill(void* out, const void* query, const void*
   cudaError_t err;
   const bool bf16 = q_dtype == PKV_BF16, d128 = head_dim == 128;
   if (tc5)
-    err = pf::launch_prefill_tc5(p, mk, mv, head_dim, bf16, num_seqs, st);
+    err = pf::launch_prefill_tc5(p, mk, mv, head_dim, bf16, f8, num_seqs, st);
   else if (f8 && bf16)
     err = d128 ? pf::launch_t<__nv_bfloat16, 128, true>(p, mk, mv, max_q_len, num_seqs, st)
                : pf::launch_t<__nv_bfloat16, 64, true>(p, mk, mv, max_q_len, num_seqs, st);

@@ -33,6 +33,11 @@
 //    whole tokens) is one TMA box per piece of head_dim in the same layout,
 //    loaded by one softmax thread as soon as the tile's last S of the previous
 //    item has completed; otherwise the softmax threads copy their rows.
+//  * An E4M3 cache: the producer copies a chunk's codes by TMA into a staging
+//    ring (up to three chunks ahead) and widens them, exactly, to f16 in the
+//    chunk's stage, in the layout the 16-bit path gets from TMA; the MMAs are
+//    f16 (Q rounded to f16 by the softmax threads as they stage it), k_scale
+//    is folded into the score scale and v_scale into the output.
 //  * Each tile has two S buffers in tensor memory (chunk j uses buffer j % 2):
 //    S = Q K^T of the next chunk (M 128, N 64, K 16 per instruction) is
 //    computed into one while the softmax threads work on the other, so a
@@ -123,7 +128,10 @@ constexpr int kRing = 8;        // item records in flight from the producer to t
 constexpr int kPairGroup = 8;   // (sequence, KV head) pairs whose items are handed out together
 constexpr int kSchedSlots = 64; // work counters, one per launch in flight
 
-template <int D>
+// E4M3 caches: 3 stages of widened K/V and 4 stages of codes (copied by TMA
+// up to three chunks ahead of their widening), in the same shared memory.
+
+template <int D, bool F8>
 struct Cfg5 {
   static constexpr int kPlanes = D / 64;          // 128-byte pieces of head_dim
   static constexpr int kPlaneKV = kChunk * 128;   // one piece of a K (or V) chunk
@@ -139,9 +147,17 @@ struct Cfg5 {
   static_assert(kColO + kTiles * D <= kTmemCols, "tensor memory per CTA");
   // full, empty, s_full [tile][buffer], p_full [tile][buffer], q_full [tile], o_done [tile],
   // drain; then item_full and item_empty [kRing] and the ring of item records
-  static constexpr int kBars = 2 * kNS + 6 * kTiles + 1;
-  static constexpr int kSmem = 1024 + kNS * kStage + kTiles * kQ + kBars * 8 + 16 +
-                               kRing * (16 + (int)sizeof(Item));
+  static constexpr int kNSx = F8 ? 3 : kNS;   // stages of 16-bit K/V
+  static constexpr int kNS8x = F8 ? 4 : 0;    // stages of E4M3 codes
+  static constexpr int kBars = 2 * kNSx + 6 * kTiles + 1;
+  // F8: per stage the E4M3 codes of a chunk's K, then of its V, as they land
+  // (rows of min(D, 128) bytes in the 128B (64B when D = 64) swizzle).
+  static constexpr int kRowB8 = D < 128 ? D : 128;
+  static_assert(kRowB8 == 64 || kRowB8 == 128, "E4M3 rows are one 64- or 128-byte box");
+  static constexpr int kKV8 = kChunk * D;
+  static constexpr int kStage8 = F8 ? 2 * kKV8 : 0;
+  static constexpr int kSmem = 1024 + kNSx * kStage + kNS8x * kStage8 + kTiles * kQ + kBars * 8 +
+                               kNS8x * 8 + 16 + kRing * (16 + (int)sizeof(Item));
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA exceeds 227 KB");
 };
 
@@ -353,28 +369,33 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
 
 // QT: Q is copied by TMA (g divides 128, so a tile's rows are whole tokens);
 // otherwise the softmax threads copy their rows.
-template <typename T, int D, bool QT>
+// OT: query/output type. F8: the cache holds E4M3 codes, widened to f16 in
+// shared memory by the producer; Q is rounded to f16 (the MMAs are f16).
+template <typename OT, int D, bool QT, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc5_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_v,
                        const __grid_constant__ CUtensorMap tmap_q, int num_seqs, int tiles,
                        int n_items, int* sched) {
-  using C = Cfg5<D>;
+  using T = typename std::conditional<F8, __half, OT>::type;  // MMA operand type
+  using C = Cfg5<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* ring = smem;                          // kNS stages: K pieces, V pieces
-  uint8_t* qs = ring + kNS * C::kStage;          // Q pieces of tile 0, then of tile 1
+  uint8_t* ring = smem;                          // C::kNSx stages: K pieces, V pieces
+  uint8_t* ring8 = ring + C::kNSx * C::kStage;       // F8: C::kNS8x stages of E4M3 codes
+  uint8_t* qs = ring8 + C::kNS8x * C::kStage8;       // Q pieces of tile 0, then of tile 1
   uint64_t* full = reinterpret_cast<uint64_t*>(qs + kTiles * C::kQ);
-  uint64_t* empty = full + kNS;
-  uint64_t* s_full = empty + kNS;         // [tile][buffer] S of a chunk is in tensor memory
+  uint64_t* empty = full + C::kNSx;
+  uint64_t* s_full = empty + C::kNSx;         // [tile][buffer] S of a chunk is in tensor memory
   uint64_t* p_full = s_full + 2 * kTiles;  // [tile][buffer] P of a chunk is in tensor memory
   uint64_t* q_full = p_full + 2 * kTiles;  // [tile] Q of the tile's next item is staged
   uint64_t* o_done = q_full + kTiles;      // [tile] every PV of the tile's item has completed
   uint64_t* drain = o_done + kTiles;       // every MMA issued has completed
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* full8 = drain + 1;               // F8: [C::kNS8x] E4M3 codes of a chunk have landed
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(full8 + C::kNS8x);
   volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
-  uint64_t* item_full = drain + 2;           // [kRing] a record is published
+  uint64_t* item_full = reinterpret_cast<uint64_t*>(tslot + 2);  // [kRing] a record is published
   uint64_t* item_empty = item_full + kRing;  // [kRing] every role is done with a record
   Item* ring_items = reinterpret_cast<Item*>(item_empty + kRing);
 
@@ -382,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kNS; ++s) {
+    for (int s = 0; s < C::kNSx; ++s) {
       mbar_init(full + s, 1);
       mbar_init(empty + s, kTiles);  // one commit per tile's MMA warp
     }
@@ -395,6 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(o_done + t, 1);
     }
     mbar_init(drain, kTiles);
+    if (F8)
+      for (int s = 0; s < C::kNS8x; ++s) mbar_init(full8 + s, 1);
     for (int s = 0; s < kRing; ++s) {
       mbar_init(item_full + s, 1);
       mbar_init(item_empty + s, kTiles + kSoftWarps);  // the MMA warps and the softmax warps
@@ -452,12 +475,111 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       cur = ring_items[slot];
+      if (!QT && cur.nchunks > 0) {  // its Q rows into L2 (the softmax threads copy them)
+        for (int rr = lane; rr < kCtaRows; rr += 32) {
+          const int R = cur.row0 + rr;
+          if (R >= cur.rows) break;
+          const int tk = R / g;
+          const char* qr = reinterpret_cast<const char*>(
+              static_cast<const OT*>(p.query) + ((int64_t)(cur.q0 + tk) * Hq + cur.h * g +
+                                                 (R - tk * g)) * D);
+#pragma unroll
+          for (int b = 0; b < D * (int)sizeof(OT); b += 128)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(qr + b));
+        }
+      }
       return cur.nchunks > 0;
     };
+    if constexpr (F8) {
+      // E4M3 cache: TMA copies of a chunk's codes into the staging ring run one
+      // chunk ahead of their widening (exact) to f16 in the chunk's stage, in
+      // the same layout the 16-bit path gets from TMA; then the stage is full.
+      const int piece8 = bs * C::kRowB8;  // bytes of one (block) box of codes
+      uint32_t armed8 = 0, last8 = 0;
+      int lc = 0, lj = 0;  // load cursor: chunk within `cur`, chunk index
+      bool lhave = publish();
+      auto issue_load = [&]() {
+        const int s8 = lj % C::kNS8x;
+        const int c0 = lc * kChunk;
+        const int nblk = (min(kChunk, cur.kv_end - c0) + bs - 1) / bs;
+        const int32_t* bt = p.block_table + (int64_t)cur.seq * p.max_blocks_per_seq;
+        const int blk = lane < nblk ? __ldg(bt + c0 / bs + lane) : 0;
+        uint8_t* st8 = ring8 + s8 * C::kStage8;
+        if (lane == 0) mbar_expect_tx(full8 + s8, (uint32_t)(2 * nblk * piece8));
+        __syncwarp();
+        if (lane < nblk) {
+          if (blk < 0 || blk >= p.num_blocks) atomicOr(&g_pf5_status, 2);  // reads as zeros
+          tma_load_5d(st8 + lane * piece8, &tmap_k, 0, 0, 0, cur.h, blk, full8 + s8);
+          tma_load_5d(st8 + C::kKV8 + lane * piece8, &tmap_v, 0, 0, 0, cur.h, blk, full8 + s8);
+        }
+        armed8 |= 1u << s8;
+        last8 = (last8 & ~(1u << s8)) | (((uint32_t)(lj / C::kNS8x) & 1u) << s8);
+        ++lj;
+        if (++lc >= cur.nchunks) {
+          lc = 0;
+          lhave = publish();
+        }
+      };
+      for (int k = 0; k < C::kNS8x - 1 && lhave && ok; ++k) issue_load();
+      int ci = 0, cc = 0;  // the widening cursor: item number in the ring, chunk within it
+      for (int j = 0; ok; ++j) {
+        const int nch = ring_items[ci % kRing].nchunks;  // published by the load cursor
+        if (nch == 0) break;                              // the work is gone
+        if (lhave) issue_load();  // chunk j + kNS8x - 1, into the stage chunk j - 1 left
+        if (!ok) break;
+        const int stage = j % C::kNSx;
+        if (lane == 0) {
+          ok = wait5(empty + stage, ((uint32_t)(j / C::kNSx) & 1u) ^ 1u, abort);
+          if (ok) ok = wait5(full8 + j % C::kNS8x, (uint32_t)(j / C::kNS8x) & 1u, abort);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        const uint8_t* st8 = ring8 + (j % C::kNS8x) * C::kStage8;
+        uint8_t* st = ring + stage * C::kStage;
+        // Lane = (row a of each RPI-row band, 16-byte group jj of codes): the
+        // group, its 16-bit piece and both swizzles are fixed per lane, so the
+        // unrolled loop is loads, widenings and stores.
+        constexpr int kGpr = D / 16, kRpi = 32 / kGpr;
+        const int jj = lane % kGpr, a = lane / kGpr;
+        const int pc = jj >> 2, g0 = 2 * (jj & 3);
+#pragma unroll
+        for (int tensor = 0; tensor < 2; ++tensor) {
+#pragma unroll
+          for (int i = 0; i < kChunk / kRpi; ++i) {
+            const int r = a + kRpi * i;
+            const int x8 = C::kRowB8 == 128 ? (r & 7) : ((r >> 1) & 3);
+            const uint4 v = *reinterpret_cast<const uint4*>(st8 + tensor * C::kKV8 +
+                                                            r * C::kRowB8 + ((jj ^ x8) << 4));
+            uint8_t* d = st + tensor * C::kKV + pc * C::kPlaneKV + r * 128;
+            *reinterpret_cast<uint4*>(d + ((g0 ^ (r & 7)) << 4)) =
+                make_uint4(e4m3x2_to_f16x2(v.x), e4m3x2_to_f16x2(v.x >> 16),
+                           e4m3x2_to_f16x2(v.y), e4m3x2_to_f16x2(v.y >> 16));
+            *reinterpret_cast<uint4*>(d + (((g0 + 1) ^ (r & 7)) << 4)) =
+                make_uint4(e4m3x2_to_f16x2(v.z), e4m3x2_to_f16x2(v.z >> 16),
+                           e4m3x2_to_f16x2(v.w), e4m3x2_to_f16x2(v.w >> 16));
+          }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // for the tensor cores
+        __syncwarp();
+        if (lane == 0) mbar_arrive(full + stage);
+        if (++cc >= nch) {
+          cc = 0;
+          ++ci;
+        }
+      }
+      if (!ok && lane == 0) {  // wait, bounded, for this CTA's copies in flight
+        for (int s8 = 0; s8 < C::kNS8x; ++s8) {
+          if (!(armed8 >> s8 & 1u)) continue;
+          const long long t0 = clock64();
+          while (!mbar_try(full8 + s8, (last8 >> s8) & 1u))
+            if (clock64() - t0 > kWaitCycles) break;
+        }
+      }
+    } else {
     bool have = publish();
     for (int j = 0, c = 0; have && ok; ++j) {
-      const int stage = j % kNS;
-      const uint32_t phase = (uint32_t)(j / kNS) & 1u;
+      const int stage = j % C::kNSx;
+      const uint32_t phase = (uint32_t)(j / C::kNSx) & 1u;
       const int c0 = c * kChunk;
       const int nblk = (min(kChunk, cur.kv_end - c0) + bs - 1) / bs;
       const int32_t* bt = p.block_table + (int64_t)cur.seq * p.max_blocks_per_seq;
@@ -486,13 +608,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (!ok && lane == 0) {  // wait, bounded, for this CTA's copies in flight
-      for (int s = 0; s < kNS; ++s) {
+      for (int s = 0; s < C::kNSx; ++s) {
         if (!(armed >> s & 1u)) continue;
         const long long t0 = clock64();
         while (!mbar_try(full + s, (last_parity >> s) & 1u))
           if (clock64() - t0 > kWaitCycles) break;
       }
     }
+    }  // 16-bit cache
   } else if (warp >= kMmaWarp) {
     // ----------------------------------------------------------------- MMA ----
     // Warp kMmaWarp + t serves tile t over the chunk sequence of all this
@@ -516,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Base descriptors once; the K steps add compile-time offsets to the
       // 14-bit address field (addresses stay below 256 KB, so it never carries).
       const uint64_t a0 = sdesc(q_addr + t * C::kQ, 16);
-      const uint64_t b0 = sdesc(r_addr + (j % kNS) * C::kStage, 16);
+      const uint64_t b0 = sdesc(r_addr + (j % C::kNSx) * C::kStage, 16);
       const uint32_t dS = tm + 128 * t + 64 * (j & 1);
 #pragma unroll
       for (int s = 0; s < D / 16; ++s) {
@@ -527,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(s_full + 2 * t + (j & 1));
     };
     auto issue_pv = [&](int j, bool acc) {  // O_t (+)= P_t(j) V(j)
-      const uint64_t b0 = sdesc(r_addr + (j % kNS) * C::kStage + C::kKV, C::kPlaneKV);
+      const uint64_t b0 = sdesc(r_addr + (j % C::kNSx) * C::kStage + C::kKV, C::kPlaneKV);
       const uint32_t dO = tm + C::kColO + t * D, aP = tm + 128 * t + 64 * (j & 1);
 #pragma unroll
       for (int s = 0; s < kChunk / 16; ++s)
@@ -550,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++q_items;
       }
       // K of chunk js (waited for only now, so the PV before never waits on a copy).
-      if (!wait_warp(full + js % kNS, (uint32_t)(js / kNS) & 1u)) return false;
+      if (!wait_warp(full + js % C::kNSx, (uint32_t)(js / C::kNSx) & 1u)) return false;
       tc_fence_after();
       if (leader) issue_s(js);
       __syncwarp();
@@ -566,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool last = pv.c == pv.nchunks - 1;
       if (leader) {
         issue_pv(j, pv.c > 0);
-        umma_commit(empty + j % kNS);
+        umma_commit(empty + j % C::kNSx);
         if (last) umma_commit(o_done + t);
       }
       __syncwarp();
@@ -596,11 +719,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = R < it.rows;
       const int tok = valid ? R / g : 0, jh = valid ? R - tok * g : 0;
       const uint4* src = reinterpret_cast<const uint4*>(
-          static_cast<const T*>(p.query) + ((int64_t)(it.q0 + tok) * Hq + it.h * g + jh) * D);
+          static_cast<const OT*>(p.query) + ((int64_t)(it.q0 + tok) * Hq + it.h * g + jh) * D);
+      if constexpr (F8 && !std::is_same<OT, __half>::value) {
+        // The f16 MMAs of an E4M3 cache: Q rounded to f16 on its way in.
+        uint4 v[D / 8];
 #pragma unroll
-      for (int u = 0; u < D / 8; ++u)
-        cp_async16(qt + (u >> 3) * C::kPlaneQ + sw(r, u & 7), valid ? src + u : p.query, valid);
-      asm volatile("cp.async.commit_group;" ::: "memory");
+        for (int u = 0; u < D / 8; ++u) v[u] = valid ? __ldg(src + u) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int u = 0; u < D / 8; ++u) {
+          uint4 h;
+          h.x = to_f16x2<OT>(v[u].x);
+          h.y = to_f16x2<OT>(v[u].y);
+          h.z = to_f16x2<OT>(v[u].z);
+          h.w = to_f16x2<OT>(v[u].w);
+          *reinterpret_cast<uint4*>(qs + t * C::kQ + (u >> 3) * C::kPlaneQ + sw(r, u & 7)) = h;
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < D / 8; ++u)
+          cp_async16(qt + (u >> 3) * C::kPlaneQ + sw(r, u & 7), valid ? src + u : p.query, valid);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+      }
     };
     auto q_ready = [&]() {
       asm volatile("cp.async.wait_all;" ::: "memory");
@@ -618,7 +757,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int pc = 0; pc < C::kPlanes; ++pc)
         tma_load_q(qs + t * C::kQ + pc * C::kPlaneQ, &tmap_q, pc * 64, it.h * g, z, q_full + t);
     };
-    const float sscale = p.score_scale;
+    // E4M3: K = code * k_scale folds into the score scale, V = code * v_scale
+    // into the output.
+    const float sscale = p.score_scale * (F8 ? __ldg(p.k_scale) : 1.f);
+    const float vsc = F8 ? __ldg(p.v_scale) : 1.f;
     Walk w;
     w.start(ring_items, item_full, abort);
     if (w.ok) {
@@ -638,7 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // cannot start before O has been read.
     bool pending = false, prev_valid = false;
     uint64_t prev_lsum = 0;
-    T* prev_dst = nullptr;
+    OT* prev_dst = nullptr;
     auto epilogue = [&]() -> bool {
       pending = false;
       bool okk = wait5(o_done + t, (uint32_t)items & 1u, abort);  // every PV of the item
@@ -649,7 +791,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float l0, l1;
       asm("mov.b64 {%0, %1}, %2;" : "=f"(l0), "=f"(l1) : "l"(prev_lsum));
       const float lsum = l0 + l1;
-      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+      const float inv = lsum > 0.f ? vsc / lsum : 0.f;
 #pragma unroll
       for (int q = 0; q < D / 64; ++q) {
         float o[64];
@@ -659,10 +801,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int u = 0; u < 8; ++u) {
             uint4 wv;
             float a, b;
-            wv.x = Mma<T>::pack(o[8 * u + 0] * inv, o[8 * u + 1] * inv, a, b);
-            wv.y = Mma<T>::pack(o[8 * u + 2] * inv, o[8 * u + 3] * inv, a, b);
-            wv.z = Mma<T>::pack(o[8 * u + 4] * inv, o[8 * u + 5] * inv, a, b);
-            wv.w = Mma<T>::pack(o[8 * u + 6] * inv, o[8 * u + 7] * inv, a, b);
+            wv.x = Mma<OT>::pack(o[8 * u + 0] * inv, o[8 * u + 1] * inv, a, b);
+            wv.y = Mma<OT>::pack(o[8 * u + 2] * inv, o[8 * u + 3] * inv, a, b);
+            wv.z = Mma<OT>::pack(o[8 * u + 4] * inv, o[8 * u + 5] * inv, a, b);
+            wv.w = Mma<OT>::pack(o[8 * u + 6] * inv, o[8 * u + 7] * inv, a, b);
             *reinterpret_cast<uint4*>(prev_dst + 64 * q + 8 * u) = wv;
           }
         }
@@ -675,8 +817,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = R < w.it().rows;
       const int tok = valid ? R / g : 0, jh = valid ? R - tok * g : 0;
       const int pos = valid ? w.it().base_pos + tok : -1;
-      T* const dst =
-          static_cast<T*>(p.out) + ((int64_t)(w.it().q0 + tok) * Hq + w.it().h * g + jh) * D;
+      OT* const dst =
+          static_cast<OT*>(p.out) + ((int64_t)(w.it().q0 + tok) * Hq + w.it().h * g + jh) * D;
       __syncwarp();  // every lane has read the record
       if (lane == 0) mbar_arrive(item_empty + w.ii % kRing);
       float m_use = -INFINITY;
@@ -773,7 +915,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // Zero V rows past the range (stale or poisoned) before this tile's
           // last PV. Both tiles do it, as their PVs are issued independently
           // (the other tile's stores write the same zeros).
-          uint8_t* v = ring + (j % kNS) * C::kStage + C::kKV;
+          uint8_t* v = ring + (j % C::kNSx) * C::kStage + C::kKV;
           const int t0 = kv_end - c0, per_row = 8 * C::kPlanes;
           for (int e = r; e < (kChunk - t0) * per_row; e += kRows) {
             const int tk = t0 + e / per_row, u = e % per_row;
@@ -845,11 +987,11 @@ cudaError_t next_sched_slot(int dev, int** sched) {
   return cudaSuccess;
 }
 
-template <typename T, int D, bool QT>
+template <typename OT, int D, bool QT, bool F8>
 cudaError_t launch5(const PrefillParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
                     const CUtensorMap& mq, int num_seqs, cudaStream_t stream) {
-  using C = Cfg5<D>;
-  auto kernel = prefill_tc5_kernel<T, D, QT>;
+  using C = Cfg5<D, F8>;
+  auto kernel = prefill_tc5_kernel<OT, D, QT, F8>;
   static std::atomic<int> opted_in[64];  // the shared-memory opt-in, once per device
   static std::atomic<int> sm_count[64];
   int dev = 0;
@@ -869,9 +1011,6 @@ cudaError_t launch5(const PrefillParams& p, const CUtensorMap& mk, const CUtenso
   const int64_t n_items = tiles * num_seqs * p.num_kv_heads;
   if (n_items <= 0) return cudaSuccess;
   if (n_items > (int64_t)INT32_MAX / 2) return cudaErrorInvalidValue;
-  // Persistent: one CTA per SM (a CTA fills one), each walking items
-  // blockIdx.x, + gridDim.x, ... so that the next item's Q and K/V stream in
-  // while the current one finishes.
   // Persistent: one CTA per SM (a CTA fills one), each taking the launch's
   // items from a work counter as it becomes free.
   int* sched = nullptr;
@@ -901,13 +1040,15 @@ bool encode_q_map(CUtensorMap* map, const PrefillParams& p, int head_dim, bool b
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename T, int D>
+template <typename OT, int D>
 cudaError_t launch5q(const PrefillParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
-                     int num_seqs, cudaStream_t stream) {
+                     bool f8, int num_seqs, cudaStream_t stream) {
+  if (f8)  // Q rounded to f16 by the softmax threads
+    return launch5<OT, D, false, true>(p, mk, mv, mk, num_seqs, stream);  // mk unused as Q map
   CUtensorMap mq;
-  if (encode_q_map(&mq, p, D, std::is_same<T, __nv_bfloat16>::value))
-    return launch5<T, D, true>(p, mk, mv, mq, num_seqs, stream);
-  return launch5<T, D, false>(p, mk, mv, mk, num_seqs, stream);  // mk unused as Q map
+  if (encode_q_map(&mq, p, D, std::is_same<OT, __nv_bfloat16>::value))
+    return launch5<OT, D, true, false>(p, mk, mv, mq, num_seqs, stream);
+  return launch5<OT, D, false, false>(p, mk, mv, mk, num_seqs, stream);  // mk unused as Q map
 }
 
 }  // namespace
@@ -915,12 +1056,13 @@ cudaError_t launch5q(const PrefillParams& p, const CUtensorMap& mk, const CUtens
 bool prefill_tc5_supported(int head_dim) { return head_dim == 64 || head_dim == 128; }
 
 cudaError_t launch_prefill_tc5(const PrefillParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
-                               int head_dim, bool bf16, int num_seqs, cudaStream_t stream) {
+                               int head_dim, bool bf16, bool f8, int num_seqs,
+                               cudaStream_t stream) {
   if (bf16)
-    return head_dim == 128 ? launch5q<__nv_bfloat16, 128>(p, mk, mv, num_seqs, stream)
-                           : launch5q<__nv_bfloat16, 64>(p, mk, mv, num_seqs, stream);
-  return head_dim == 128 ? launch5q<__half, 128>(p, mk, mv, num_seqs, stream)
-                         : launch5q<__half, 64>(p, mk, mv, num_seqs, stream);
+    return head_dim == 128 ? launch5q<__nv_bfloat16, 128>(p, mk, mv, f8, num_seqs, stream)
+                           : launch5q<__nv_bfloat16, 64>(p, mk, mv, f8, num_seqs, stream);
+  return head_dim == 128 ? launch5q<__half, 128>(p, mk, mv, f8, num_seqs, stream)
+                         : launch5q<__half, 64>(p, mk, mv, f8, num_seqs, stream);
 }
 
 }  // namespace pf
