@@ -34,10 +34,12 @@
 //    loaded by one softmax thread as soon as the tile's last S of the previous
 //    item has completed; otherwise the softmax threads copy their rows.
 //  * An E4M3 cache: the producer copies a chunk's codes by TMA into a staging
-//    ring (up to three chunks ahead) and widens them, exactly, to f16 in the
-//    chunk's stage, in the layout the 16-bit path gets from TMA; the MMAs are
-//    f16 (Q rounded to f16 by the softmax threads as they stage it), k_scale
-//    is folded into the score scale and v_scale into the output.
+//    ring (up to three chunks ahead); the producer widens K and a twelfth warp
+//    widens V, exactly, to f16 in the chunk's stage, in the layout the 16-bit
+//    path gets from TMA (the widening is bound by the issue rate of the warps
+//    doing it, so it is split over two sub-partitions); the MMAs are f16 (Q
+//    rounded to f16 by the softmax threads as they stage it), k_scale is folded
+//    into the score scale and v_scale into the output.
 //  * Each tile has two S buffers in tensor memory (chunk j uses buffer j % 2):
 //    S = Q K^T of the next chunk (M 128, N 64, K 16 per instruction) is
 //    computed into one while the softmax threads work on the other, so a
@@ -96,6 +98,11 @@ constexpr int kSoftWarps = 4 * kTiles;
 constexpr int kProducerWarp = kSoftWarps;
 constexpr int kMmaWarp = kSoftWarps + 1;  // MMA warps kMmaWarp + t, one per tile
 constexpr int kThreads = (kSoftWarps + 1 + kTiles) * 32;
+// E4M3 caches: a twelfth warp widens each chunk's V while the producer widens
+// its K (on the fourth sub-partition, so it costs no registers: three warps
+// per sub-partition either way).
+constexpr int kWidenWarp = kSoftWarps + 1 + kTiles;
+constexpr int kThreads8 = kThreads + 32;
 constexpr int kNS = 4;          // K/V stages
 constexpr uint32_t kTmemCols = 512;
 
@@ -157,7 +164,7 @@ struct Cfg5 {
   static constexpr int kKV8 = kChunk * D;
   static constexpr int kStage8 = F8 ? 2 * kKV8 : 0;
   static constexpr int kSmem = 1024 + kNSx * kStage + kNS8x * kStage8 + kTiles * kQ + kBars * 8 +
-                               kNS8x * 8 + 16 + kRing * (16 + (int)sizeof(Item));
+                               2 * kNS8x * 8 + 16 + kRing * (16 + (int)sizeof(Item));
   static_assert(kSmem <= 227 * 1024, "shared memory per CTA exceeds 227 KB");
 };
 
@@ -372,7 +379,7 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
 // OT: query/output type. F8: the cache holds E4M3 codes, widened to f16 in
 // shared memory by the producer; Q is rounded to f16 (the MMAs are f16).
 template <typename OT, int D, bool QT, bool F8>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(F8 ? kThreads8 : kThreads, 1)
     prefill_tc5_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_v,
                        const __grid_constant__ CUtensorMap tmap_q, int num_seqs, int tiles,
@@ -392,8 +399,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* q_full = p_full + 2 * kTiles;  // [tile] Q of the tile's next item is staged
   uint64_t* o_done = q_full + kTiles;      // [tile] every PV of the tile's item has completed
   uint64_t* drain = o_done + kTiles;       // every MMA issued has completed
-  uint64_t* full8 = drain + 1;               // F8: [C::kNS8x] E4M3 codes of a chunk have landed
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(full8 + C::kNS8x);
+  uint64_t* full8 = drain + 1;               // F8: [kNS8x] E4M3 codes of a chunk have landed
+  uint64_t* free8 = full8 + C::kNS8x;        // F8: [kNS8x] both halves of its chunk are widened
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(free8 + C::kNS8x);
   volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
   uint64_t* item_full = reinterpret_cast<uint64_t*>(tslot + 2);  // [kRing] a record is published
   uint64_t* item_empty = item_full + kRing;  // [kRing] every role is done with a record
@@ -404,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kNSx; ++s) {
-      mbar_init(full + s, 1);
+      mbar_init(full + s, F8 ? 2 : 1);  // F8: the producer (K) and the widening warp (V)
       mbar_init(empty + s, kTiles);  // one commit per tile's MMA warp
     }
     for (int t = 0; t < kTiles; ++t) {
@@ -417,7 +425,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(drain, kTiles);
     if (F8)
-      for (int s = 0; s < C::kNS8x; ++s) mbar_init(full8 + s, 1);
+      for (int s = 0; s < C::kNS8x; ++s) {
+        mbar_init(full8 + s, 1);
+        mbar_init(free8 + s, 2);
+      }
     for (int s = 0; s < kRing; ++s) {
       mbar_init(item_full + s, 1);
       mbar_init(item_empty + s, kTiles + kSoftWarps);  // the MMA warps and the softmax warps
@@ -436,6 +447,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+
+  // F8: one tensor (0 = K, 1 = V) of a chunk's codes widened, exactly, to f16
+  // in the chunk's 16-bit stage. Lane = (row a of each kRpi-row band, 16-byte
+  // group jj of codes): the group, its 16-bit piece and both swizzles are fixed
+  // per lane, so the unrolled loop is loads, widenings and stores.
+  auto widen_half = [&](const uint8_t* st8, uint8_t* st, int tensor) {
+    constexpr int kGpr = D / 16, kRpi = 32 / kGpr;
+    const int jj = lane % kGpr, a = lane / kGpr;
+    const int pc = jj >> 2, g0 = 2 * (jj & 3);
+#pragma unroll
+    for (int i = 0; i < kChunk / kRpi; ++i) {
+      const int r = a + kRpi * i;
+      const int x8 = C::kRowB8 == 128 ? (r & 7) : ((r >> 1) & 3);
+      const uint4 v = *reinterpret_cast<const uint4*>(st8 + tensor * C::kKV8 + r * C::kRowB8 +
+                                                      ((jj ^ x8) << 4));
+      uint8_t* d = st + tensor * C::kKV + pc * C::kPlaneKV + r * 128;
+      *reinterpret_cast<uint4*>(d + ((g0 ^ (r & 7)) << 4)) =
+          make_uint4(e4m3x2_to_f16x2(v.x), e4m3x2_to_f16x2(v.x >> 16),
+                     e4m3x2_to_f16x2(v.y), e4m3x2_to_f16x2(v.y >> 16));
+      *reinterpret_cast<uint4*>(d + (((g0 + 1) ^ (r & 7)) << 4)) =
+          make_uint4(e4m3x2_to_f16x2(v.z), e4m3x2_to_f16x2(v.z >> 16),
+                     e4m3x2_to_f16x2(v.w), e4m3x2_to_f16x2(v.w >> 16));
+    }
+  };
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer ----
@@ -500,6 +535,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool lhave = publish();
       auto issue_load = [&]() {
         const int s8 = lj % C::kNS8x;
+        // Both halves of the slot's previous chunk have been widened.
+        if (lane == 0) ok = wait5(free8 + s8, ((uint32_t)(lj / C::kNS8x) & 1u) ^ 1u, abort);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) return;
         const int c0 = lc * kChunk;
         const int nblk = (min(kChunk, cur.kv_end - c0) + bs - 1) / bs;
         const int32_t* bt = p.block_table + (int64_t)cur.seq * p.max_blocks_per_seq;
@@ -536,32 +575,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         const uint8_t* st8 = ring8 + (j % C::kNS8x) * C::kStage8;
         uint8_t* st = ring + stage * C::kStage;
-        // Lane = (row a of each RPI-row band, 16-byte group jj of codes): the
-        // group, its 16-bit piece and both swizzles are fixed per lane, so the
-        // unrolled loop is loads, widenings and stores.
-        constexpr int kGpr = D / 16, kRpi = 32 / kGpr;
-        const int jj = lane % kGpr, a = lane / kGpr;
-        const int pc = jj >> 2, g0 = 2 * (jj & 3);
-#pragma unroll
-        for (int tensor = 0; tensor < 2; ++tensor) {
-#pragma unroll
-          for (int i = 0; i < kChunk / kRpi; ++i) {
-            const int r = a + kRpi * i;
-            const int x8 = C::kRowB8 == 128 ? (r & 7) : ((r >> 1) & 3);
-            const uint4 v = *reinterpret_cast<const uint4*>(st8 + tensor * C::kKV8 +
-                                                            r * C::kRowB8 + ((jj ^ x8) << 4));
-            uint8_t* d = st + tensor * C::kKV + pc * C::kPlaneKV + r * 128;
-            *reinterpret_cast<uint4*>(d + ((g0 ^ (r & 7)) << 4)) =
-                make_uint4(e4m3x2_to_f16x2(v.x), e4m3x2_to_f16x2(v.x >> 16),
-                           e4m3x2_to_f16x2(v.y), e4m3x2_to_f16x2(v.y >> 16));
-            *reinterpret_cast<uint4*>(d + (((g0 + 1) ^ (r & 7)) << 4)) =
-                make_uint4(e4m3x2_to_f16x2(v.z), e4m3x2_to_f16x2(v.z >> 16),
-                           e4m3x2_to_f16x2(v.w), e4m3x2_to_f16x2(v.w >> 16));
-          }
-        }
+        widen_half(st8, st, 0);  // K (the widening warp does V)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // for the tensor cores
         __syncwarp();
-        if (lane == 0) mbar_arrive(full + stage);
+        if (lane == 0) {
+          mbar_arrive(full + stage);
+          mbar_arrive(free8 + j % C::kNS8x);
+        }
         if (++cc >= nch) {
           cc = 0;
           ++ci;
@@ -616,7 +636,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     }  // 16-bit cache
-  } else if (warp >= kMmaWarp) {
+  } else if (warp == kWidenWarp) {  // only launched with an E4M3 cache
+    // ------------------------------------------------------ V widening (F8) ----
+    if constexpr (F8) {
+    Walk w;
+    w.start(ring_items, item_full, abort);
+    bool ok = true;
+    for (int j = 0; w.ok && ok; ++j) {
+      const int stage = j % C::kNSx;
+      if (lane == 0) {
+        ok = wait5(empty + stage, ((uint32_t)(j / C::kNSx) & 1u) ^ 1u, abort);
+        if (ok) ok = wait5(full8 + j % C::kNS8x, (uint32_t)(j / C::kNS8x) & 1u, abort);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      widen_half(ring8 + (j % C::kNS8x) * C::kStage8, ring + stage * C::kStage, 1);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // for the tensor cores
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(full + stage);
+        mbar_arrive(free8 + j % C::kNS8x);
+      }
+      w.advance();
+    }
+    }
+  } else if (warp >= kMmaWarp && warp < kMmaWarp + kTiles) {
     // ----------------------------------------------------------------- MMA ----
     // Warp kMmaWarp + t serves tile t over the chunk sequence of all this
     // CTA's items: S of chunks 0 and 1 up front (one S buffer each), then per
@@ -1017,7 +1061,7 @@ cudaError_t launch5(const PrefillParams& p, const CUtensorMap& mk, const CUtenso
   const cudaError_t es = next_sched_slot(dev, &sched);
   if (es != cudaSuccess) return es;
   const int64_t grid = std::min<int64_t>(n_items, sm_count[dev].load(std::memory_order_relaxed));
-  kernel<<<(unsigned)grid, kThreads, C::kSmem, stream>>>(p, mk, mv, mq, num_seqs, (int)tiles,
+  kernel<<<(unsigned)grid, F8 ? kThreads8 : kThreads, C::kSmem, stream>>>(p, mk, mv, mq, num_seqs, (int)tiles,
                                                          (int)n_items, sched);
   return cudaGetLastError();
 }
