@@ -173,6 +173,13 @@ __device__ __forceinline__ bool wait5(uint64_t* bar, uint32_t parity, volatile i
   return mbar_wait_or_abort(bar, parity, abort, &g_pf5_status);
 }
 
+// Four E4M3 codes (one 32-bit word) widened exactly to two f16 pairs; the
+// halves of the word are taken as 16-bit registers, so no shift is needed.
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n .reg .b16 a, b;\n mov.b32 {a, b}, %2;\n cvt.rn.f16x2.e4m3x2 %0, a;\n"
+      " cvt.rn.f16x2.e4m3x2 %1, b;\n}" : "=r"(lo), "=r"(hi) : "r"(w));
+}
+
 // Shared-memory matrix descriptor: 128B swizzle, 8-row groups 1024 bytes apart,
 // `lbo` between 64-element pieces (MN-major operands).
 __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo) {
@@ -452,24 +459,34 @@ __global__ void __launch_bounds__(F8 ? kThreads8 : kThreads, 1)
   // F8: one tensor (0 = K, 1 = V) of a chunk's codes widened, exactly, to f16
   // in the chunk's 16-bit stage. Lane = (row a of each kRpi-row band, 16-byte
   // group jj of codes): the group, its 16-bit piece and both swizzles are fixed
-  // per lane, so the unrolled loop is loads, widenings and stores.
+  // per lane. All of the lane's codes are loaded before the first store: the
+  // stores may alias the loads as far as the compiler knows, so loads left
+  // between them would each wait out a shared-memory round trip (measured 2x
+  // slower in isolation).
   auto widen_half = [&](const uint8_t* st8, uint8_t* st, int tensor) {
     constexpr int kGpr = D / 16, kRpi = 32 / kGpr;
     const int jj = lane % kGpr, a = lane / kGpr;
     const int pc = jj >> 2, g0 = 2 * (jj & 3);
+    constexpr int kN = kChunk / kRpi;
+    uint4 v[kN];
 #pragma unroll
-    for (int i = 0; i < kChunk / kRpi; ++i) {
+    for (int i = 0; i < kN; ++i) {
       const int r = a + kRpi * i;
       const int x8 = C::kRowB8 == 128 ? (r & 7) : ((r >> 1) & 3);
-      const uint4 v = *reinterpret_cast<const uint4*>(st8 + tensor * C::kKV8 + r * C::kRowB8 +
-                                                      ((jj ^ x8) << 4));
+      v[i] = *reinterpret_cast<const uint4*>(st8 + tensor * C::kKV8 + r * C::kRowB8 +
+                                             ((jj ^ x8) << 4));
+    }
+#pragma unroll
+    for (int i = 0; i < kN; ++i) {
+      const int r = a + kRpi * i;
       uint8_t* d = st + tensor * C::kKV + pc * C::kPlaneKV + r * 128;
-      *reinterpret_cast<uint4*>(d + ((g0 ^ (r & 7)) << 4)) =
-          make_uint4(e4m3x2_to_f16x2(v.x), e4m3x2_to_f16x2(v.x >> 16),
-                     e4m3x2_to_f16x2(v.y), e4m3x2_to_f16x2(v.y >> 16));
-      *reinterpret_cast<uint4*>(d + (((g0 + 1) ^ (r & 7)) << 4)) =
-          make_uint4(e4m3x2_to_f16x2(v.z), e4m3x2_to_f16x2(v.z >> 16),
-                     e4m3x2_to_f16x2(v.w), e4m3x2_to_f16x2(v.w >> 16));
+      uint4 o0, o1;
+      e4m3x4_to_f16x4(v[i].x, o0.x, o0.y);
+      e4m3x4_to_f16x4(v[i].y, o0.z, o0.w);
+      e4m3x4_to_f16x4(v[i].z, o1.x, o1.y);
+      e4m3x4_to_f16x4(v[i].w, o1.z, o1.w);
+      *reinterpret_cast<uint4*>(d + ((g0 ^ (r & 7)) << 4)) = o0;
+      *reinterpret_cast<uint4*>(d + (((g0 + 1) ^ (r & 7)) << 4)) = o1;
     }
   };
 
@@ -948,8 +965,18 @@ __global__ void __launch_bounds__(F8 ? kThreads8 : kThreads, 1)
             asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rr) : "l"(xy), "l"(sc), "l"(mm));
             asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(rr));
           }
-          float lo, hi;  // the row sums take P as the tensor cores see it (rounded)
-          pk[i] = Mma<T>::pack(fast_exp2(x0), fast_exp2(x1), lo, hi);
+          float lo, hi;  // the row sums take P as the tensor cores see it (bf16: rounded)
+          if constexpr (F8) {
+            // f16 P is within 2^-11 (relative) of the fp32 value, and reading
+            // it back would cost two conversions per pair: the row sums take
+            // the fp32 values.
+            lo = fast_exp2(x0);
+            hi = fast_exp2(x1);
+            const __half2 hv = __floats2half2_rn(lo, hi);
+            pk[i] = *reinterpret_cast<const uint32_t*>(&hv);
+          } else {
+            pk[i] = Mma<T>::pack(fast_exp2(x0), fast_exp2(x1), lo, hi);
+          }
           {
             uint64_t pp;
             asm("mov.b64 %0, {%1, %2};" : "=l"(pp) : "f"(lo), "f"(hi));
