@@ -420,7 +420,8 @@ __global__ void __launch_bounds__(F8 ? kThreads8 : kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kNSx; ++s) {
-      mbar_init(full + s, F8 ? 2 : 1);  // F8: the producer (K) and the widening warp (V)
+      // F8: every lane of the producer (K) and of the widening warp (V)
+      mbar_init(full + s, F8 ? 64 : 1);
       mbar_init(empty + s, kTiles);  // one commit per tile's MMA warp
     }
     for (int t = 0; t < kTiles; ++t) {
@@ -435,7 +436,7 @@ __global__ void __launch_bounds__(F8 ? kThreads8 : kThreads, 1)
     if (F8)
       for (int s = 0; s < C::kNS8x; ++s) {
         mbar_init(full8 + s, 1);
-        mbar_init(free8 + s, 2);
+        mbar_init(free8 + s, 64);  // every lane of both widening warps
       }
     for (int s = 0; s < kRing; ++s) {
       mbar_init(item_full + s, 1);
@@ -554,9 +555,11 @@ __global__ void __launch_bounds__(F8 ? kThreads8 : kThreads, 1)
       auto issue_load = [&]() {
         const int s8 = lj % C::kNS8x;
         // Both halves of the slot's previous chunk have been widened.
-        if (lane == 0) ok = wait5(free8 + s8, ((uint32_t)(lj / C::kNS8x) & 1u) ^ 1u, abort);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) return;
+        ok = wait5(free8 + s8, ((uint32_t)(lj / C::kNS8x) & 1u) ^ 1u, abort);
+        if (__any_sync(0xffffffffu, !ok)) {
+          ok = false;
+          return;
+        }
         const int c0 = lc * kChunk;
         const int nblk = (min(kChunk, cur.kv_end - c0) + bs - 1) / bs;
         const int32_t* bt = p.block_table + (int64_t)cur.seq * p.max_blocks_per_seq;
@@ -585,21 +588,21 @@ __global__ void __launch_bounds__(F8 ? kThreads8 : kThreads, 1)
         if (lhave) issue_load();  // chunk j + kNS8x - 1, into the slot chunk j - 1 left
         if (!ok) break;
         const int stage = j % C::kNSx;
-        if (lane == 0) {
-          ok = wait5(empty + stage, ((uint32_t)(j / C::kNSx) & 1u) ^ 1u, abort);
-          if (ok) ok = wait5(full8 + j % C::kNS8x, (uint32_t)(j / C::kNS8x) & 1u, abort);
+        // Every lane waits, widens, fences its own stores and arrives: with a
+        // wait in one lane and a warp sync before the arrival, the warp ran
+        // the widening as two groups of lanes, one after the other (measured).
+        ok = wait5(empty + stage, ((uint32_t)(j / C::kNSx) & 1u) ^ 1u, abort);
+        if (ok) ok = wait5(full8 + j % C::kNS8x, (uint32_t)(j / C::kNS8x) & 1u, abort);
+        if (__any_sync(0xffffffffu, !ok)) {
+          ok = false;
+          break;
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
         const uint8_t* st8 = ring8 + (j % C::kNS8x) * C::kStage8;
         uint8_t* st = ring + stage * C::kStage;
         widen_half(st8, st, 0);  // K (the widening warp does V)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // for the tensor cores
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(full + stage);
-          mbar_arrive(free8 + j % C::kNS8x);
-        }
+        mbar_arrive(full + stage);
+        mbar_arrive(free8 + j % C::kNS8x);
         if (++cc >= nch) {
           cc = 0;
           ++ci;
@@ -662,19 +665,17 @@ __global__ void __launch_bounds__(F8 ? kThreads8 : kThreads, 1)
     bool ok = true;
     for (int j = 0; w.ok && ok; ++j) {
       const int stage = j % C::kNSx;
-      if (lane == 0) {
-        ok = wait5(empty + stage, ((uint32_t)(j / C::kNSx) & 1u) ^ 1u, abort);
-        if (ok) ok = wait5(full8 + j % C::kNS8x, (uint32_t)(j / C::kNS8x) & 1u, abort);
+      // As in the producer, every lane waits, widens and arrives.
+      ok = wait5(empty + stage, ((uint32_t)(j / C::kNSx) & 1u) ^ 1u, abort);
+      if (ok) ok = wait5(full8 + j % C::kNS8x, (uint32_t)(j / C::kNS8x) & 1u, abort);
+      if (__any_sync(0xffffffffu, !ok)) {
+        ok = false;
+        break;
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
       widen_half(ring8 + (j % C::kNS8x) * C::kStage8, ring + stage * C::kStage, 1);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // for the tensor cores
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(full + stage);
-        mbar_arrive(free8 + j % C::kNS8x);
-      }
+      mbar_arrive(full + stage);
+      mbar_arrive(free8 + j % C::kNS8x);
       w.advance();
     }
     }
