@@ -315,13 +315,14 @@ def _cudart():
     return _CUDART
 
 
-def e2e_time_ms(args, wl, append, decode, out, world):
+def e2e_time_ms(args, wl, c_calls, out, world):
     """Per-step time of the step through the public API with host buffers.
 
     Every step copies its inputs (query, new K/V, slot mapping, block table,
-    lengths), packed in one pinned host buffer, to the device in one copy, runs
-    paged_kv_append and paged_attention_decode through the binding, and copies
-    the output back to pinned host memory. Inputs and outputs are double
+    lengths), packed in one pinned host buffer, to the device in one copy, calls
+    paged_kv_append and paged_attention_decode through the C ABI (their
+    arguments marshalled once per buffer by `c_calls`), and copies the output
+    back to pinned host memory. Inputs and outputs are double
     buffered and the copies run on their own streams, so step k+1's inputs and
     step k-1's output move while step k computes; the timed region spans the
     first input copy to the last output copy. The copies and the events that
@@ -353,10 +354,9 @@ def e2e_time_ms(args, wl, append, decode, out, world):
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     cs, si, so = compute.cuda_stream, s_in.cuda_stream, s_out.cuda_stream
     ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_used = [torch.cuda.Event() for _ in range(2)]     # step done with its inputs
-    ev_out = [torch.cuda.Event() for _ in range(2)]      # output ready
+    ev_done = [torch.cuda.Event() for _ in range(2)]     # step done: inputs free, output ready
     ev_read = [torch.cuda.Event() for _ in range(2)]     # output copied to the host
-    for evs in (ev_in, ev_used, ev_out, ev_read):        # create the events
+    for evs in (ev_in, ev_done, ev_read):                # create the events
         for e in evs:
             e.record(compute)
     torch.cuda.synchronize()
@@ -365,25 +365,29 @@ def e2e_time_ms(args, wl, append, decode, out, world):
     hout = [h.data_ptr() for h in h_out]
     dout = [o.data_ptr() for o in outs]
     H2D, D2H = 1, 2
+    calls = [c_calls(*views[b], outs[b], cs) for b in range(2)]
+    evi = [e.cuda_event for e in ev_in]
+    evd = [e.cuda_event for e in ev_done]
+    evr = [e.cuda_event for e in ev_read]
 
     def run(steps):
         for k in range(steps):
             b = k & 1
             if k >= 2:
-                cr.cudaStreamWaitEvent(si, ev_used[b].cuda_event, 0)
+                cr.cudaStreamWaitEvent(si, evd[b], 0)
             cr.cudaMemcpyAsync(din[b], hin[b], h2d, H2D, si)
-            cr.cudaEventRecord(ev_in[b].cuda_event, si)
-            cr.cudaStreamWaitEvent(cs, ev_in[b].cuda_event, 0)
+            cr.cudaEventRecord(evi[b], si)
+            cr.cudaStreamWaitEvent(cs, evi[b], 0)
             if k >= 2:
-                cr.cudaStreamWaitEvent(cs, ev_read[b].cuda_event, 0)
-            q, nk, nv, sl, bt, ln = views[b]
-            append(nk, nv, sl)
-            decode(q, bt, ln, outs[b])
-            cr.cudaEventRecord(ev_used[b].cuda_event, cs)
-            cr.cudaEventRecord(ev_out[b].cuda_event, cs)
-            cr.cudaStreamWaitEvent(so, ev_out[b].cuda_event, 0)
+                cr.cudaStreamWaitEvent(cs, evr[b], 0)
+            for fn, a in calls[b]:
+                st = fn(*a)
+                if st != 0:
+                    raise pkv.PagedKVError(fn.__name__, st)
+            cr.cudaEventRecord(evd[b], cs)
+            cr.cudaStreamWaitEvent(so, evd[b], 0)
             cr.cudaMemcpyAsync(hout[b], dout[b], d2h, D2H, so)
-            cr.cudaEventRecord(ev_read[b].cuda_event, so)
+            cr.cudaEventRecord(evr[b], so)
 
     run(4)
     torch.cuda.synchronize()
@@ -486,7 +490,25 @@ def run_ours(args, rank, world, dev):
     status = pkv.pkv_device_status(clear=True)
     assert status == 0, f"device wait expired (status {status})"
 
-    e2e_ms, KE, h2d, d2h, h_out = e2e_time_ms(args, wl, append, decode, out, world)
+    lib = pkv.load_library()
+    e2e_flags = args.flags | serving
+
+    def c_calls(q, nk, nv, sl, bt_t, ln, out_t, stream):
+        """The step's two C-ABI calls on these buffers, each argument converted
+        to its C type once."""
+        def prebuilt(fn, a):
+            return fn, tuple(t(x) for t, x in zip(fn.argtypes, a))
+        return (prebuilt(lib.paged_kv_append,
+                         pkv.append_args(nk, nv, wl.k_cache, wl.v_cache, sl, k_scale=ks,
+                                         v_scale=vs, stream=stream)),
+                prebuilt(lib.paged_attention_decode,
+                         pkv.decode_args(out_t, q, wl.k_cache, wl.v_cache, bt_t, ln,
+                                         max_seq_len=msl, scale=c.scale, partition_size=P,
+                                         workspace=ws, k_scale=ks, v_scale=vs,
+                                         max_ctas=args.max_ctas, flags=e2e_flags,
+                                         stream=stream)))
+
+    e2e_ms, KE, h2d, d2h, h_out = e2e_time_ms(args, wl, c_calls, out, world)
     assert torch.isfinite(h_out.float()).all(), "non-finite decode output"
 
     if world > 1:
@@ -518,7 +540,8 @@ def run_ours(args, rank, world, dev):
                 "d2h_bytes_per_step": d2h,
                 "how": "each step: one H2D copy of the step's packed inputs (query, new K/V, "
                        "slot mapping, block table, lengths) from pinned host memory, "
-                       "paged_kv_append and paged_attention_decode through the Python binding, "
+                       "paged_kv_append and paged_attention_decode through the C ABI "
+                       "(arguments marshalled once per double buffer), "
                        "one D2H copy of the output to pinned host memory; copies run on two "
                        "copy streams, double-buffered, so step k+1's inputs and step k-1's "
                        "output move while step k computes; copies and events issued through "

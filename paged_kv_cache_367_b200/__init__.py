@@ -16,7 +16,7 @@ import torch
 
 __all__ = ["paged_kv_append", "paged_attention_decode", "paged_attention_workspace_size",
            "paged_attention_decode_static", "paged_kv_copy_blocks", "paged_kv_swap_blocks",
-           "paged_attention_prefill",
+           "paged_attention_prefill", "append_args", "decode_args",
            "pkv_device_status", "pkv_selftest_expired_wait", "pkv_status_string", "pkv_version",
            "load_library", "PagedKVError",
            "PKV_F32", "PKV_F16", "PKV_BF16", "PKV_FP8_E4M3", "PKV_DECODE_FORCE_SIMT",
@@ -178,16 +178,25 @@ def _stream(stream):
     return stream.cuda_stream
 
 
+def append_args(key, value, k_cache, v_cache, slot_mapping, *, k_scale=None, v_scale=None,
+                stream=None) -> tuple:
+    """The arguments of the C call paged_kv_append for these tensors (pointers,
+    sizes, dtype codes, stream), in its order: a caller that repeats the call on
+    the same buffers can marshal them once."""
+    T, Hkv, D = key.shape
+    nb, bs = k_cache.shape[0], k_cache.shape[1]
+    return (_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), T, Hkv, D,
+            bs, nb, _dtype_code(key), _dtype_code(k_cache), _ptr(k_scale), _ptr(v_scale),
+            _stream(stream))
+
+
 def paged_kv_append(key, value, k_cache, v_cache, slot_mapping, *, k_scale=None, v_scale=None,
                     stream=None) -> None:
     """Write key/value [T, Hkv, D] into the pool [num_blocks, bs, Hkv, D] at
     slot_mapping [T] (int64); see paged_kv_append in include/pagedkv.h."""
-    lib = load_library()
-    T, Hkv, D = key.shape
-    nb, bs = k_cache.shape[0], k_cache.shape[1]
-    st = lib.paged_kv_append(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
-                             _ptr(slot_mapping), T, Hkv, D, bs, nb, _dtype_code(key),
-                             _dtype_code(k_cache), _ptr(k_scale), _ptr(v_scale), _stream(stream))
+    st = load_library().paged_kv_append(*append_args(key, value, k_cache, v_cache, slot_mapping,
+                                                     k_scale=k_scale, v_scale=v_scale,
+                                                     stream=stream))
     if st != 0:
         raise PagedKVError("paged_kv_append", st)
 
@@ -198,22 +207,31 @@ def paged_attention_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, 
                                                          head_dim, max_seq_len, partition_size)
 
 
+def decode_args(out, query, k_cache, v_cache, block_table, seq_lens, *, max_seq_len, scale,
+                partition_size=0, workspace=None, k_scale=None, v_scale=None, max_ctas=0,
+                flags=0, stream=None) -> tuple:
+    """The arguments of the C call paged_attention_decode for these tensors, in
+    its order (see append_args)."""
+    S, Hq, D = query.shape
+    nb, bs, Hkv, _ = k_cache.shape
+    mbps = block_table.shape[1]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return (_ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+            _ptr(seq_lens), S, Hq, Hkv, D, bs, mbps, nb, int(max_seq_len), float(scale),
+            _dtype_code(query), _dtype_code(k_cache), _ptr(k_scale), _ptr(v_scale),
+            int(partition_size), int(max_ctas), int(flags), _ptr(workspace), ws_bytes,
+            _stream(stream))
+
+
 def paged_attention_decode(out, query, k_cache, v_cache, block_table, seq_lens, *, max_seq_len,
                            scale, partition_size=0, workspace=None, k_scale=None, v_scale=None,
                            max_ctas=0, flags=0, stream=None) -> None:
     """out[i, j] = softmax attention of query[i, j] over sequence i's paged K/V;
     see paged_attention_decode in include/pagedkv.h."""
-    lib = load_library()
-    S, Hq, D = query.shape
-    nb, bs, Hkv, _ = k_cache.shape
-    mbps = block_table.shape[1]
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.paged_attention_decode(_ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache),
-                                    _ptr(block_table), _ptr(seq_lens), S, Hq, Hkv, D, bs, mbps,
-                                    nb, int(max_seq_len), float(scale), _dtype_code(query),
-                                    _dtype_code(k_cache), _ptr(k_scale), _ptr(v_scale),
-                                    int(partition_size), int(max_ctas), int(flags),
-                                    _ptr(workspace), ws_bytes, _stream(stream))
+    st = load_library().paged_attention_decode(*decode_args(
+        out, query, k_cache, v_cache, block_table, seq_lens, max_seq_len=max_seq_len, scale=scale,
+        partition_size=partition_size, workspace=workspace, k_scale=k_scale, v_scale=v_scale,
+        max_ctas=max_ctas, flags=flags, stream=stream))
     if st != 0:
         raise PagedKVError("paged_attention_decode", st)
 

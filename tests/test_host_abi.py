@@ -202,3 +202,26 @@ def test_decode_rejects_unknown_flags(lib):
     assert decode(lib, flags=32) == ESHAPE
     assert decode(lib, flags=1 << 31) == ESHAPE
     assert decode(lib, flags=8 | 16) == ESHAPE          # tensor cores and CUDA cores at once
+
+
+def test_marshalled_argument_lists_match_the_c_signatures(lib):
+    """append_args / decode_args give one value per C parameter, each one its
+    declared ctypes type accepts, with the sizes in their places; a decode call
+    made with them on an empty batch succeeds without touching the GPU."""
+    import torch
+    import paged_kv_cache_367_b200 as pkv
+    key = torch.zeros(3, 2, 64, dtype=torch.bfloat16)
+    pool = torch.zeros(4, 16, 2, 64, dtype=torch.bfloat16)
+    slots = torch.full((3,), -1, dtype=torch.int64)
+    a = pkv.append_args(key, key, pool, pool, slots, stream=0)
+    assert len(a) == len(lib.paged_kv_append.argtypes)
+    conv = [t(x) for t, x in zip(lib.paged_kv_append.argtypes, a)]
+    assert [c.value for c in conv[5:10]] == [3, 2, 64, 16, 4]
+    q = torch.zeros(0, 4, 64, dtype=torch.bfloat16)
+    bt = torch.zeros(0, 1, dtype=torch.int32)
+    ln = torch.zeros(0, dtype=torch.int32)
+    d = pkv.decode_args(q, q, pool, pool, bt, ln, max_seq_len=0, scale=0.125, stream=0)
+    assert len(d) == len(lib.paged_attention_decode.argtypes)
+    conv = [t(x) for t, x in zip(lib.paged_attention_decode.argtypes, d)]
+    assert [c.value for c in conv[6:13]] == [0, 4, 2, 64, 16, 1, 4]
+    assert lib.paged_attention_decode(*conv) == OK
