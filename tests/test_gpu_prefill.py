@@ -208,8 +208,8 @@ def test_block_ids_outside_the_pool_read_as_zeros(cuda_dev, flags):
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (32, 8), (16, 1), (12, 2)])
 @pytest.mark.parametrize("D", [64, 128])
 def test_prefill_fp8_cache_parity(cuda_dev, case, Hq, Hkv, D):
-    # E4M3 caches: codes widened in registers, k_scale folded into the scores,
-    # v_scale into the output; the tcgen05 flag has no effect on this path.
+    # E4M3 caches on the tcgen05 kernel: codes widened to f16 in shared memory,
+    # k_scale folded into the scores, v_scale into the output.
     lens, qlens = CASES[case]
     c = make_case(lens, qlens, Hq, Hkv, D, 16, "bf16", cuda_dev, seed=Hq + D, cache="e4m3")
     check(run_gpu(c), run_oracle(c), "e4m3")
@@ -218,10 +218,13 @@ def test_prefill_fp8_cache_parity(cuda_dev, case, Hq, Hkv, D):
 @pytest.mark.parametrize("bs", [8, 16, 32])
 @pytest.mark.parametrize("dt", ["bf16", "f16"])
 @pytest.mark.parametrize("D", [64, 128])
-def test_prefill_fp8_cache_blocks_dtypes(cuda_dev, bs, dt, D):
+@pytest.mark.parametrize("flags", KERNELS)
+def test_prefill_fp8_cache_blocks_dtypes(cuda_dev, bs, dt, D, flags):
+    # Both kernels over an E4M3 cache: tcgen05 (codes widened in shared memory)
+    # and mma.sync (codes widened in registers).
     c = make_case([400, 90, 33], [200, 90, 5], 16, 4, D, bs, dt, cuda_dev, seed=D + bs + 1,
                   cache="e4m3")
-    check(run_gpu(c, flags=pkv.PKV_PREFILL_MMA_SYNC), run_oracle(c), "e4m3")
+    check(run_gpu(c, flags=flags), run_oracle(c), "e4m3")
 
 
 def test_prefill_fp8_out_of_pool_and_prefix_hit_matches_decode(cuda_dev):
@@ -330,3 +333,42 @@ def test_prefill_many_one_chunk_items(cuda_dev):
     qlens = [int(min(L, q)) for L, q in zip(lens, rng.integers(1, 4, size=300))]
     c = make_case(lens, qlens, 32, 8, 128, 16, "bf16", cuda_dev, seed=9)
     check(run_gpu(c), run_oracle(c), "bf16")
+
+
+BENCH_SHAPES = {  # the prefill workloads bench.py times: 64 query / 8 KV heads, D 128, block 16
+    "1024-token chunks after 2048 cached": ([3072] * 8, [1024] * 8),
+    "4096-token prompts": ([4096] * 4, [4096] * 4),
+    "512-token prompts": ([512] * 16, [512] * 16),
+}
+
+
+@pytest.mark.parametrize("shape", list(BENCH_SHAPES))
+@pytest.mark.parametrize("cache", ["bf16", "e4m3"])
+def test_prefill_bench_workloads_at_full_size_sampled(cuda_dev, shape, cache):
+    # The workloads the benchmark times, at their full sizes, on the default
+    # kernel as it launches there; the fp64 oracle computes 1,536 sampled
+    # (row, query head) outputs: the first and last rows of every chunk and of
+    # every 256-row item boundary in the first sequence, and random ones.
+    lens, qlens = BENCH_SHAPES[shape]
+    c = make_case(lens, qlens, 64, 8, 128, 16, "bf16", cuda_dev, seed=len(lens),
+                  cache=None if cache == "bf16" else cache)
+    got = run_gpu(c)
+    T = int(c["qs"][-1])
+    rng = np.random.default_rng(5)
+    rows = set(int(x) for x in c["qs"][:-1]) | set(int(x) - 1 for x in c["qs"][1:])
+    rows |= set(range(0, min(T, qlens[0]), 32)) | set(range(31, min(T, qlens[0]), 32))
+    rows = sorted(rows)
+    items = [(r, int(h)) for r in rows for h in rng.choice(64, 2, replace=False)]
+    items += [(int(r), int(h)) for r, h in zip(rng.integers(0, T, 1536 - len(items)),
+                                                rng.integers(0, 64, 1536 - len(items)))]
+    items = np.asarray(items[:1536], np.int32)
+    want, _ = oracle.prefill(W.host(c["q"]), W.host(c["kc"]), W.host(c["vc"]), c["bt"],
+                             c["lens"], c["qs"], num_heads=64, num_kv_heads=8, head_dim=128,
+                             block_size=16, scale=128 ** -0.5, q_dtype="bf16",
+                             cache_dtype=c["cache"], k_scale=c["sc"], v_scale=c["sc"],
+                             items=items)
+    g = got[items[:, 0], items[:, 1]].float().cpu().numpy().astype(np.float64)
+    err = np.abs(g - want)
+    tol = TOL["e4m3" if cache == "e4m3" else "bf16"]
+    assert np.all(np.isfinite(g))
+    assert err.max() <= tol[0] and err.mean() <= tol[1], (err.max(), err.mean())
