@@ -239,8 +239,8 @@ int paged_attention_decode_static(void* out, const void* query, const void* k_ca
  * p < 0 gets zeros. max_q_len must be >= every q_i: a longer chunk has only its
  * last max_q_len rows computed. Lengths are clamped to max_blocks_per_seq *
  * block_size and query_start to [0, num_q_tokens]. head_dim 64 or 128,
- * block_size 8/16/32. With a 16-bit cache the default kernel runs on the
- * tcgen05 tensor cores with tensor-memory accumulators: a persistent kernel,
+ * block_size 8/16/32. The default kernel (16-bit and FP8-E4M3 caches) runs on
+ * the tcgen05 tensor cores with tensor-memory accumulators: a persistent kernel,
  * one CTA per SM taking items of 256 query rows (two tiles) from a work counter
  * in device memory. Each call takes the next of 64 such counters (the call's
  * last CTA resets it), so up to 64 prefill calls may be in flight at once, on
