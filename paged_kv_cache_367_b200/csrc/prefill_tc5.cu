@@ -385,7 +385,9 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
 // QT: Q is copied by TMA (g divides 128, so a tile's rows are whole tokens);
 // otherwise the softmax threads copy their rows.
 // OT: query/output type. F8: the cache holds E4M3 codes, widened to f16 in
-// shared memory by the producer; Q is rounded to f16 (the MMAs are f16).
+// shared memory by the producer and the widening warp; a bf16 Q is rounded to
+// f16 (the MMAs are f16): in place by the tile's MMA warp when it came by TMA,
+// by the softmax threads as they stage it otherwise.
 template <typename OT, int D, bool QT, bool F8>
 __global__ void __launch_bounds__(F8 ? kThreads8 : kThreads, 1)
     prefill_tc5_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmap_k,
@@ -734,6 +736,20 @@ __global__ void __launch_bounds__(F8 ? kThreads8 : kThreads, 1)
       if (sn.c == 0) {  // the first S of an item: its Q must be staged
         if (!wait_warp(q_full + t, (uint32_t)q_items & 1u)) return false;
         ++q_items;
+        if constexpr (F8 && QT && !std::is_same<OT, __half>::value) {
+          // The tile's Q came by TMA as bf16: rounded to f16 in place for the
+          // f16 MMAs (every 16-bit element on its own, so the swizzle does not
+          // matter); each lane fences its stores before the warp sync.
+          uint4* qb = reinterpret_cast<uint4*>(qs + t * C::kQ);
+#pragma unroll 4
+          for (int e = lane; e < C::kQ / 16; e += 32) {
+            const uint4 v = qb[e];
+            qb[e] = make_uint4(to_f16x2<OT>(v.x), to_f16x2<OT>(v.y), to_f16x2<OT>(v.z),
+                               to_f16x2<OT>(v.w));
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+        }
       }
       // K of chunk js (waited for only now, so the PV before never waits on a copy).
       if (!wait_warp(full + js % C::kNSx, (uint32_t)(js / C::kNSx) & 1u)) return false;
@@ -1116,11 +1132,12 @@ bool encode_q_map(CUtensorMap* map, const PrefillParams& p, int head_dim, bool b
 template <typename OT, int D>
 cudaError_t launch5q(const PrefillParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
                      bool f8, int num_seqs, cudaStream_t stream) {
-  if (f8)  // Q rounded to f16 by the softmax threads
-    return launch5<OT, D, false, true>(p, mk, mv, mk, num_seqs, stream);  // mk unused as Q map
   CUtensorMap mq;
-  if (encode_q_map(&mq, p, D, std::is_same<OT, __nv_bfloat16>::value))
-    return launch5<OT, D, true, false>(p, mk, mv, mq, num_seqs, stream);
+  const bool qt = encode_q_map(&mq, p, D, std::is_same<OT, __nv_bfloat16>::value);
+  if (f8)  // a bf16 Q is rounded to f16, in place, for the f16 MMAs
+    return qt ? launch5<OT, D, true, true>(p, mk, mv, mq, num_seqs, stream)
+              : launch5<OT, D, false, true>(p, mk, mv, mk, num_seqs, stream);  // mk: no Q map
+  if (qt) return launch5<OT, D, true, false>(p, mk, mv, mq, num_seqs, stream);
   return launch5<OT, D, false, false>(p, mk, mv, mk, num_seqs, stream);  // mk unused as Q map
 }
 
