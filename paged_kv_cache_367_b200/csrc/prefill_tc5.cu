@@ -858,6 +858,8 @@ __global__ void __launch_bounds__(F8 ? kThreads8 : kThreads, 1)
     // overlaps useful work, and the next item's first PV, which overwrites O,
     // cannot start before O has been read.
     bool pending = false, prev_valid = false;
+    // Output rows are D * 2 bytes: all 32-byte aligned when the output is.
+    const bool out32 = !F8 && (reinterpret_cast<uintptr_t>(p.out) & 31u) == 0;
     uint64_t prev_lsum = 0;
     OT* prev_dst = nullptr;
     auto epilogue = [&]() -> bool {
@@ -875,7 +877,25 @@ __global__ void __launch_bounds__(F8 ? kThreads8 : kThreads, 1)
       for (int q = 0; q < D / 64; ++q) {
         float o[64];
         tmem_ld64(tO + 64 * q, o);  // two loads in flight, one wait
-        if (prev_valid) {
+        if (!F8 && prev_valid && out32) {
+          // 16-bit caches: 32 bytes (a whole sector) per store when the output
+          // is 32-byte aligned; sixteen-byte stores left each sector half
+          // written by two instructions (the E4M3 form keeps them: measured
+          // faster there)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint32_t wv[8];
+            float a, b;
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              wv[k] = Mma<OT>::pack(o[16 * u + 2 * k] * inv, o[16 * u + 2 * k + 1] * inv, a, b);
+            asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(
+                             prev_dst + 64 * q + 16 * u),
+                         "r"(wv[0]), "r"(wv[1]), "r"(wv[2]), "r"(wv[3]), "r"(wv[4]), "r"(wv[5]),
+                         "r"(wv[6]), "r"(wv[7])
+                         : "memory");
+          }
+        } else if (prev_valid) {
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             uint4 wv;

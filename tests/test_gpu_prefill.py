@@ -372,3 +372,23 @@ def test_prefill_bench_workloads_at_full_size_sampled(cuda_dev, shape, cache):
     tol = TOL["e4m3" if cache == "e4m3" else "bf16"]
     assert np.all(np.isfinite(g))
     assert err.max() <= tol[0] and err.mean() <= tol[1], (err.max(), err.mean())
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_prefill_output_only_16_byte_aligned(cuda_dev, D):
+    # The epilogue stores 32 bytes at a time when the output is 32-byte aligned
+    # and 16 at a time otherwise: an output 16 bytes past an aligned allocation
+    # takes the second path.
+    c = make_case([400, 90, 33], [200, 90, 5], 16, 4, D, 16, "bf16", cuda_dev, seed=D + 3)
+    n = int(c["q"].numel())
+    buf = torch.full((n + 8,), float("nan"), dtype=c["q"].dtype, device=cuda_dev)
+    out = buf[8:].view(c["q"].shape)
+    assert out.data_ptr() % 32 == 16
+    pkv.paged_attention_prefill(out, c["q"], c["kc"], c["vc"], torch.from_numpy(c["bt"]).to(cuda_dev),
+                                torch.from_numpy(c["lens"]).to(cuda_dev),
+                                torch.from_numpy(c["qs"]).to(cuda_dev),
+                                max_q_len=int(np.diff(c["qs"]).max()), scale=D ** -0.5)
+    torch.cuda.synchronize()
+    assert pkv.pkv_device_status(clear=True) == 0
+    assert torch.isnan(buf[:8].float()).all()  # nothing written before the output
+    check(out, run_oracle(c), "bf16")
