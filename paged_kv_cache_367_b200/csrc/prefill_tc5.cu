@@ -991,6 +991,8 @@ __global__ void __launch_bounds__(F8 ? kThreads8 : kThreads, 1)
         if (raise) m_use = mx;
         const float msub = m_use == -INFINITY ? 0.f : m_use;
         uint32_t pk[32];
+        float ls0, ls1;  // the two halves of the row sums, for the 16-bit adds below
+        asm("mov.b64 {%0, %1}, %2;" : "=f"(ls0), "=f"(ls1) : "l"(lsum2));
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           float x0, x1;  // s * scale - m for a pair, as one packed f32x2 FMA
@@ -1014,12 +1016,25 @@ __global__ void __launch_bounds__(F8 ? kThreads8 : kThreads, 1)
           } else {
             pk[i] = Mma<T>::pack(fast_exp2(x0), fast_exp2(x1), lo, hi);
           }
-          {
+          if constexpr (F8) {
             uint64_t pp;
             asm("mov.b64 %0, {%1, %2};" : "=l"(pp) : "f"(lo), "f"(hi));
             asm("add.rn.f32x2 %0, %0, %1;" : "+l"(lsum2) : "l"(pp));
+          } else {
+            // The rounded pair added to the sums as it is: each 16-bit value is
+            // converted exactly and added in fp32 by one instruction (sm_100's
+            // mixed-precision add), where unpacking the pair first took three.
+            (void)lo;
+            (void)hi;
+            if constexpr (std::is_same<T, __nv_bfloat16>::value)
+              asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n add.rn.f32.bf16 %0, l, %0;\n"
+                  " add.rn.f32.bf16 %1, h, %1;\n}" : "+f"(ls0), "+f"(ls1) : "r"(pk[i]));
+            else
+              asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n add.rn.f32.f16 %0, l, %0;\n"
+                  " add.rn.f32.f16 %1, h, %1;\n}" : "+f"(ls0), "+f"(ls1) : "r"(pk[i]));
           }
         }
+        if constexpr (!F8) asm("mov.b64 %0, {%1, %2};" : "=l"(lsum2) : "f"(ls0), "f"(ls1));
         if (c == nchunks - 1 && c0 + kChunk > kv_end) {
           // Zero V rows past the range (stale or poisoned) before this tile's
           // last PV. Both tiles do it, as their PVs are issued independently
