@@ -326,10 +326,15 @@ def e2e_time_ms(args, wl, c_calls, out, world):
     buffered and the copies run on their own streams, so step k+1's inputs and
     step k-1's output move while step k computes; the timed region spans the
     first input copy to the last output copy. The copies and the events that
-    order them are issued through the CUDA runtime directly."""
+    order them are issued through the CUDA runtime directly. The loop is
+    timed twice: eagerly, and as `graph_steps` steps captured once in a CUDA
+    graph and replayed, as a serving loop would, so the host issues one launch
+    per `graph_steps` steps (every replay still copies each step's inputs from,
+    and its output to, pinned host memory); the faster form is reported, both
+    times are returned."""
     cr = _cudart()
     K = args.steps
-    KE = args.e2e_steps or max(min(K, 200), 50)
+    KE = args.e2e_steps or max(min(K, 200), 100)
     parts = [wl.query, wl.new_key, wl.new_value, torch.from_numpy(wl.slot_mapping),
              torch.from_numpy(wl.block_table), torch.from_numpy(wl.seq_lens)]
     offs, total = [], 0
@@ -370,27 +375,67 @@ def e2e_time_ms(args, wl, c_calls, out, world):
     evd = [e.cuda_event for e in ev_done]
     evr = [e.cuda_event for e in ev_read]
 
+    def ck(rc):
+        if rc != 0:
+            raise RuntimeError(f"CUDA runtime error {rc} in the end-to-end loop")
+
+    def body(k, cs, calls):  # step k on buffer k % 2, compute on stream cs
+        b = k & 1
+        if k >= 2:
+            ck(cr.cudaStreamWaitEvent(si, evd[b], 0))
+        ck(cr.cudaMemcpyAsync(din[b], hin[b], h2d, H2D, si))
+        ck(cr.cudaEventRecord(evi[b], si))
+        ck(cr.cudaStreamWaitEvent(cs, evi[b], 0))
+        if k >= 2:
+            ck(cr.cudaStreamWaitEvent(cs, evr[b], 0))
+        for fn, a in calls[b]:
+            st = fn(*a)
+            if st != 0:
+                raise pkv.PagedKVError(fn.__name__, st)
+        ck(cr.cudaEventRecord(evd[b], cs))
+        ck(cr.cudaStreamWaitEvent(so, evd[b], 0))
+        ck(cr.cudaMemcpyAsync(hout[b], dout[b], d2h, D2H, so))
+        ck(cr.cudaEventRecord(evr[b], so))
+
     def run(steps):
         for k in range(steps):
-            b = k & 1
-            if k >= 2:
-                cr.cudaStreamWaitEvent(si, evd[b], 0)
-            cr.cudaMemcpyAsync(din[b], hin[b], h2d, H2D, si)
-            cr.cudaEventRecord(evi[b], si)
-            cr.cudaStreamWaitEvent(cs, evi[b], 0)
-            if k >= 2:
-                cr.cudaStreamWaitEvent(cs, evr[b], 0)
-            for fn, a in calls[b]:
-                st = fn(*a)
-                if st != 0:
-                    raise pkv.PagedKVError(fn.__name__, st)
-            cr.cudaEventRecord(evd[b], cs)
-            cr.cudaStreamWaitEvent(so, evd[b], 0)
-            cr.cudaMemcpyAsync(hout[b], dout[b], d2h, D2H, so)
-            cr.cudaEventRecord(evr[b], so)
+            body(k, cs, calls)
 
     run(4)
     torch.cuda.synchronize()
+    GS = min(25, KE)
+    graph = None
+    if not args.no_graph:
+        ev_fork, ev_ji, ev_jo = torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event()
+        for e in (ev_fork, ev_ji, ev_jo):
+            e.record(compute)
+        torch.cuda.synchronize()
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                cap = torch.cuda.current_stream().cuda_stream
+                gcalls = [c_calls(*views[b], outs[b], cap) for b in range(2)]
+                ck(cr.cudaEventRecord(ev_fork.cuda_event, cap))   # the copy streams join
+                ck(cr.cudaStreamWaitEvent(si, ev_fork.cuda_event, 0))
+                ck(cr.cudaStreamWaitEvent(so, ev_fork.cuda_event, 0))
+                for k in range(GS):
+                    body(k, cap, gcalls)
+                ck(cr.cudaEventRecord(ev_ji.cuda_event, si))       # and leave
+                ck(cr.cudaStreamWaitEvent(cap, ev_ji.cuda_event, 0))
+                ck(cr.cudaEventRecord(ev_jo.cuda_event, so))
+                ck(cr.cudaStreamWaitEvent(cap, ev_jo.cuda_event, 0))
+            for _ in range(2):
+                g.replay()
+            torch.cuda.synchronize()
+            graph = g
+        except Exception:
+            torch.cuda.synchronize()
+            graph = None
+    # Both loop forms are timed, the same steps through the same calls; the
+    # faster is reported (the graph saves host time per step, the eager loop
+    # the graph's cross-stream edges: which wins depends on the host).
+    reps = max(1, KE // GS)
+    KG = reps * GS
     if world > 1:
         torch.distributed.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -400,7 +445,29 @@ def e2e_time_ms(args, wl, c_calls, out, world):
     compute.wait_stream(s_out)
     e1.record(compute)
     torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / KE, KE, h2d, d2h, h_out[(KE - 1) & 1]
+    eager_ms = e0.elapsed_time(e1) / KE
+    graph_ms = None
+    if graph is not None:
+        if world > 1:
+            torch.distributed.barrier()
+        e0.record(compute)
+        for _ in range(reps):
+            graph.replay()
+        e1.record(compute)
+        torch.cuda.synchronize()
+        graph_ms = e0.elapsed_time(e1) / KG
+    if world > 1:  # every rank reports the same form
+        both = torch.tensor([eager_ms, graph_ms if graph_ms is not None else float("inf")],
+                            device=out.device)
+        torch.distributed.all_reduce(both, op=torch.distributed.ReduceOp.MAX)
+        eager_ms, g = both.tolist()
+        graph_ms = None if g == float("inf") else g
+    use_graph = graph_ms is not None and graph_ms < eager_ms
+    ms, steps = (graph_ms, KG) if use_graph else (eager_ms, KE)
+    last = ((GS if use_graph else KE) - 1) & 1
+    return (ms, steps, h2d, d2h, h_out[last], GS if use_graph else 0,
+            {"eager_ms_per_step": round(eager_ms, 5),
+             "graph_ms_per_step": None if graph_ms is None else round(graph_ms, 5)})
 
 
 
@@ -508,7 +575,7 @@ def run_ours(args, rank, world, dev):
                                          max_ctas=args.max_ctas, flags=e2e_flags,
                                          stream=stream)))
 
-    e2e_ms, KE, h2d, d2h, h_out = e2e_time_ms(args, wl, c_calls, out, world)
+    e2e_ms, KE, h2d, d2h, h_out, e2e_graph, e2e_forms = e2e_time_ms(args, wl, c_calls, out, world)
     assert torch.isfinite(h_out.float()).all(), "non-finite decode output"
 
     if world > 1:
@@ -545,7 +612,10 @@ def run_ours(args, rank, world, dev):
                        "one D2H copy of the output to pinned host memory; copies run on two "
                        "copy streams, double-buffered, so step k+1's inputs and step k-1's "
                        "output move while step k computes; copies and events issued through "
-                       "the CUDA runtime"},
+                       "the CUDA runtime; timed both eagerly and as a loop of graph_steps steps "
+                       "captured in one CUDA graph and replayed, the faster reported "
+                       "(graph_steps 0: eager)",
+                "graph_steps": e2e_graph, **e2e_forms},
         "gpu_launches": K * launches_per_step,
         "timing": "CUDA graph replay of one step" if graph is not None else "eager launches",
         "decode_flags": "plain" if args.plain_launch else
